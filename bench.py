@@ -1,0 +1,405 @@
+"""Benchmark of one routed-expert MoE FFN layer with block-scaled FP4 expert
+weights on B200 (sm_100a), through the library's C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one whole layer (route -> quantise -> permute -> FC1 + SwiGLU +
+requantise -> FC2 -> combine) over one batch of T synthetic tokens.  Default
+workload: the prefill layer (T = 2048, E = 256, top-6, d = 7168, I = 2048,
+MXFP4, skewed router bias).  Under torchrun every rank runs its own replica
+on its own GPU (independent token shards, no data-path collective; weak
+scaling); the timed region is bracketed by barriers and reported as the max
+over ranks.  Prints one JSON line (rank 0).
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/s"
+UNIT = "tokens/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="prefill")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget-s", type=float, default=15.0)
+    return ap.parse_args()
+
+
+def workload_desc(wl):
+    fmt = "MXFP4" if wl.fmt == 0 else "NVFP4"
+    if wl.dense:
+        return f"dense FP4 GEMM M={wl.T} N={wl.I} K={wl.d} {fmt}"
+    bias = f", router bias N(0,{wl.bias_sigma})" if wl.bias_sigma else ""
+    return f"MoE layer T={wl.T} E={wl.E} top-{wl.k} d={wl.d} I={wl.I} {fmt}{bias}"
+
+
+# ---------------------------------------------------------------------------
+# oracle timing on the host cores (cpu_baseline leg and --impl reference)
+# ---------------------------------------------------------------------------
+_WCACHE = {}
+
+
+def oracle_sample(wl, ntok, seed=0):
+    """Times the oracle on the first `ntok` tokens of the workload: routing,
+    quantisation, permutation, FC1, SwiGLU, requantisation, FC2 and combine,
+    over the experts those tokens touch (weights quantised beforehand, not
+    timed).  Returns (seconds, tokens)."""
+    import oracle
+    import synth
+    from synth import workloads
+    lg = workloads.host_logits(wl, seed)[:ntok]
+    xb = workloads.host_x_bits(wl, seed)[:ntok]
+    x = synth.bf16_bits_to_f32(xb)
+    idx, _ = oracle.route_topk(lg, wl.k)
+    touched = np.unique(idx)
+    remap = np.full(wl.E, -1, np.int64)
+    remap[touched] = np.arange(len(touched))
+    fmt = wl.fmt
+    w1s, w2s = [], []
+    for e in touched:
+        key = (wl.name, int(e), seed)
+        if key not in _WCACHE:
+            _WCACHE[key] = (oracle.quantize(workloads.host_w1(wl, int(e), seed), fmt),
+                            oracle.quantize(workloads.host_w2(wl, int(e), seed), fmt))
+        w1s.append(_WCACHE[key][0])
+        w2s.append(_WCACHE[key][1])
+    g_h = workloads.G_H if fmt == oracle.NV else None
+    t0 = time.perf_counter()
+    idx, w = oracle.route_topk(lg, wl.k)
+    cidx = remap[idx].astype(np.int32)
+    E2 = len(touched)
+    xq = oracle.quantize(x, fmt)
+    offsets, r2s, s2r = oracle.moe_permute(cidx, E2)
+    a = oracle.gather_rows(xq, r2s, wl.k)
+    y1 = np.empty((a.data.shape[0], 2 * wl.I))
+    for j in range(E2):
+        r0, r1 = offsets[j], offsets[j + 1]
+        if r1 > r0:
+            y1[r0:r1], _ = oracle.expert_gemm_rows(a, np.arange(r0, r1), w1s[j], (0, 2 * wl.I))
+    h = oracle.swiglu(y1.astype(np.float32))
+    hq = oracle.quantize(h, fmt, g=g_h)
+    y2 = np.empty((a.data.shape[0], wl.d))
+    for j in range(E2):
+        r0, r1 = offsets[j], offsets[j + 1]
+        if r1 > r0:
+            y2[r0:r1], _ = oracle.expert_gemm_rows(hq, np.arange(r0, r1), w2s[j], (0, wl.d))
+    oracle.moe_combine(y2.astype(np.float32).astype(np.float64), s2r, w)
+    return time.perf_counter() - t0, ntok
+
+
+def cpu_cores():
+    n = os.environ.get("OMP_NUM_THREADS")
+    return int(n) if n else (os.cpu_count() or 1)
+
+
+def cpu_baseline(wl, budget_s):
+    # grow the token sample until one run takes a meaningful share of the budget
+    ntok, dt = 1, 0.0
+    while True:
+        dt, n = oracle_sample(wl, ntok)
+        if dt > budget_s / 4 or ntok >= wl.T:
+            break
+        ntok = min(wl.T, max(ntok * 2, int(ntok * budget_s / 4 / max(dt, 1e-3))))
+    return {"value": n / dt, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+            "sample": f"first {n} of {wl.T} tokens of the same workload (full layer over the experts they touch; "
+                      f"weights quantised beforehand, untimed), {dt:.2f} s"}
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.samples = []
+        self._stop = threading.Event()
+        self._t = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                out = subprocess.run(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                                      "--format=csv,noheader,nounits"], capture_output=True, text=True,
+                                     timeout=5).stdout.strip()
+                if out:
+                    self.samples.append([v.strip() for v in out.split(",")])
+            except Exception:
+                pass
+            self._stop.wait(0.2)
+
+    def __enter__(self):
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t:
+            self._t.join(timeout=10)
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        sm = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
+        smax = [float(s[2]) for s in self.samples if s[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for s in self.samples:
+            for i, nm in enumerate(names):
+                if len(s) > 5 + i and s[5 + i].lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+def algorithmic(wl, offsets):
+    """bytes and flops of one layer and of its FC1 call, from the routing"""
+    counts = np.diff(offsets)
+    touched = int((counts > 0).sum())
+    S = wl.S
+    blk = 32 if wl.fmt == 0 else 16
+    row1 = wl.d // 2 + wl.d // blk            # packed bytes + scale bytes of one K=d row
+    row2 = wl.I // 2 + wl.I // blk
+    w1_bytes = touched * 2 * wl.I * row1
+    w2_bytes = touched * wl.d * row2
+    fc1_bytes = w1_bytes + S * row1 + S * row2
+    fc1_flops = 2.0 * S * 2 * wl.I * wl.d
+    fc2_flops = 2.0 * S * wl.d * wl.I
+    layer_bytes = (wl.T * wl.d * 2 + wl.T * wl.E * 4 + wl.T * row1 + 2 * S * row1 + fc1_bytes - S * row1
+                   + w2_bytes + S * row2 + 2 * S * wl.d * 4 + wl.T * wl.d * 4)
+    return dict(touched=touched, fc1_bytes=fc1_bytes, fc1_flops=fc1_flops, layer_flops=fc1_flops + fc2_flops,
+                layer_bytes=layer_bytes, max_rows=int(counts.max()))
+
+
+def max_over_ranks(ms, world, device):
+    """the slowest rank's elapsed time (barrier-bracketed regions)"""
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def tokens_per_s(T, steps, ms, world):
+    """whole-job throughput: every rank processed T tokens per step"""
+    return world * T * steps / (ms / 1e3)
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from synth import workloads
+    import synth
+    from block_scaled_fp4_topk_b200 import ds4g
+    from block_scaled_fp4_topk_b200.layer import MoeLayer
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = workloads.WORKLOADS[args.workload]
+    assert not wl.dense, "the bench times MoE layers"
+    st = torch.cuda.current_stream()
+    w1, w2 = MoeLayer.synthetic_weights(wl.E, wl.d, wl.I, wl.fmt, device=dev)
+    layer = MoeLayer(w1, w2, wl.E, wl.k, wl.d, wl.I, wl.fmt, g_h=workloads.G_H)
+    # inputs resident in HBM (bf16 activations, fp32 logits), each rank its own token shard
+    x = torch.empty((wl.T, wl.d), dtype=torch.bfloat16, device=dev)
+    lg = torch.empty((wl.T, wl.E), dtype=torch.float32, device=dev)
+    seed = rank
+    synth.cuda_fill_normal_bf16(x.data_ptr(), x.numel(), seed, synth.STREAM_X, 1.0, 0, st.cuda_stream)
+    synth.cuda_fill_logits(lg.data_ptr(), wl.T, wl.E, seed, wl.bias_sigma, st.cuda_stream)
+    torch.cuda.synchronize()
+
+    # instrumented step: CUDA events around FC1 (the dominant kernel) on the launching stream
+    b = layer.buffers(wl.T, dev)
+
+    def step(ev=None):
+        ds4g.ds4g_route_topk(lg, layer.k, idx=b["idx"], w=b["w"])
+        ds4g.ds4g_quantize_mx(x, layer.fmt, out=b["xq"], workspace=b["qws"])
+        ds4g.ds4g_moe_permute(b["idx"], layer.E, b["xq"], offsets=b["offsets"], row_to_slot=b["r2s"],
+                              slot_to_row=b["s2r"], a_perm=b["a"], workspace=b["pws"])
+        if ev is not None:
+            ev[0].record(st)
+        ds4g.ds4g_grouped_gemm_fp4(b["a"], b["offsets"], layer.E, wl.T, layer.w1, 2 * layer.I,
+                                   ds4g.EPI_SWIGLU_REQUANT, out_q=b["hq"])
+        if ev is not None:
+            ev[1].record(st)
+        ds4g.ds4g_grouped_gemm_fp4(b["hq"], b["offsets"], layer.E, wl.T, layer.w2, layer.d, ds4g.EPI_NONE,
+                                   out=b["y2"])
+        ds4g.ds4g_moe_combine(b["y2"], b["s2r"][:wl.S], b["w"], out=b["out"])
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    ds4g.ds4g_check_device()
+    offsets = b["offsets"].cpu().numpy()
+    alg = algorithmic(wl, offsets)
+    launches_per_step = (1 + (1 if wl.fmt == 0 else 3) + 4 + 1 + 1 + 1)
+
+    fc1_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else
+                      int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local_rank])) as clk:
+        e0.record(st)
+        for i in range(args.steps):
+            step(fc1_ev[i])
+        e1.record(st)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ds4g.ds4g_check_device()
+    ms_total = e0.elapsed_time(e1)
+    fc1_ms = float(np.mean([a.elapsed_time(c) for a, c in fc1_ev]))
+    ms_total = max_over_ranks(ms_total, world, dev)
+
+    # end to end through the public API: pinned host inputs -> device, layer, result -> host
+    xh = torch.empty((wl.T, wl.d), dtype=torch.bfloat16, pin_memory=True)
+    lh = torch.empty((wl.T, wl.E), dtype=torch.float32, pin_memory=True)
+    xh.copy_(x)
+    lh.copy_(lg)
+    oh = torch.empty((wl.T, wl.d), dtype=torch.float32, pin_memory=True)
+    xd = torch.empty_like(x)
+    ld = torch.empty_like(lg)
+
+    def e2e_step():
+        xd.copy_(xh, non_blocking=True)
+        ld.copy_(lh, non_blocking=True)
+        out = layer.forward(xd, ld)
+        oh.copy_(out, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0.record(st)
+    for _ in range(args.steps):
+        e2e_step()
+    a1.record(st)
+    torch.cuda.synchronize()
+    e2e_ms = a0.elapsed_time(a1)
+    e2e_ms = max_over_ranks(e2e_ms, world, dev)
+
+    if rank != 0:
+        return None
+    import json as _json
+    peaks = {}
+    pk_path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(pk_path):
+        peaks = _json.load(open(pk_path))
+    hbm_peak = peaks.get("hbm_gbs", 6650.0)
+    bf16_peak = peaks.get("bf16_tflops", 1590.0)
+    fp4_peak = bf16_peak * 4.0          # dense FP4 : bf16 = 9 : 2.25 (nominal ratio)
+    t_hbm = alg["fc1_bytes"] / (hbm_peak * 1e9)
+    t_tc = alg["fc1_flops"] / (fp4_peak * 1e12)
+    fc1_s = fc1_ms / 1e3
+    if t_hbm >= t_tc:
+        roof = {"bound": "hbm", "achieved": alg["fc1_bytes"] / fc1_s / 1e9, "peak": hbm_peak, "unit": "GB/s"}
+    else:
+        roof = {"bound": "tensor", "achieved": alg["fc1_flops"] / fc1_s / 1e12, "peak": fp4_peak, "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = None
+    roof["kernel"] = "grouped FP4 GEMM FC1 + fused SwiGLU/requant (tcgen05)" if wl.T > 8 else "grouped FP4 GEMV FC1"
+    roof["peak_source"] = ("measured (MEASURED_PEAKS.json" + ("; FP4 = bf16 burst x 4 nominal ratio" if
+                           roof["bound"] == "tensor" else "") + ")") if peaks else "fallback"
+    roof["fc1_ms"] = fc1_ms
+    roof["fc1_tflops"] = alg["fc1_flops"] / fc1_s / 1e12
+    roof["fc1_gbs"] = alg["fc1_bytes"] / fc1_s / 1e9
+    roof["algorithmic_bytes"] = alg["fc1_bytes"]
+    roof["algorithmic_flops"] = alg["fc1_flops"]
+
+    ms_step = ms_total / args.steps
+    value = tokens_per_s(wl.T, args.steps, ms_total, world)
+    e2e_value = tokens_per_s(wl.T, args.steps, e2e_ms, world)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "mxfp4" if wl.fmt == 0 else "nvfp4", "data": "synthetic",
+        "config": {"workload": workload_desc(wl), "tokens_per_gpu": wl.T, "experts_touched": alg["touched"],
+                   "max_rows_per_expert": alg["max_rows"], "parallelism": f"replicas x{world} (token shards)",
+                   "l2": f"no flush: the step's working set (~{alg['layer_bytes'] / 1e9:.2f} GB) exceeds the "
+                         f"126 MB L2", "layer_tflops": alg["layer_flops"] / (ms_step / 1e3) / 1e12},
+        "roofline": roof,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": wl.T * wl.d * 2 + wl.T * wl.E * 4,
+                "d2h_bytes_per_step": wl.T * wl.d * 4},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+    }
+    return line
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    from synth import workloads
+    wl = workloads.WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        for _ in range(args.warmup):
+            oracle_sample(wl, 1)
+        tot_t, tot_n = 0.0, 0
+        ntok = 2 if wl.T >= 2 else 1
+        for _ in range(args.steps):
+            dt, n = oracle_sample(wl, ntok)
+            tot_t += dt
+            tot_n += n
+        v = tot_n / tot_t
+        print(json.dumps({
+            "impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": workload_desc(wl)},
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+                             "sample": f"each step: the first {ntok} tokens of the workload (full layer over the "
+                                       f"experts they touch)"},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }), flush=True)
+        return 0
+
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+        from datetime import timedelta
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    line = run_ours(args, rank, world, local_rank)
+    if rank == 0:
+        if not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(wl, args.cpu_budget_s)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,636 @@
+// gemm_tc.cu -- prefill-sized grouped block-scaled FP4 GEMM on the 5th
+// generation tensor cores (tcgen05), sm_100a.
+//
+// What it computes: "DGX Spark native FP4 matrix instructions: how DwarfStar
+// uses Blackwell", sec. 1-2 (one block-scaled FP4 MMA consumes E2M1 operands
+// and their UE8M0 / UE4M3 block scales directly, no dequantisation) and the
+// grouped "contiguous" GEMM of "[DeepSeek V4] Triton FP4 optimisation in
+// practice", "Step 0" (each expert's rows form one segment).  The page's
+// kernel is the warp-level mma.sync m16n8k64 form of sm_12x; on sm_100a the
+// same math is tcgen05.mma kind::mxf4 (.block32, UE8M0) / kind::mxf4nvf4
+// (.block16, UE4M3) with the accumulator in tensor memory.
+//
+// Design (one persistent CTA per SM, 256 threads, warp-specialised):
+//   warp 0  TMA producer: packed FP4 tiles of A (128 rows x 256 K) and W
+//           (256 rows x 256 K) -> 128B-swizzled shared memory, 4 stages
+//   warp 1  MMA issuer: scale factors shared -> TMEM with tcgen05.cp
+//           (32x128b.warpx4), 4 x tcgen05.mma (M128 N256 K64) per stage,
+//           tcgen05.commit releases the stage / publishes the accumulator
+//   warp 2  scale-factor loader: cp.async of the row-major scale bytes into
+//           the 32-line x 16-byte chunk order tcgen05.cp expects
+//   warp 3  TMEM allocator
+//   warps 4-7  epilogue: tcgen05.ld of the fp32 accumulator (thread i owns
+//           tile row i), then either the fp32 store or SwiGLU + requantise
+// Tiles (expert, n-tile, m-tile) are enumerated on the device from the
+// expert offsets (no host read-back); every CTA walks tile t, t + #CTAs, ...
+// Every mbarrier wait is bounded: past ~4 s it records kErrWaitTimeout in
+// the device error word and the CTA winds down.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace ds4g {
+
+namespace tc {
+
+constexpr int BM = 128;            // tile rows (tokens)
+constexpr int BN = 256;            // tile columns (weight rows)
+constexpr int BKB = 128;           // bytes of K per stage per row (256 FP4)
+constexpr int BK = 256;            // K elements per stage
+constexpr int STAGES = 4;
+constexpr int kThreads = 256;
+constexpr int A_BYTES = BM * BKB;  // 16 KB
+constexpr int B_BYTES = BN * BKB;  // 32 KB
+constexpr int kTmemCols = 512;
+constexpr int kColAcc = 0;
+constexpr int kColSFA = 256;
+constexpr int kColSFB = 272;
+constexpr int kMaxE = 1024;
+constexpr int kSfLag = 2;          // stages the SF loader keeps in flight
+constexpr unsigned long long kWaitNs = 4000000000ull;
+
+template <int FMT>
+struct Cfg {
+    static constexpr int WORDS = (FMT == DS4G_MXFP4) ? 2 : 4;   // 4-scale words per row per stage
+    static constexpr int SFA_BYTES = WORDS * 512;
+    static constexpr int SFB_BYTES = WORDS * 1024;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+    static constexpr int K_PER_WORD = (FMT == DS4G_MXFP4) ? 128 : 64;
+    static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + 256 + (kMaxE + 1) * 4;
+};
+
+// ---- PTX wrappers ----------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ uint64_t globaltimer()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t a, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(a), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_tx(uint32_t a, uint32_t tx)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(a), "r"(tx) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t a)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(a) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint32_t a, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(a), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// bounded wait; false when it gave up (or another role already gave up)
+__device__ __forceinline__ bool mbar_wait(uint32_t a, uint32_t parity, volatile int* abort_flag)
+{
+    if (mbar_try(a, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try(a, parity)) return true;
+        if ((it & 255u) == 0) {
+            if (*abort_flag) return false;
+            if (globaltimer() - t0 > kWaitNs) {
+                *abort_flag = 1;
+                raise_error(kErrWaitTimeout);
+                return false;
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void fence_barrier_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t mbar, int x, int y)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
+        ::"r"(dst), "l"((uint64_t)map), "r"(mbar), "r"(x), "r"(y)
+        : "memory");
+}
+
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src, uint32_t src_size)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(src_size) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// shared-memory matrix descriptor (tcgen05): K-major, 128-byte swizzle,
+// 8-row core groups 1024 bytes apart
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr)
+{
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFF);
+    d |= (uint64_t)(1024 >> 4) << 32;     // stride byte offset
+    d |= (uint64_t)1 << 46;               // descriptor version (sm_100)
+    d |= (uint64_t)2 << 61;               // SWIZZLE_128B
+    return d;
+}
+
+// descriptor of one 32 x 16-byte scale-factor chunk (no swizzle, 8-row core
+// matrices 128 bytes apart)
+__device__ __forceinline__ uint64_t desc_sf(uint32_t saddr)
+{
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFF);
+    d |= (uint64_t)(128 >> 4) << 32;
+    d |= (uint64_t)1 << 46;
+    return d;
+}
+
+// instruction descriptor: E2M1 x E2M1, fp32 accumulate, K-major A and B,
+// N = 256, M = 128; scale format UE8M0 (MX) or UE4M3 (NV)
+template <int FMT>
+__device__ __forceinline__ uint32_t idesc_base()
+{
+    return (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((FMT == DS4G_MXFP4 ? 1u : 0u) << 23) |
+           ((uint32_t)(BM >> 4) << 24);
+}
+
+template <int FMT>
+__device__ __forceinline__ void mma(uint32_t d_tmem, uint64_t ad, uint64_t bd, uint32_t idesc, uint32_t acc,
+                                    uint32_t sfa, uint32_t sfb)
+{
+    if (FMT == DS4G_MXFP4) {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+            ::"r"(d_tmem), "l"(ad), "l"(bd), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb)
+            : "memory");
+    } else {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+            ::"r"(d_tmem), "l"(ad), "l"(bd), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb)
+            : "memory");
+    }
+}
+
+__device__ __forceinline__ void utccp(uint32_t taddr, uint64_t sdesc)
+{
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+__device__ __forceinline__ void tc_commit(uint32_t mbar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(mbar)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v)
+{
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// ---- tile enumeration --------------------------------------------------------
+struct Tile {
+    int e;        // expert
+    int nt;       // column tile
+    int64_t m0;   // first row of the tile
+    int64_t end;  // end of the expert's segment
+};
+
+__device__ __forceinline__ Tile tile_of(int64_t t, const int32_t* prefix, const int32_t* offsets, int E,
+                                        int n_tiles)
+{
+    int lo = 0, hi = E - 1;   // largest e with prefix[e] <= t (prefix non-decreasing)
+    while (lo < hi) {
+        int mid = (lo + hi + 1) >> 1;
+        if (prefix[mid] <= t) lo = mid; else hi = mid - 1;
+    }
+    Tile r;
+    r.e = lo;
+    const int64_t beg = offsets[lo];
+    r.end = offsets[lo + 1];
+    const int64_t mt_cnt = ceil_div(r.end - beg, BM);
+    const int64_t local = t - prefix[lo];
+    r.nt = (int)(local / mt_cnt);
+    r.m0 = beg + (local % mt_cnt) * BM;
+    return r;
+}
+
+template <int FMT, int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b, const GemmArgs p)
+{
+    using C = Cfg<FMT>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = sA + STAGES * A_BYTES;
+    uint8_t* sSFA = sB + STAGES * B_BYTES;
+    uint8_t* sSFB = sSFA + STAGES * C::SFA_BYTES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sSFB + STAGES * C::SFB_BYTES);
+    uint64_t* full = bars;                    // [STAGES]
+    uint64_t* empty = bars + STAGES;          // [STAGES]
+    uint64_t* tmem_full = bars + 2 * STAGES;
+    uint64_t* tmem_empty = tmem_full + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tmem_empty + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    int32_t* total_tiles = reinterpret_cast<int32_t*>(tmem_slot + 2);
+    int32_t* prefix = reinterpret_cast<int32_t*>(smem + STAGES * C::STAGE_BYTES + 256);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int E = p.E;
+    const int64_t K = p.K;
+    const int nks = (int)ceil_div(K, BK);
+    const int I = p.N / 2;
+    const int n_tiles = (EPI == DS4G_EPI_SWIGLU_REQUANT) ? (I / 128) : (p.N / BN);
+
+    // ---- prologue
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(smem_u32(&full[s]), 2);
+            mbar_init(smem_u32(&empty[s]), 1);
+        }
+        mbar_init(smem_u32(tmem_full), 1);
+        mbar_init(smem_u32(tmem_empty), 128);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        // tiles per expert, exclusive scan by one warp
+        const int per = (E + 31) / 32;
+        int32_t local[32];
+        int32_t sum = 0;
+        for (int i = 0; i < per; ++i) {
+            const int e = lane * per + i;
+            int32_t v = 0;
+            if (e < E) {
+                const int64_t rows = (int64_t)p.offsets[e + 1] - p.offsets[e];
+                v = (int32_t)(ceil_div(rows, BM) * n_tiles);
+            }
+            local[i < 32 ? i : 31] = v;
+            sum += v;
+        }
+        int32_t incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            int32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        int32_t run = incl - sum;
+        for (int i = 0; i < per; ++i) {
+            const int e = lane * per + i;
+            if (e < E) prefix[e] = run;
+            run += local[i < 32 ? i : 31];
+        }
+        if (lane == 31) {
+            prefix[E] = incl;
+            int32_t tot = incl;
+            if ((int64_t)p.offsets[E] > p.S) {   // inconsistent offsets: do nothing
+                raise_error(kErrBadOffsets);
+                tot = 0;
+            }
+            *total_tiles = tot;
+        }
+        if (lane == 0) {
+            asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&map_a) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&map_b) : "memory");
+        }
+    }
+    if (warp == 3) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int64_t ntiles = *total_tiles;
+
+    if (warp == 0) {
+        // ================= TMA producer =================
+        if (lane == 0) {
+            uint32_t it = 0;
+            bool ok = true;
+            for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+                const Tile tl = tile_of(t, prefix, p.offsets, E, n_tiles);
+                const int64_t wbase = (int64_t)tl.e * p.N;
+                int yb0, yb1;
+                if (EPI == DS4G_EPI_SWIGLU_REQUANT) {
+                    yb0 = (int)(wbase + (int64_t)tl.nt * 128);
+                    yb1 = (int)(wbase + I + (int64_t)tl.nt * 128);
+                } else {
+                    yb0 = (int)(wbase + (int64_t)tl.nt * BN);
+                    yb1 = yb0 + 128;
+                }
+                for (int ks = 0; ks < nks; ++ks, ++it) {
+                    const int s = it % STAGES;
+                    const uint32_t ph = (it / STAGES) & 1;
+                    if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1, abort_flag)) { ok = false; break; }
+                    const uint32_t fb = smem_u32(&full[s]);
+                    mbar_arrive_tx(fb, A_BYTES + B_BYTES);
+                    tma_load_2d(smem_u32(sA + s * A_BYTES), &map_a, fb, ks * BKB, (int)tl.m0);
+                    tma_load_2d(smem_u32(sB + s * B_BYTES), &map_b, fb, ks * BKB, yb0);
+                    tma_load_2d(smem_u32(sB + s * B_BYTES + B_BYTES / 2), &map_b, fb, ks * BKB, yb1);
+                }
+            }
+            if (!ok) {
+                // let copies already issued land before the CTA goes away
+                for (uint32_t j = (it > STAGES ? it - STAGES : 0); j < it; ++j) {
+                    volatile int dummy = 0;
+                    mbar_wait(smem_u32(&full[j % STAGES]), (j / STAGES) & 1, &dummy);
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ================= MMA issuer =================
+        if (lane == 0) {
+            const uint32_t ibase = idesc_base<FMT>();
+            uint32_t it = 0, tcount = 0;
+            bool ok = true;
+            for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++tcount) {
+                if (!mbar_wait(smem_u32(tmem_empty), (tcount & 1) ^ 1, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                for (int ks = 0; ks < nks; ++ks, ++it) {
+                    const int s = it % STAGES;
+                    const uint32_t ph = (it / STAGES) & 1;
+                    if (!mbar_wait(smem_u32(&full[s]), ph, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    // scale factors of this stage -> TMEM
+                    const uint32_t sfa_s = smem_u32(sSFA + s * C::SFA_BYTES);
+                    const uint32_t sfb_s = smem_u32(sSFB + s * C::SFB_BYTES);
+#pragma unroll
+                    for (int c = 0; c < C::WORDS; ++c) {
+                        utccp(tmem + kColSFA + 4 * c, desc_sf(sfa_s + c * 512));
+                        utccp(tmem + kColSFB + 8 * c, desc_sf(sfb_s + c * 1024));
+                        utccp(tmem + kColSFB + 8 * c + 4, desc_sf(sfb_s + c * 1024 + 512));
+                    }
+                    const int64_t krem = K - (int64_t)ks * BK;
+                    const int nmma = krem >= BK ? 4 : (int)(krem / 64);
+                    const uint32_t a_s = smem_u32(sA + s * A_BYTES);
+                    const uint32_t b_s = smem_u32(sB + s * B_BYTES);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        if (j < nmma) {
+                            const int c = (FMT == DS4G_MXFP4) ? (j >> 1) : j;
+                            const uint32_t sfid = (FMT == DS4G_MXFP4) ? (uint32_t)((j & 1) * 2) : 0u;
+                            const uint32_t idesc = ibase | (sfid << 4) | (sfid << 29);
+                            mma<FMT>(tmem + kColAcc, desc_sw128(a_s + 32 * j), desc_sw128(b_s + 32 * j), idesc,
+                                     (ks > 0 || j > 0) ? 1u : 0u, tmem + kColSFA + 4 * c, tmem + kColSFB + 8 * c);
+                        }
+                    }
+                    tc_commit(smem_u32(&empty[s]));
+                }
+                if (!ok) break;
+                tc_commit(smem_u32(tmem_full));
+            }
+        }
+        __syncwarp();
+    } else if (warp == 2) {
+        // ================= scale-factor loader =================
+        uint32_t it = 0, pending_from = 0;
+        bool ok = true;
+        const int64_t sa_row = K / ((FMT == DS4G_MXFP4) ? 32 : 16);   // scale bytes per row
+        for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+            const Tile tl = tile_of(t, prefix, p.offsets, E, n_tiles);
+            const int64_t wbase = (int64_t)tl.e * p.N;
+            for (int ks = 0; ks < nks; ++ks, ++it) {
+                const int s = it % STAGES;
+                const uint32_t ph = (it / STAGES) & 1;
+                bool w_ok = true;
+                if (lane == 0) w_ok = mbar_wait(smem_u32(&empty[s]), ph ^ 1, abort_flag);
+                w_ok = __shfl_sync(0xffffffffu, w_ok ? 1 : 0, 0) != 0;
+                if (!w_ok) { ok = false; break; }
+                const int64_t krem = K - (int64_t)ks * BK;
+                const int nw = (int)min((int64_t)C::WORDS, krem / C::K_PER_WORD);
+                const int64_t kb = (int64_t)ks * (C::WORDS * 4);          // first scale byte of the stage
+                const uint32_t sfa_s = smem_u32(sSFA + s * C::SFA_BYTES);
+                const uint32_t sfb_s = smem_u32(sSFB + s * C::SFB_BYTES);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int64_t row = tl.m0 + lane + 32 * q;
+                    const bool valid = row < p.S;
+                    for (int c = 0; c < nw; ++c) {
+                        const uint8_t* src = valid ? (p.a_scales + row * sa_row + kb + 4 * c) : p.a_scales;
+                        cp_async4(sfa_s + c * 512 + lane * 16 + q * 4, src, valid ? 4u : 0u);
+                    }
+                }
+#pragma unroll
+                for (int g = 0; g < 2; ++g) {
+                    int64_t brow0;
+                    if (EPI == DS4G_EPI_SWIGLU_REQUANT) brow0 = wbase + (g ? I : 0) + (int64_t)tl.nt * 128;
+                    else brow0 = wbase + (int64_t)tl.nt * BN + 128 * g;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int64_t row = brow0 + lane + 32 * q;
+                        for (int c = 0; c < nw; ++c)
+                            cp_async4(sfb_s + c * 1024 + g * 512 + lane * 16 + q * 4,
+                                      p.w_scales + row * sa_row + kb + 4 * c, 4u);
+                    }
+                }
+                cp_async_commit();
+                if (it >= pending_from + kSfLag) {
+                    cp_async_wait<kSfLag>();
+                    fence_proxy_async();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(smem_u32(&full[(it - kSfLag) % STAGES]));
+                }
+                if (it + 1 < pending_from + kSfLag) { /* still filling the lag window */ }
+            }
+        }
+        // publish the stages still in flight
+        cp_async_wait<0>();
+        fence_proxy_async();
+        __syncwarp();
+        if (lane == 0) {
+            const uint32_t first = it >= kSfLag ? it - kSfLag : 0;
+            for (uint32_t j = first; j < it; ++j) mbar_arrive(smem_u32(&full[j % STAGES]));
+        }
+        (void)pending_from;
+    } else if (warp >= 4) {
+        // ================= epilogue =================
+        const int ew = warp - 4;
+        uint32_t tcount = 0;
+        const float gh = (FMT == DS4G_NVFP4 && EPI == DS4G_EPI_SWIGLU_REQUANT) ? *p.oq_g : 1.0f;
+        for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, ++tcount) {
+            if (!mbar_wait(smem_u32(tmem_full), tcount & 1, abort_flag)) break;
+            tc_fence_after();
+            const Tile tl = tile_of(t, prefix, p.offsets, E, n_tiles);
+            const float gscale = (FMT == DS4G_NVFP4) ? __fmul_rn(p.a_g[0], p.w_g[tl.e]) : 1.0f;
+            const int64_t row = tl.m0 + 32 * ew + lane;
+            const bool valid = row < tl.end;
+            const uint32_t tbase = tmem + kColAcc + ((uint32_t)(32 * ew) << 16);
+            if (EPI == DS4G_EPI_NONE) {
+#pragma unroll 1
+                for (int c8 = 0; c8 < BN / 32; ++c8) {
+                    float v[32];
+                    tmem_ld32(tbase + 32 * c8, v);
+                    if (valid) {
+                        float4* dst = reinterpret_cast<float4*>(p.out + row * p.N + (int64_t)tl.nt * BN + 32 * c8);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            dst[i] = make_float4(v[4 * i] * gscale, v[4 * i + 1] * gscale, v[4 * i + 2] * gscale,
+                                                 v[4 * i + 3] * gscale);
+                    }
+                }
+            } else {
+#pragma unroll 1
+                for (int j = 0; j < 4; ++j) {
+                    float gv[32], uv[32];
+                    tmem_ld32(tbase + 32 * j, gv);
+                    tmem_ld32(tbase + 128 + 32 * j, uv);
+                    const int64_t col0 = (int64_t)tl.nt * 128 + 32 * j;
+                    float h[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const float g = gv[i] * gscale, u = uv[i] * gscale;
+                        h[i] = __fmul_rn(__fdiv_rn(g, __fadd_rn(1.0f, expf(-g))), u);
+                    }
+                    if (valid) {
+                        if (p.h_debug) {
+                            float4* hd = reinterpret_cast<float4*>(p.h_debug + row * I + col0);
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) hd[i] = make_float4(h[4 * i], h[4 * i + 1], h[4 * i + 2], h[4 * i + 3]);
+                        }
+                        uint32_t wq[4] = {0, 0, 0, 0};
+                        if (FMT == DS4G_MXFP4) {
+                            float m = 0.f;
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) m = fmaxf(m, fabsf(h[i]));
+                            const int X = mx_shared_exp(m);
+                            const float inv = exp2i(-X);
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) wq[i >> 3] |= e2m1_code(__fmul_rn(h[i], inv)) << (4 * (i & 7));
+                            p.oq_scales[row * (I / 32) + col0 / 32] = (uint8_t)(X + 127);
+                        } else {
+                            uint32_t sb[2];
+#pragma unroll
+                            for (int hb = 0; hb < 2; ++hb) {
+                                float m = 0.f;
+#pragma unroll
+                                for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(h[16 * hb + i]));
+                                const uint32_t s = ue4m3_encode(__fdiv_rn(m, __fmul_rn(6.0f, gh)));
+                                const float ds = ue4m3_value(s);
+                                const float den = __fmul_rn(ds, gh);
+#pragma unroll
+                                for (int i = 0; i < 16; ++i) {
+                                    const float x = h[16 * hb + i];
+                                    const uint32_t code =
+                                        (ds == 0.0f) ? ((__float_as_uint(x) >> 28) & 8u) : e2m1_code(__fdiv_rn(x, den));
+                                    wq[2 * hb + (i >> 3)] |= code << (4 * (i & 7));
+                                }
+                                sb[hb] = s;
+                            }
+                            *reinterpret_cast<uint16_t*>(p.oq_scales + row * (I / 16) + col0 / 16) =
+                                (uint16_t)(sb[0] | (sb[1] << 8));
+                        }
+                        *reinterpret_cast<uint4*>(p.oq_data + row * (I / 2) + col0 / 2) =
+                            make_uint4(wq[0], wq[1], wq[2], wq[3]);
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(smem_u32(tmem_empty));
+        }
+    }
+
+    // ---- teardown
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 3) {
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+    }
+}
+
+}  // namespace tc
+
+// ---- host side -----------------------------------------------------------------
+typedef CUresult (*PFN_encodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static PFN_encodeTiled get_encode()
+{
+    static PFN_encodeTiled fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_encodeTiled>(ptr);
+    }
+    return fn;
+}
+
+// 2-D map over a packed FP4 matrix [rows][K/2] bytes, box 128 bytes x 128 rows
+static bool make_map(CUtensorMap* m, const uint8_t* base, int64_t rows, int64_t K)
+{
+    PFN_encodeTiled enc = get_encode();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
+    cuuint32_t box[2] = {128, 128};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int FMT, int EPI>
+static cudaError_t run_tc(const GemmArgs& a, const CUtensorMap& ma, const CUtensorMap& mb, cudaStream_t st)
+{
+    auto kern = tc::k_gemm_tc<FMT, EPI>;
+    const size_t shm = tc::Cfg<FMT>::SMEM;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)shm);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = kNumSMs;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    kern<<<sms, tc::kThreads, shm, st>>>(ma, mb, a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st)
+{
+    if (a.S == 0) return cudaSuccess;
+    if (a.E > tc::kMaxE) return cudaErrorInvalidValue;
+    CUtensorMap ma, mb;
+    if (!make_map(&ma, a.a_data, a.S, a.K) || !make_map(&mb, a.w_data, (int64_t)a.E * a.N, a.K))
+        return cudaErrorInvalidValue;
+    if (a.fmt == DS4G_MXFP4)
+        return a.epilogue == DS4G_EPI_NONE ? run_tc<DS4G_MXFP4, DS4G_EPI_NONE>(a, ma, mb, st)
+                                           : run_tc<DS4G_MXFP4, DS4G_EPI_SWIGLU_REQUANT>(a, ma, mb, st);
+    return a.epilogue == DS4G_EPI_NONE ? run_tc<DS4G_NVFP4, DS4G_EPI_NONE>(a, ma, mb, st)
+                                       : run_tc<DS4G_NVFP4, DS4G_EPI_SWIGLU_REQUANT>(a, ma, mb, st);
+}
+
+}  // namespace ds4g

@@ -1,0 +1,144 @@
+// permute.cu -- expert-contiguous permutation of the routed slots and the
+// gather of the quantised rows ("[DeepSeek V4] Triton FP4 optimisation in
+// practice", "Step 0": the grouped GEMM takes the rows of each expert as one
+// contiguous segment).
+//
+// Slots s = t*k + j are split into chunks of kChunk.  Three small kernels:
+//   hist     per-chunk expert histogram          -> ws[e * B + b]
+//   scan     exclusive scan of ws in (e, b) order -> segment bases, offsets
+//   rank     per chunk, one warp walks its slots in order; __match_any_sync
+//            ranks equal experts inside each group of 32 and a shared
+//            running count carries the rank across groups, so the order
+//            inside an expert is ascending slot id (stable)
+// and a gather that copies each permuted row's packed data and scales with
+// 16-byte loads, one warp per row.
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace ds4g {
+
+constexpr int kChunk = 1024;
+
+size_t permute_workspace_bytes(int T, int k, int E)
+{
+    int64_t S = (int64_t)T * k;
+    int64_t B = ceil_div(S, kChunk);
+    if (B < 1) B = 1;
+    return (size_t)(E * B) * sizeof(int32_t);
+}
+
+__global__ void k_perm_hist(const int32_t* __restrict__ idx, int64_t S, int E, int B, int32_t* __restrict__ ws)
+{
+    extern __shared__ int32_t h[];
+    for (int e = threadIdx.x; e < E; e += blockDim.x) h[e] = 0;
+    __syncthreads();
+    const int64_t s0 = (int64_t)blockIdx.x * kChunk;
+    const int64_t s1 = min(s0 + kChunk, S);
+    for (int64_t s = s0 + threadIdx.x; s < s1; s += blockDim.x) atomicAdd(&h[idx[s]], 1);
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) ws[(int64_t)e * B + blockIdx.x] = h[e];
+}
+
+// exclusive scan of n = E*B ints in place (one block of 1024 threads); also
+// offsets[e] = scanned[e*B], offsets[E] = S
+__global__ void k_perm_scan(int32_t* __restrict__ ws, int n, int E, int B, int64_t S, int32_t* __restrict__ offsets)
+{
+    __shared__ int32_t part[1024];
+    const int tid = threadIdx.x;
+    const int per = (n + blockDim.x - 1) / blockDim.x;
+    const int b0 = tid * per, b1 = min(b0 + per, n);
+    int32_t sum = 0;
+    for (int i = b0; i < b1; ++i) sum += ws[i];
+    part[tid] = sum;
+    __syncthreads();
+    for (int o = 1; o < (int)blockDim.x; o <<= 1) {   // Hillis-Steele inclusive scan
+        int32_t v = (tid >= o) ? part[tid - o] : 0;
+        __syncthreads();
+        part[tid] += v;
+        __syncthreads();
+    }
+    int32_t run = part[tid] - sum;                      // exclusive base of this thread
+    for (int i = b0; i < b1; ++i) {
+        int32_t c = ws[i];
+        ws[i] = run;
+        run += c;
+    }
+    __syncthreads();
+    for (int e = tid; e < E; e += blockDim.x) offsets[e] = ws[(int64_t)e * B];
+    if (tid == 0) offsets[E] = (int32_t)S;
+}
+
+__global__ void k_perm_rank(const int32_t* __restrict__ idx, int64_t S, int E, int B,
+                            const int32_t* __restrict__ base, int32_t* __restrict__ row_to_slot,
+                            int32_t* __restrict__ slot_to_row)
+{
+    extern __shared__ int32_t cnt[];
+    const int lane = threadIdx.x;
+    for (int e = lane; e < E; e += 32) cnt[e] = 0;
+    __syncwarp();
+    const int64_t s0 = (int64_t)blockIdx.x * kChunk;
+    const int64_t s1 = min(s0 + kChunk, S);
+    for (int64_t g = s0; g < s1; g += 32) {
+        const int64_t s = g + lane;
+        const bool valid = s < s1;
+        const int e = valid ? idx[s] : -1 - lane;     // invalid lanes never match a real expert
+        const unsigned peers = __match_any_sync(0xffffffffu, e);
+        const int rank = __popc(peers & ((1u << lane) - 1u));
+        int32_t pos = 0;
+        if (valid) pos = base[(int64_t)e * B + blockIdx.x] + cnt[e] + rank;
+        __syncwarp();
+        if (valid && rank == 0) cnt[e] += __popc(peers);
+        __syncwarp();
+        if (valid) {
+            row_to_slot[pos] = (int32_t)s;
+            slot_to_row[s] = pos;
+        }
+    }
+}
+
+// one warp per permuted row: copy data (K/2 bytes, 16-byte pieces) and scales
+__global__ void k_perm_gather(const uint8_t* __restrict__ xd, const uint8_t* __restrict__ xs,
+                              const float* __restrict__ xg, int64_t S, int k, int64_t K, int blk,
+                              const int32_t* __restrict__ row_to_slot, uint8_t* __restrict__ ad,
+                              uint8_t* __restrict__ as, float* __restrict__ ag)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (ag && r == 0 && lane == 0) *ag = *xg;
+    if (r >= S) return;
+    const int64_t t = row_to_slot[r] / k;
+    const int64_t nvec = K / 32;                         // 16-byte pieces of K/2 bytes
+    const uint4* src = reinterpret_cast<const uint4*>(xd + t * (K / 2));
+    uint4* dst = reinterpret_cast<uint4*>(ad + r * (K / 2));
+    for (int64_t i = lane; i < nvec; i += 32) dst[i] = src[i];
+    const int64_t ns = K / blk;                          // scale bytes per row (even)
+    const uint16_t* ss = reinterpret_cast<const uint16_t*>(xs + t * ns);
+    uint16_t* sd = reinterpret_cast<uint16_t*>(as + r * ns);
+    for (int64_t i = lane; i < ns / 2; i += 32) sd[i] = ss[i];
+}
+
+cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, const uint8_t* xd, const uint8_t* xs,
+                           const float* xg, int64_t K, int fmt, int32_t* offsets, int32_t* row_to_slot,
+                           int32_t* slot_to_row, uint8_t* ad, uint8_t* as, float* ag, void* ws_,
+                           cudaStream_t st)
+{
+    const int64_t S = (int64_t)T * k;
+    int32_t* ws = reinterpret_cast<int32_t*>(ws_);
+    const int B = (int)(S > 0 ? ceil_div(S, kChunk) : 1);
+    const size_t shm = (size_t)E * sizeof(int32_t);
+    if (S == 0) {
+        cudaError_t e = cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (E + 1), st);
+        if (e != cudaSuccess) return e;
+        if (fmt == DS4G_NVFP4 && ag) return cudaMemcpyAsync(ag, xg, sizeof(float), cudaMemcpyDeviceToDevice, st);
+        return cudaSuccess;
+    }
+    k_perm_hist<<<B, 256, shm, st>>>(idx, S, E, B, ws);
+    k_perm_scan<<<1, 1024, 0, st>>>(ws, E * B, E, B, S, offsets);
+    k_perm_rank<<<B, 32, shm, st>>>(idx, S, E, B, ws, row_to_slot, slot_to_row);
+    const int blk = (fmt == DS4G_MXFP4) ? 32 : 16;
+    k_perm_gather<<<(unsigned)ceil_div(S, 8), 256, 0, st>>>(xd, xs, xg, S, k, K, blk, row_to_slot, ad, as,
+                                                          fmt == DS4G_NVFP4 ? ag : nullptr);
+    return cudaGetLastError();
+}
+
+}  // namespace ds4g

@@ -1,0 +1,202 @@
+"""Thin Python binding of libds4g (include/ds4g.h).
+
+Argument marshalling only: every step runs in the library's CUDA kernels.
+PyTorch provides device memory and the current stream.  If the compiled
+library is missing, importing this module raises: there is no fallback.
+"""
+import ctypes
+import os
+
+import torch
+
+from . import build as _build
+
+MXFP4 = 0
+NVFP4 = 1
+BF16 = 0
+F32 = 1
+EPI_NONE = 0
+EPI_SWIGLU_REQUANT = 1
+BLOCK = {MXFP4: 32, NVFP4: 16}
+
+_STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "unsupported device", 4: "CUDA error",
+           5: "device-side wait gave up", 6: "workspace missing or too small"}
+
+
+class Ds4gError(RuntimeError):
+    def __init__(self, call, status):
+        self.status = status
+        super().__init__(f"{call}: {_STATUS.get(status, status)} (status {status})")
+
+
+class _Fp4C(ctypes.Structure):
+    _fields_ = [("data", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("g", ctypes.c_void_p),
+                ("rows", ctypes.c_int64), ("K", ctypes.c_int64), ("fmt", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
+
+
+if not os.path.exists(_build.LIB):
+    raise ImportError(f"libds4g.so is not built ({_build.LIB}); run block_scaled_fp4_topk_b200/build.py")
+
+_lib = ctypes.CDLL(_build.LIB)
+_vp, _i32, _i64, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+_P = ctypes.POINTER(_Fp4C)
+_SIGS = {
+    "ds4g_status_str": ([_i32], ctypes.c_char_p),
+    "ds4g_device_supported": ([], _i32),
+    "ds4g_check_device": ([_vp], _i32),
+    "ds4g_quantize_workspace_bytes": ([_i32, _i32], _sz),
+    "ds4g_quantize_mx": ([_vp, _i32, _i64, _i64, _i32, _vp, _P, _vp, _sz, _vp], _i32),
+    "ds4g_route_topk": ([_vp, _i32, _i32, _i32, _vp, _vp, _vp], _i32),
+    "ds4g_permute_workspace_bytes": ([_i32, _i32, _i32], _sz),
+    "ds4g_moe_permute": ([_vp, _i32, _i32, _i32, _P, _vp, _vp, _vp, _P, _vp, _sz, _vp], _i32),
+    "ds4g_grouped_gemm_fp4": ([_P, _vp, _i32, _i32, _P, _i32, _i32, _vp, _P, _vp, _vp], _i32),
+    "ds4g_swiglu_requant": ([_vp, _i64, _i32, _i32, _P, _vp, _vp], _i32),
+    "ds4g_moe_combine": ([_vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp], _i32),
+}
+for _name, (_args, _res) in _SIGS.items():
+    _f = getattr(_lib, _name)
+    _f.argtypes = _args
+    _f.restype = _res
+
+LIB_PATH = _build.LIB
+EXPORTED = tuple(_SIGS)
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _stream():
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _check(name, st):
+    if st != 0:
+        raise Ds4gError(name, st)
+
+
+class Fp4Tensor:
+    """Device FP4 tensor: data uint8 [rows][K/2], scales uint8 [rows][K/blk],
+    g float32 [1] (NVFP4 tensor scale) or None, fmt."""
+
+    def __init__(self, data, scales, g, fmt):
+        self.data, self.scales, self.g, self.fmt = data, scales, g, fmt
+
+    @property
+    def rows(self):
+        return self.data.shape[0]
+
+    @property
+    def K(self):
+        return self.data.shape[1] * 2
+
+    @staticmethod
+    def empty(rows, K, fmt, device="cuda"):
+        g = torch.ones(1, dtype=torch.float32, device=device) if fmt == NVFP4 else None
+        return Fp4Tensor(torch.empty((rows, K // 2), dtype=torch.uint8, device=device),
+                         torch.empty((rows, K // BLOCK[fmt]), dtype=torch.uint8, device=device), g, fmt)
+
+    def c(self):
+        return _Fp4C(self.data.data_ptr(), self.scales.data_ptr(), _ptr(self.g), self.rows, self.K, self.fmt, 0)
+
+    def view_rows(self, r0, r1):
+        return Fp4Tensor(self.data[r0:r1], self.scales[r0:r1], self.g, self.fmt)
+
+
+def ds4g_device_supported():
+    return _lib.ds4g_device_supported() == 0
+
+
+def ds4g_check_device():
+    _check("ds4g_check_device", _lib.ds4g_check_device(_stream()))
+
+
+def ds4g_quantize_mx(x, fmt, g_in=None, out=None, workspace=None):
+    rows, K = x.shape
+    dtype = BF16 if x.dtype == torch.bfloat16 else F32
+    if out is None:
+        out = Fp4Tensor.empty(rows, K, fmt, x.device)
+    need = _lib.ds4g_quantize_workspace_bytes(fmt, 1 if g_in is not None else 0)
+    if need and workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=x.device)
+    c = out.c()
+    _check("ds4g_quantize_mx", _lib.ds4g_quantize_mx(x.data_ptr(), dtype, rows, K, fmt, _ptr(g_in), ctypes.byref(c),
+                                                     _ptr(workspace), 0 if workspace is None else workspace.numel(),
+                                                     _stream()))
+    return out
+
+
+def ds4g_route_topk(logits, k, idx=None, w=None):
+    T, E = logits.shape
+    if idx is None:
+        idx = torch.empty((T, k), dtype=torch.int32, device=logits.device)
+    if w is None:
+        w = torch.empty((T, k), dtype=torch.float32, device=logits.device)
+    _check("ds4g_route_topk", _lib.ds4g_route_topk(logits.data_ptr(), T, E, k, idx.data_ptr(), w.data_ptr(), _stream()))
+    return idx, w
+
+
+def permute_workspace(T, k, E, device="cuda"):
+    n = _lib.ds4g_permute_workspace_bytes(T, k, E)
+    return torch.empty(max(n, 16), dtype=torch.uint8, device=device)
+
+
+def ds4g_moe_permute(idx, E, x_q, offsets=None, row_to_slot=None, slot_to_row=None, a_perm=None, workspace=None):
+    T, k = idx.shape
+    S = T * k
+    dev = idx.device
+    if offsets is None:
+        offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    if row_to_slot is None:
+        row_to_slot = torch.empty(max(S, 1), dtype=torch.int32, device=dev)
+    if slot_to_row is None:
+        slot_to_row = torch.empty(max(S, 1), dtype=torch.int32, device=dev)
+    if a_perm is None:
+        a_perm = Fp4Tensor.empty(S, x_q.K, x_q.fmt, dev)
+    if workspace is None:
+        workspace = permute_workspace(T, k, E, dev)
+    xc, ac = x_q.c(), a_perm.c()
+    _check("ds4g_moe_permute", _lib.ds4g_moe_permute(idx.data_ptr(), T, k, E, ctypes.byref(xc), offsets.data_ptr(),
+                                                     row_to_slot.data_ptr(), slot_to_row.data_ptr(), ctypes.byref(ac),
+                                                     workspace.data_ptr(), workspace.numel(), _stream()))
+    return offsets, row_to_slot[:S], slot_to_row[:S], a_perm
+
+
+def ds4g_grouped_gemm_fp4(a, offsets, E, max_rows_per_expert, w, N, epilogue=EPI_NONE, out=None, out_q=None,
+                          h_debug=None):
+    S = a.rows
+    if epilogue == EPI_NONE and out is None:
+        out = torch.empty((S, N), dtype=torch.float32, device=a.data.device)
+    if epilogue == EPI_SWIGLU_REQUANT and out_q is None:
+        raise ValueError("SWIGLU_REQUANT needs out_q (and out_q.g for NVFP4)")
+    ac, wc = a.c(), w.c()
+    qc = out_q.c() if out_q is not None else None
+    _check("ds4g_grouped_gemm_fp4",
+           _lib.ds4g_grouped_gemm_fp4(ctypes.byref(ac), offsets.data_ptr(), E, max_rows_per_expert, ctypes.byref(wc),
+                                      N, epilogue, _ptr(out), ctypes.byref(qc) if qc is not None else None,
+                                      _ptr(h_debug), _stream()))
+    return out if epilogue == EPI_NONE else out_q
+
+
+def ds4g_swiglu_requant(y1, fmt, h_q=None, h_debug=None, g_h=None):
+    rows, two_i = y1.shape
+    I = two_i // 2
+    if h_q is None:
+        h_q = Fp4Tensor.empty(rows, I, fmt, y1.device)
+        if fmt == NVFP4 and g_h is not None:
+            h_q.g.copy_(g_h)
+    hc = h_q.c()
+    _check("ds4g_swiglu_requant", _lib.ds4g_swiglu_requant(y1.data_ptr(), rows, I, fmt, ctypes.byref(hc),
+                                                           _ptr(h_debug), _stream()))
+    return h_q
+
+
+def ds4g_moe_combine(y2, slot_to_row, w, out=None):
+    T, k = w.shape
+    d = y2.shape[1]
+    if out is None:
+        out = torch.empty((T, d), dtype=torch.float32, device=y2.device)
+    _check("ds4g_moe_combine", _lib.ds4g_moe_combine(y2.data_ptr(), slot_to_row.data_ptr(), w.data_ptr(), T, k, d,
+                                                     out.data_ptr(), _stream()))
+    return out

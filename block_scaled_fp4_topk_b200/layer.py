@@ -1,0 +1,105 @@
+"""One routed-expert MoE FFN layer with block-scaled FP4 expert weights,
+run as the sequence of libds4g calls (route -> quantise -> permute -> FC1
+with fused SwiGLU + requantisation -> FC2 -> combine) on one stream.
+
+All arithmetic happens in the library's kernels; this module only owns the
+device buffers and issues the calls.
+"""
+import torch
+
+from . import ds4g
+from .ds4g import EPI_NONE, EPI_SWIGLU_REQUANT, NVFP4, Fp4Tensor
+
+
+class MoeLayer:
+    def __init__(self, w1, w2, E, k, d, I, fmt, g_h=None, fused=True):
+        """w1: Fp4Tensor [E*2I][d] (gate rows then up rows per expert),
+        w2: Fp4Tensor [E*d][I]; NVFP4 weights carry one tensor scale per
+        expert (w.g has E floats); g_h: the static NVFP4 tensor scale of h."""
+        self.w1, self.w2 = w1, w2
+        self.E, self.k, self.d, self.I, self.fmt = E, k, d, I, fmt
+        self.fused = fused
+        self.g_h = None
+        if fmt == NVFP4:
+            dev = w1.data.device
+            self.g_h = torch.tensor([g_h if g_h is not None else 1.0], dtype=torch.float32, device=dev)
+        self._bufs = {}
+
+    def buffers(self, T, device):
+        key = (T, str(device))
+        b = self._bufs.get(key)
+        if b is None:
+            S = T * self.k
+            b = dict(
+                idx=torch.empty((T, self.k), dtype=torch.int32, device=device),
+                w=torch.empty((T, self.k), dtype=torch.float32, device=device),
+                xq=Fp4Tensor.empty(T, self.d, self.fmt, device),
+                offsets=torch.empty(self.E + 1, dtype=torch.int32, device=device),
+                r2s=torch.empty(max(S, 1), dtype=torch.int32, device=device),
+                s2r=torch.empty(max(S, 1), dtype=torch.int32, device=device),
+                a=Fp4Tensor.empty(S, self.d, self.fmt, device),
+                hq=Fp4Tensor.empty(S, self.I, self.fmt, device),
+                y2=torch.empty((S, self.d), dtype=torch.float32, device=device),
+                out=torch.empty((T, self.d), dtype=torch.float32, device=device),
+                pws=ds4g.permute_workspace(T, self.k, self.E, device),
+                qws=torch.empty(16, dtype=torch.uint8, device=device),
+            )
+            if self.fmt == NVFP4:
+                b["hq"].g = self.g_h
+            if not self.fused:
+                b["y1"] = torch.empty((S, 2 * self.I), dtype=torch.float32, device=device)
+            self._bufs[key] = b
+        return b
+
+    def forward(self, x, logits, h_debug=None):
+        """x: bf16 [T][d] (device), logits: fp32 [T][E] (device) -> fp32 [T][d]"""
+        T = x.shape[0]
+        b = self.buffers(T, x.device)
+        ds4g.ds4g_route_topk(logits, self.k, idx=b["idx"], w=b["w"])
+        ds4g.ds4g_quantize_mx(x, self.fmt, out=b["xq"], workspace=b["qws"])
+        ds4g.ds4g_moe_permute(b["idx"], self.E, b["xq"], offsets=b["offsets"], row_to_slot=b["r2s"],
+                              slot_to_row=b["s2r"], a_perm=b["a"], workspace=b["pws"])
+        if self.fused:
+            ds4g.ds4g_grouped_gemm_fp4(b["a"], b["offsets"], self.E, T, self.w1, 2 * self.I, EPI_SWIGLU_REQUANT,
+                                       out_q=b["hq"], h_debug=h_debug)
+        else:
+            ds4g.ds4g_grouped_gemm_fp4(b["a"], b["offsets"], self.E, T, self.w1, 2 * self.I, EPI_NONE, out=b["y1"])
+            ds4g.ds4g_swiglu_requant(b["y1"], self.fmt, h_q=b["hq"], h_debug=h_debug)
+        ds4g.ds4g_grouped_gemm_fp4(b["hq"], b["offsets"], self.E, T, self.w2, self.d, EPI_NONE, out=b["y2"])
+        ds4g.ds4g_moe_combine(b["y2"], b["s2r"][:T * self.k], b["w"], out=b["out"])
+        return b["out"]
+
+    # -- synthetic weights -----------------------------------------------------
+    @staticmethod
+    def synthetic_weights(E, d, I, fmt, seed=0, device="cuda", rows_w1=None, chunk=8):
+        """Expert weights drawn on the device by the seeded generator
+        (W1[e] ~ N(0, 0.02) [2I][d], W2[e] ~ N(0, 0.02) [d][I]) and quantised
+        with the library's own quantiser (offline, not part of a step)."""
+        import synth
+        from synth.workloads import W_SIGMA
+        r1 = rows_w1 if rows_w1 is not None else 2 * I
+        st = torch.cuda.current_stream().cuda_stream
+        w1 = Fp4Tensor.empty(E * r1, d, fmt, device)
+        w2 = Fp4Tensor.empty(E * d, I, fmt, device)
+        if fmt == NVFP4:
+            w1.g = torch.empty(E, dtype=torch.float32, device=device)
+            w2.g = torch.empty(E, dtype=torch.float32, device=device)
+        ws = torch.empty(16, dtype=torch.uint8, device=device)
+        for dst, rows, cols, base in ((w1, r1, d, synth.STREAM_W1), (w2, d, I, synth.STREAM_W2)):
+            buf = torch.empty((chunk * rows, cols), dtype=torch.float32, device=device)
+            for e0 in range(0, E, chunk):
+                n = min(chunk, E - e0)
+                for j in range(n):
+                    synth.cuda_fill_normal_f32(buf[j * rows:(j + 1) * rows].data_ptr(), rows * cols, seed,
+                                               base + e0 + j, W_SIGMA, 0, st)
+                if fmt == NVFP4:
+                    for j in range(n):
+                        e = e0 + j
+                        part = Fp4Tensor(dst.data[e * rows:(e + 1) * rows], dst.scales[e * rows:(e + 1) * rows],
+                                         dst.g[e:e + 1], fmt)
+                        ds4g.ds4g_quantize_mx(buf[j * rows:(j + 1) * rows], fmt, out=part, workspace=ws)
+                else:
+                    part = dst.view_rows(e0 * rows, (e0 + n) * rows)
+                    ds4g.ds4g_quantize_mx(buf[:n * rows], fmt, out=part)
+            del buf
+        return w1, w2

@@ -1,0 +1,182 @@
+/*
+ * ds4g.h -- C ABI of the block-scaled FP4 routed-expert MoE FFN library
+ * (libds4g.so, sm_100a only).
+ *
+ * One MoE layer is, in order:
+ *   ds4g_route_topk       top-k routing of each token over E experts
+ *   ds4g_quantize_mx      activations -> MXFP4 / NVFP4 (on the fly)
+ *   ds4g_moe_permute      expert-contiguous reordering of the quantised rows
+ *   ds4g_grouped_gemm_fp4 FC1 (gate+up), optionally with the SwiGLU +
+ *                         requantisation epilogue fused
+ *   ds4g_swiglu_requant   the same epilogue as a separate step
+ *   ds4g_grouped_gemm_fp4 FC2
+ *   ds4g_moe_combine      routing-weighted sum of each token's k expert rows
+ *
+ * Sources: "DGX Spark native FP4 matrix instructions: how DwarfStar uses
+ * Blackwell" (sec. 1 FP4 formats and the block-scaled MMA, sec. 2 MoE
+ * routing and batched expert GEMM with FP4 weights and activations, sec. 3
+ * the K % 64 shape check with an error instead of a silent fallback);
+ * "[DeepSeek V4] Triton FP4 optimisation in practice" ("What is the FP4 MoE
+ * GEMM": 256 experts, 6 active, 2 FC per expert; "Step 0": the grouped
+ * contiguous GEMM; "Step 2": packed FP4, even column = low nibble);
+ * "Moore Threads full-link adaptation of DeepSeek-V4" (fused SwiGLU +
+ * quantisation; MoE routing / combine).
+ *
+ * Conventions (every entry point):
+ *   - All pointers are DEVICE pointers unless stated otherwise; the caller
+ *     allocates and owns all memory.  The library never allocates device
+ *     memory; scratch space comes from a caller-provided workspace whose size
+ *     the matching *_workspace_bytes() call returns.
+ *   - Calls are asynchronous on the given stream (cudaStream_t passed as
+ *     void*; NULL = the legacy default stream).
+ *   - Arguments and shapes are validated on the host before any launch; a bad
+ *     argument returns an error status and launches nothing.  There is no
+ *     silent fallback and no CPU path.
+ *   - Launch failures return DS4G_ERR_CUDA.  A device-side wait that gives up
+ *     (a bounded spin in a persistent kernel) records an error word that
+ *     ds4g_check_device() turns into DS4G_ERR_DEVICE.
+ *   - Inputs must be finite (no NaN / Inf).
+ */
+#ifndef DS4G_H
+#define DS4G_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    DS4G_OK = 0,
+    DS4G_ERR_INVALID_ARG = 1,   /* null pointer, bad enum, misaligned pointer, k > E ... */
+    DS4G_ERR_SHAPE = 2,         /* K % 64 != 0 and other shape rules below */
+    DS4G_ERR_UNSUPPORTED = 3,   /* device is not sm_100 */
+    DS4G_ERR_CUDA = 4,          /* a CUDA runtime / launch error */
+    DS4G_ERR_DEVICE = 5,        /* a device-side bounded wait gave up */
+    DS4G_ERR_WORKSPACE = 6      /* workspace missing or too small */
+} ds4g_status;
+
+typedef enum { DS4G_MXFP4 = 0, DS4G_NVFP4 = 1 } ds4g_fmt;
+typedef enum { DS4G_BF16 = 0, DS4G_F32 = 1 } ds4g_dtype;
+typedef enum { DS4G_EPI_NONE = 0, DS4G_EPI_SWIGLU_REQUANT = 1 } ds4g_epilogue;
+
+/* An FP4 tensor of `rows` x `K` elements (row-major along K).
+ *   data   [rows][K/2] bytes: E2M1 codes (sign, 2 exponent, 1 mantissa bit),
+ *          element 2i in the low nibble of byte i, 2i+1 in the high nibble.
+ *   scales [rows][K/32] UE8M0 bytes (MXFP4: value 2^(b-127)) or
+ *          [rows][K/16] UE4M3 bytes (NVFP4: unsigned E4M3, max 448).
+ *   g      NVFP4 only: one fp32 tensor scale (device); element value =
+ *          E2M1 * UE4M3 * g.  Ignored (may be NULL) for MXFP4.
+ *   data and scales must be 16-byte aligned. */
+typedef struct {
+    uint8_t* data;
+    uint8_t* scales;
+    float* g;
+    int64_t rows;
+    int64_t K;
+    int32_t fmt;   /* ds4g_fmt */
+    int32_t reserved;
+} ds4g_fp4;
+
+/* Human-readable name of a status code (static string). */
+const char* ds4g_status_str(ds4g_status s);
+
+/* DS4G_OK when the current device is sm_100 (B200 class). */
+ds4g_status ds4g_device_supported(void);
+
+/* Synchronises `stream`, then reports (and clears) the device error word:
+ * DS4G_ERR_DEVICE if a bounded device wait gave up since the last check. */
+ds4g_status ds4g_check_device(void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Quantise rows of x (bf16 or fp32, [rows][K]) to MXFP4 or NVFP4.
+ *   MXFP4 ("DGX Spark native FP4 ..." sec. 1, E2M1 + UE8M0 per 32): per
+ *     block, X = floor(log2(amax)) - 2 clamped to [-127, 127] (the OCP MX
+ *     rule), scale byte X + 127, code = E2M1 round-to-nearest-even of
+ *     v * 2^-X, saturating at 6, sign bit kept.
+ *   NVFP4 (sec. 1, kind::mxf4nvf4: E2M1 + UE4M3 per 16) with a tensor scale
+ *     g: g = *g_in if g_in != NULL, else amax(x) / 2688 computed on the
+ *     device (1 if amax is 0) and written to out->g; per block
+ *     s = E4M3_RNE(amax_b / fp32(6 g)) saturating at 448, code =
+ *     E2M1_RNE(v / fp32(dec(s) g)); all fp32, IEEE rounding.
+ * K % 64 == 0 (DS4G_ERR_SHAPE otherwise).  out->rows/K/fmt must match.
+ * Workspace: ds4g_quantize_workspace_bytes(fmt, g_in != NULL) bytes (16 for
+ * NVFP4 without g_in, else 0). */
+size_t ds4g_quantize_workspace_bytes(int fmt, int has_g_in);
+ds4g_status ds4g_quantize_mx(const void* x, int dtype, int64_t rows, int64_t K, int fmt,
+                             const float* g_in, ds4g_fp4* out,
+                             void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Top-k routing ("DGX Spark native FP4 ..." sec. 2; "[DeepSeek V4] Triton
+ * FP4 ..." "What is the FP4 MoE GEMM").  For each token t of logits [T][E]
+ * (fp32): the k largest logits, ties to the lower expert index, written in
+ * descending order to idx [T][k] (int32); weights w [T][k] (fp32) are the
+ * softmax over the k selected logits (they sum to 1).  1 <= k <= min(E, 32),
+ * E <= 1024. */
+ds4g_status ds4g_route_topk(const float* logits, int T, int E, int k, int32_t* idx, float* w,
+                            void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Expert-contiguous permutation ("[DeepSeek V4] Triton FP4 ..." "Step 0":
+ * rows grouped per expert).  From idx [T][k]:
+ *   offsets [E+1]   exclusive prefix sum of the per-expert slot counts
+ *   row_to_slot [S] slot s = t*k + j of permuted row r; within an expert the
+ *                   slots are in ascending order (stable)
+ *   slot_to_row [S] the inverse
+ *   a_perm          row r = row t = row_to_slot[r] / k of x_q (data and
+ *                   scales copied; for NVFP4 a_perm->g receives x_q->g)
+ * S = T*k; a_perm->rows must be S, same K and fmt as x_q.
+ * Workspace: ds4g_permute_workspace_bytes(T, k, E). */
+size_t ds4g_permute_workspace_bytes(int T, int k, int E);
+ds4g_status ds4g_moe_permute(const int32_t* idx, int T, int k, int E, const ds4g_fp4* x_q,
+                             int32_t* offsets, int32_t* row_to_slot, int32_t* slot_to_row,
+                             ds4g_fp4* a_perm, void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Grouped block-scaled FP4 GEMM ("DGX Spark native FP4 ..." sec. 1-2; the
+ * grouped contiguous GEMM of "[DeepSeek V4] Triton FP4 ..." "Step 0").
+ * For every expert e and every row r of its segment [offsets[e],
+ * offsets[e+1]) of a (a->rows = S rows, K columns):
+ *   y[r][n] = sum_k deq(a[r][k]) * deq(w[e*N + n][k])   (fp32 accumulate;
+ *             NVFP4: times a->g[0] * w->g[e])
+ * w has E*N rows of K columns, same fmt as a; for NVFP4 w->g holds one fp32
+ * tensor scale per expert ([E] floats, each expert's weight matrix being its
+ * own tensor).
+ * epilogue DS4G_EPI_NONE: out = y, fp32 [S][N].
+ * epilogue DS4G_EPI_SWIGLU_REQUANT (FC1 with N = 2I): columns [0, I) are the
+ *   gate and [I, 2I) the up projection; h = silu(gate) * up (fp32,
+ *   silu(x) = x / (1 + e^-x)) is quantised to out_q ([S][I], same rule as
+ *   ds4g_quantize_mx; for NVFP4 *out_q->g is the caller's static tensor
+ *   scale of h, read, not written); h_debug (nullable) receives h fp32 [S][I].
+ * max_rows_per_expert: an upper bound on any segment length (T for top-k
+ *   routing).  <= 8 selects the weight-streaming GEMV kernel, otherwise the
+ *   tcgen05 tensor-core kernel (which also needs K % 128 == 0).
+ * Shapes: K % 64 == 0; NONE needs N % 256 == 0 (tensor-core path) or
+ *   N % 64 == 0 (GEMV path); SWIGLU_REQUANT needs I % 128 == 0 (tensor-core)
+ *   or I % 32 == 0 (GEMV).  offsets[E] must equal S. */
+ds4g_status ds4g_grouped_gemm_fp4(const ds4g_fp4* a, const int32_t* offsets, int E,
+                                  int max_rows_per_expert, const ds4g_fp4* w, int N, int epilogue,
+                                  float* out, ds4g_fp4* out_q, float* h_debug, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * The SwiGLU + requantisation epilogue as its own step ("Moore Threads ..."
+ * fused SwiGLU + quant pattern): y1 fp32 [rows][2I] -> h_q (fmt, [rows][I]);
+ * h_debug (nullable) receives h fp32.  For NVFP4 *h_q->g is the static
+ * tensor scale (input).  I % 32 == 0. */
+ds4g_status ds4g_swiglu_requant(const float* y1, int64_t rows, int I, int fmt, ds4g_fp4* h_q,
+                                float* h_debug, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Combine ("Moore Threads ..." MoE combine): out[t][c] =
+ *   sum_{j=0..k-1} w[t][j] * y2[slot_to_row[t*k + j]][c]   (fp32, j order)
+ * y2 fp32 [T*k][d], w fp32 [T][k], out fp32 [T][d]; d % 4 == 0. */
+ds4g_status ds4g_moe_combine(const float* y2, const int32_t* slot_to_row, const float* w, int T,
+                             int k, int d, float* out, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DS4G_H */

@@ -30,12 +30,14 @@ double orc_e2m1_decode(int code)
  * of the code is the sign bit of y. */
 int orc_e2m1_encode(double y)
 {
+    /* the 8 non-negative grid values, from the field decode above */
+    static const double grid[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
     int sign = signbit(y) ? 8 : 0;
     double a = fabs(y);
     int best = 0;
     double best_d = INFINITY;
     for (int c = 0; c < 8; ++c) {
-        double d = fabs(a - orc_e2m1_decode(c));
+        double d = fabs(a - grid[c]);
         if (d < best_d || (d == best_d && (c & 1) == 0 && (best & 1) == 1)) {
             best = c;
             best_d = d;
@@ -114,6 +116,7 @@ static int get_nibble(const uint8_t* row, int64_t k)
  * ------------------------------------------------------------------------- */
 void orc_quantize_mx(const float* x, int64_t rows, int64_t K, uint8_t* data, uint8_t* scales)
 {
+#pragma omp parallel for schedule(static)
     for (int64_t r = 0; r < rows; ++r) {
         const float* xr = x + r * K;
         uint8_t* dr = data + r * (K / 2);
@@ -165,7 +168,8 @@ void orc_quantize_nv(const float* x, int64_t rows, int64_t K, const float* g_in,
         g = (amax == 0.0f) ? 1.0f : amax / 2688.0f;
     }
     if (g_out) *g_out = g;
-    volatile float six_g = 6.0f * g;
+    const float six_g = 6.0f * g;
+#pragma omp parallel for schedule(static)
     for (int64_t r = 0; r < rows; ++r) {
         const float* xr = x + r * K;
         uint8_t* dr = data + r * (K / 2);
@@ -176,18 +180,18 @@ void orc_quantize_nv(const float* x, int64_t rows, int64_t K, const float* g_in,
                 float v = fabsf(xr[b * 16 + i]);
                 if (v > amax) amax = v;
             }
-            volatile float ratio = amax / six_g;
+            float ratio = amax / six_g;
             int s = orc_ue4m3_encode((double)ratio);
             scales[r * (K / 16) + b] = (uint8_t)s;
             float ds = (float)orc_ue4m3_decode(s);
-            volatile float denom = ds * g;
+            float denom = ds * g;
             for (int i = 0; i < 16; ++i) {
                 float v = xr[b * 16 + i];
                 int code;
                 if (ds == 0.0f) {
                     code = signbit(v) ? 8 : 0;
                 } else {
-                    volatile float y = v / denom;
+                    float y = v / denom;
                     code = orc_e2m1_encode((double)y);
                 }
                 put_nibble(dr, b * 16 + i, code);

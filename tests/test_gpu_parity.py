@@ -1,0 +1,275 @@
+"""GPU parity: every library call against the CPU oracle on the same seeded
+inputs, through the C ABI.  Bytes, indices and offsets bit-exact; GEMM
+outputs within |gpu - ref| <= 1e-5 * sum|a w| + 1e-6 per element; FP4 codes
+that the GPU derives from its own fp32 arithmetic checked for validity
+against the oracle's values; full layers within relative L2 <= 1e-2."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from parity_helpers import (assert_gemm_close, bf16_dev, check_requant, dev, from_dev, to_dev, unpack)
+from synth.workloads import G_H
+
+pytestmark = pytest.mark.gpu
+
+ds4g = pytest.importorskip("block_scaled_fp4_topk_b200.ds4g")
+MX, NV = oracle.MX, oracle.NV
+
+
+def _x_f32(rows, K, stream, sigma=1.0):
+    return synth.normal_f32((rows, K), 0, stream, sigma)
+
+
+# ---- generator: host and device produce the same bits ----------------------
+
+def test_generator_device_matches_host():
+    n = 1 << 20
+    ref = synth.normal_f32((n,), 0, 4242, 0.02, offset=12345)
+    buf = torch.empty(n, dtype=torch.float32, device=dev())
+    synth.cuda_fill_normal_f32(buf.data_ptr(), n, 0, 4242, 0.02, 12345, torch.cuda.current_stream().cuda_stream)
+    assert np.array_equal(buf.cpu().numpy().view(np.uint32), ref.view(np.uint32))
+    bits = synth.normal_bf16_bits((n,), 0, synth.STREAM_X)
+    bb = torch.empty(n, dtype=torch.int16, device=dev())
+    synth.cuda_fill_normal_bf16(bb.data_ptr(), n, 0, synth.STREAM_X, 1.0, 0, torch.cuda.current_stream().cuda_stream)
+    assert np.array_equal(bb.cpu().numpy().view(np.uint16), bits)
+    lg = synth.logits(64, 256, 0, 1.5)
+    lt = torch.empty((64, 256), dtype=torch.float32, device=dev())
+    synth.cuda_fill_logits(lt.data_ptr(), 64, 256, 0, 1.5, torch.cuda.current_stream().cuda_stream)
+    assert np.array_equal(lt.cpu().numpy().view(np.uint32), lg.view(np.uint32))
+
+
+# ---- quantisation ------------------------------------------------------------
+
+def _special_rows(x):
+    x = x.copy()
+    x[0, :64] = 0.0
+    x[0, 64:96] = -0.0
+    x[1, :32] *= 1e-38          # subnormal-range block
+    x[1, 32:64] = 3e4           # large block
+    x[2, 5] = 6.0 * 2 ** 10     # exact grid values / ties
+    x[2, 6] = 5.0 * 2 ** 10
+    x[2, 7] = -2.5 * 2 ** 10
+    return x
+
+
+@pytest.mark.parametrize("fmt", [MX, NV])
+@pytest.mark.parametrize("src", ["bf16", "f32"])
+@pytest.mark.parametrize("rows,K", [(37, 7168), (5, 64), (1, 2048)])
+def test_quantize_bitexact(fmt, src, rows, K):
+    x = _special_rows(_x_f32(rows, K, 7)) if rows >= 3 else _x_f32(rows, K, 7)
+    if src == "bf16":
+        bits = (x.view(np.uint32) + 0x7FFF + ((x.view(np.uint32) >> 16) & 1)) >> 16
+        bits = bits.astype(np.uint16)
+        xin = bf16_dev(bits)
+        xf = synth.bf16_bits_to_f32(bits)
+    else:
+        xin = torch.from_numpy(x).to(dev())
+        xf = x
+    q = ds4g.ds4g_quantize_mx(xin, fmt)
+    ref = oracle.quantize(xf, fmt)
+    got = from_dev(q)
+    assert np.array_equal(got.scales, ref.scales)
+    assert np.array_equal(got.data, ref.data)
+    if fmt == NV:
+        assert np.float32(got.g) == np.float32(ref.g)
+
+
+def test_quantize_nv_given_g():
+    x = _x_f32(16, 512, 8, 3.0)
+    g = np.float32(0.0123)
+    q = ds4g.ds4g_quantize_mx(torch.from_numpy(x).to(dev()), NV, g_in=torch.tensor([g], device=dev()))
+    ref = oracle.quantize(x, NV, g=float(g))
+    got = from_dev(q)
+    assert np.array_equal(got.scales, ref.scales) and np.array_equal(got.data, ref.data)
+
+
+def test_quantize_rejects_bad_k():
+    x = torch.zeros((4, 96), dtype=torch.float32, device=dev())
+    with pytest.raises(ds4g.Ds4gError) as ei:
+        ds4g.ds4g_quantize_mx(x, MX, out=ds4g.Fp4Tensor.empty(4, 96, MX, dev()))
+    assert ei.value.status == 2
+
+
+# ---- routing -------------------------------------------------------------------
+
+@pytest.mark.parametrize("T,E,k,bias", [(16, 8, 2, 0.0), (37, 256, 6, 1.5), (5, 256, 6, 0.0), (3, 1000, 32, 0.0),
+                                        (4, 8, 8, 0.0)])
+def test_route_topk(T, E, k, bias):
+    lg = synth.logits(T, E, 0, bias)
+    lg[0, 3] = lg[0, 5] = lg[0].max() + 1.0     # a tie at the top: lower index first
+    idx, w = ds4g.ds4g_route_topk(torch.from_numpy(lg).to(dev()), k)
+    ridx, rw = oracle.route_topk(lg, k)
+    assert np.array_equal(idx.cpu().numpy(), ridx)
+    assert np.allclose(w.cpu().numpy(), rw, rtol=0, atol=2e-6)
+
+
+# ---- permutation ---------------------------------------------------------------
+
+@pytest.mark.parametrize("T,k,E,fmt", [(16, 2, 8, MX), (1000, 6, 256, MX), (333, 6, 256, NV), (1, 6, 256, MX),
+                                       (2048, 6, 256, MX)])
+def test_permute_bitexact(T, k, E, fmt):
+    K = 256
+    lg = synth.logits(T, E, 0, 1.5)
+    ridx, _ = oracle.route_topk(lg, k)
+    xq = oracle.quantize(_x_f32(T, K, 9), fmt)
+    offs, r2s, s2r, a = ds4g.ds4g_moe_permute(torch.from_numpy(ridx).to(dev()), E, to_dev(xq))
+    roffs, rr2s, rs2r = oracle.moe_permute(ridx, E)
+    assert np.array_equal(offs.cpu().numpy(), roffs)
+    assert np.array_equal(r2s.cpu().numpy(), rr2s)
+    assert np.array_equal(s2r.cpu().numpy(), rs2r)
+    ra = oracle.gather_rows(xq, rr2s, k)
+    got = from_dev(a)
+    assert np.array_equal(got.data, ra.data) and np.array_equal(got.scales, ra.scales)
+    if fmt == NV:
+        assert np.float32(got.g) == np.float32(xq.g)
+
+
+def test_permute_empty():
+    E = 8
+    idx = torch.empty((0, 2), dtype=torch.int32, device=dev())
+    xq = ds4g.Fp4Tensor.empty(0, 64, MX, dev())
+    offs, _, _, _ = ds4g.ds4g_moe_permute(idx, E, xq)
+    assert np.array_equal(offs.cpu().numpy(), np.zeros(E + 1, np.int32))
+
+
+# ---- grouped GEMM ------------------------------------------------------------------
+
+def _grouped_problem(seg, N, K, fmt, stream=11):
+    E = len(seg)
+    offsets = np.concatenate([[0], np.cumsum(seg)]).astype(np.int32)
+    S = int(offsets[-1])
+    a = oracle.quantize(_x_f32(max(S, 1), K, stream)[:S] if S else np.zeros((0, K), np.float32), fmt)
+    wf = synth.normal_f32((E * N, K), 0, stream + 1, 0.02)
+    if fmt == NV:
+        ws = [oracle.quantize(wf[e * N:(e + 1) * N], NV) for e in range(E)]
+        w = oracle.Fp4(np.concatenate([t.data for t in ws]), np.concatenate([t.scales for t in ws]), 1.0, NV)
+        gw = [t.g for t in ws]
+    else:
+        w = oracle.quantize(wf, MX)
+        gw = None
+    return offsets, a, w, gw
+
+
+def _ref_gemm(a, offsets, w, gw, N):
+    """oracle result; NV weights carry one scale per expert"""
+    if a.fmt == MX:
+        return oracle.grouped_gemm(a, offsets, w, N)
+    S = a.data.shape[0]
+    out = np.full((S, N), np.nan)
+    ab = np.full((S, N), np.nan)
+    for e in range(len(offsets) - 1):
+        r0, r1 = offsets[e], offsets[e + 1]
+        if r1 == r0:
+            continue
+        we = oracle.Fp4(w.data[e * N:(e + 1) * N], w.scales[e * N:(e + 1) * N], gw[e], NV)
+        o, s = oracle.expert_gemm_rows(a, np.arange(r0, r1), we, (0, N))
+        out[r0:r1], ab[r0:r1] = o, s
+    return out, ab
+
+
+GEMV_CASES = [([3, 0, 1, 8, 5], 512, 7168), ([1, 1, 1, 1, 1, 1], 256, 2048), ([2, 0, 0, 7], 256, 256),
+              ([8], 4096, 256), ([1], 128, 128)]
+TC_CASES = [([300, 0, 1, 129, 77], 512, 512), ([256, 128], 256, 384), ([9, 200, 0, 0, 1000], 256, 256),
+            ([130], 512, 7168)]
+
+
+@pytest.mark.parametrize("fmt", [MX, NV])
+@pytest.mark.parametrize("case", GEMV_CASES + TC_CASES)
+def test_grouped_gemm_plain(fmt, case):
+    seg, N, K = case
+    offsets, a, w, gw = _grouped_problem(seg, N, K, fmt)
+    max_rows = max(seg)
+    if max_rows > 8 and N % 256:
+        pytest.skip("tensor-core path needs N % 256 == 0")
+    out = ds4g.ds4g_grouped_gemm_fp4(to_dev(a), torch.from_numpy(offsets).to(dev()), len(seg), max_rows,
+                                     to_dev(w, g_per_expert=gw), N)
+    ds4g.ds4g_check_device()
+    ref, ab = _ref_gemm(a, offsets, w, gw, N)
+    assert_gemm_close(out.cpu().numpy(), ref, ab, f"{'gemv' if max_rows <= 8 else 'tcgen05'} {case}")
+
+
+def _h_bound(y1_ref, ab1, I):
+    g, u = y1_ref[:, :I], y1_ref[:, I:]
+    dg = 1e-5 * ab1[:, :I] + 1e-6
+    du = 1e-5 * ab1[:, I:] + 1e-6
+    sig = 1.0 / (1.0 + np.exp(-g))
+    dsilu = sig * (1 + g * (1 - sig))
+    h = g * sig * u
+    return h, np.abs(dsilu) * np.abs(u) * dg + np.abs(g * sig) * du + 8 * np.abs(h) * 2.0 ** -24 + 1e-30
+
+
+@pytest.mark.parametrize("fmt", [MX, NV])
+@pytest.mark.parametrize("case", [([3, 0, 1, 8, 5], 256, 7168), ([300, 0, 1, 129, 77], 256, 512),
+                                  ([2, 1], 64, 256), ([131], 128, 2048)])
+def test_fc1_fused_swiglu_requant(fmt, case):
+    seg, I, K = case
+    offsets, a, w, gw = _grouped_problem(seg, 2 * I, K, fmt, stream=21)
+    S = int(offsets[-1])
+    max_rows = max(seg)
+    hq = ds4g.Fp4Tensor.empty(S, I, fmt, dev())
+    g_h = G_H
+    if fmt == NV:
+        hq.g.fill_(g_h)
+    hdbg = torch.empty((S, I), dtype=torch.float32, device=dev())
+    ds4g.ds4g_grouped_gemm_fp4(to_dev(a), torch.from_numpy(offsets).to(dev()), len(seg), max_rows,
+                               to_dev(w, g_per_expert=gw), 2 * I, ds4g.EPI_SWIGLU_REQUANT, out_q=hq, h_debug=hdbg)
+    ds4g.ds4g_check_device()
+    y1, ab1 = _ref_gemm(a, offsets, w, gw, 2 * I)
+    h_ref, dh = _h_bound(y1, ab1, I)
+    h_gpu = hdbg.cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(h_gpu - h_ref) <= dh * 1.000001), "h outside its error bound"
+    check_requant(from_dev(hq), h_ref, dh, fmt, g=g_h)
+
+
+@pytest.mark.parametrize("fmt", [MX, NV])
+def test_swiglu_requant(fmt):
+    rows, I = 70, 256
+    y1 = synth.normal_f32((rows, 2 * I), 0, 31, 2.0)
+    g_h = G_H
+    hdbg = torch.empty((rows, I), dtype=torch.float32, device=dev())
+    hq = ds4g.ds4g_swiglu_requant(torch.from_numpy(y1).to(dev()), fmt, h_debug=hdbg,
+                                  g_h=torch.tensor([g_h], device=dev()) if fmt == NV else None)
+    h_ref = oracle.swiglu(y1).astype(np.float64)
+    h_gpu = hdbg.cpu().numpy().astype(np.float64)
+    dh = 4 * np.abs(h_ref) * 2.0 ** -23 + 1e-38
+    assert np.all(np.abs(h_gpu - h_ref) <= dh)
+    check_requant(from_dev(hq), h_ref, dh, fmt, g=g_h, min_exact=0.9999)
+
+
+# ---- combine -----------------------------------------------------------------------
+
+def test_combine():
+    T, k, d, E = 33, 6, 7168, 256
+    lg = synth.logits(T, E, 0)
+    ridx, rw = oracle.route_topk(lg, k)
+    _, _, s2r = oracle.moe_permute(ridx, E)
+    y2 = synth.normal_f32((T * k, d), 0, 41, 3.0)
+    w32 = rw.astype(np.float32)
+    out = ds4g.ds4g_moe_combine(torch.from_numpy(y2).to(dev()), torch.from_numpy(s2r).to(dev()),
+                                torch.from_numpy(w32).to(dev()))
+    ref = oracle.moe_combine(y2.astype(np.float64), s2r, w32.astype(np.float64))
+    absref = oracle.moe_combine(np.abs(y2.astype(np.float64)), s2r, np.abs(w32.astype(np.float64)))
+    assert np.all(np.abs(out.cpu().numpy() - ref) <= 1e-6 * absref + 1e-7)
+
+
+# ---- full layer --------------------------------------------------------------------
+
+@pytest.mark.parametrize("fused", [True, False])
+def test_layer_tiny(fused):
+    from synth import workloads
+    from block_scaled_fp4_topk_b200.layer import MoeLayer
+    wl = workloads.WORKLOADS["tiny"]
+    w1, w2 = MoeLayer.synthetic_weights(wl.E, wl.d, wl.I, wl.fmt, device=dev())
+    layer = MoeLayer(w1, w2, wl.E, wl.k, wl.d, wl.I, wl.fmt, fused=fused)
+    xb = workloads.host_x_bits(wl)
+    lg = workloads.host_logits(wl)
+    out = layer.forward(bf16_dev(xb), torch.from_numpy(lg).to(dev())).cpu().numpy()
+    ds4g.ds4g_check_device()
+    W1 = oracle.quantize(np.concatenate([workloads.host_w1(wl, e) for e in range(wl.E)]), MX)
+    W2 = oracle.quantize(np.concatenate([workloads.host_w2(wl, e) for e in range(wl.E)]), MX)
+    assert np.array_equal(from_dev(w1).data, W1.data) and np.array_equal(from_dev(w2).scales, W2.scales)
+    res = oracle.moe_layer(synth.bf16_bits_to_f32(xb), lg, W1, W2, wl.k, MX)
+    rel = np.linalg.norm(out - res["out"]) / np.linalg.norm(res["out"])
+    assert rel <= 1e-2, rel
