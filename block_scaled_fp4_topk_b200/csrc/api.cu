@@ -131,7 +131,9 @@ ds4g_status ds4g_grouped_gemm_fp4(const ds4g_fp4* a, const int32_t* offsets, int
     if (st != DS4G_OK) return st;
     st = check_fp4(w, (int64_t)E * N, K, fmt, true);
     if (st != DS4G_OK) return st;
-    const bool gemv = max_rows_per_expert <= 8;
+    // kernel choice: the weight-streaming GEMV for decode-sized segments (and
+    // for K the tensor-core kernel's scale loads cannot tile), else tcgen05
+    const bool gemv = max_rows_per_expert <= 8 || !gemm_tc_supports(fmt, K);
     const int64_t Sr = a->rows;
     if (epilogue == DS4G_EPI_NONE) {
         if (Sr > 0 && (!out || !aligned16(out))) return DS4G_ERR_INVALID_ARG;
@@ -144,7 +146,6 @@ ds4g_status ds4g_grouped_gemm_fp4(const ds4g_fp4* a, const int32_t* offsets, int
         if (st != DS4G_OK) return st;
         if (h_debug && !aligned16(h_debug)) return DS4G_ERR_INVALID_ARG;
     }
-    if (!gemv && K % 128 != 0) return DS4G_ERR_SHAPE;
     if ((int64_t)E * N > 0x7FFFFFFF) return DS4G_ERR_SHAPE;
     GemmArgs g;
     g.a_data = a->data;

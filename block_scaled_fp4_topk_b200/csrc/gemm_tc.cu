@@ -10,17 +10,20 @@
 // same math is tcgen05.mma kind::mxf4 (.block32, UE8M0) / kind::mxf4nvf4
 // (.block16, UE4M3) with the accumulator in tensor memory.
 //
-// Design (one persistent CTA per SM, 256 threads, warp-specialised):
-//   warp 0  TMA producer: packed FP4 tiles of A (128 rows x 256 K) and W
-//           (256 rows x 256 K) -> 128B-swizzled shared memory, 4 stages
-//   warp 1  MMA issuer: scale factors shared -> TMEM with tcgen05.cp
-//           (32x128b.warpx4), 4 x tcgen05.mma (M128 N256 K64) per stage,
-//           tcgen05.commit releases the stage / publishes the accumulator
-//   warp 2  scale-factor loader: cp.async of the row-major scale bytes into
-//           the 32-line x 16-byte chunk order tcgen05.cp expects
-//   warp 3  TMEM allocator
-//   warps 4-7  epilogue: tcgen05.ld of the fp32 accumulator (thread i owns
-//           tile row i), then either the fp32 store or SwiGLU + requantise
+// Design (one persistent CTA per SM, 384 threads, warp-specialised):
+//   warp 0   TMA producer: packed FP4 tiles of A (128 rows x 256 K) and W
+//            (256 rows x 256 K) into 128B-swizzled shared memory (4 stages),
+//            and the row-major scale bytes of 512 K (two stages) of both as
+//            16 / 32-byte row boxes (2 scale stages)
+//   warp 1   MMA issuer: the stage's scale words shared -> TMEM with
+//            tcgen05.cp (32x128b.warpx4), 4 x tcgen05.mma (M128 N256 K64),
+//            tcgen05.commit releases the stage / publishes the accumulator
+//   warp 2   scale transposer: rewrites each scale stage in place from row
+//            order into the 32-line x 16-byte chunks tcgen05.cp expects
+//   warp 3   TMEM allocator
+//   warps 4-11  epilogue: two warps per TMEM lane quarter, each reading half
+//            of the tile's columns with tcgen05.ld (thread = tile row), then
+//            the fp32 store or SwiGLU + requantisation
 // Tiles (expert, n-tile, m-tile) are enumerated on the device from the
 // expert offsets (no host read-back); every CTA walks tile t, t + #CTAs, ...
 // Every mbarrier wait is bounded: past ~4 s it records kErrWaitTimeout in
@@ -40,7 +43,9 @@ constexpr int BN = 256;            // tile columns (weight rows)
 constexpr int BKB = 128;           // bytes of K per stage per row (256 FP4)
 constexpr int BK = 256;            // K elements per stage
 constexpr int STAGES = 4;
-constexpr int kThreads = 256;
+constexpr int SF_STAGES = 2;       // scale stages, each covering two K stages (512 K)
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 32 * (4 + kEpiWarps);
 constexpr int A_BYTES = BM * BKB;  // 16 KB
 constexpr int B_BYTES = BN * BKB;  // 32 KB
 constexpr int kTmemCols = 512;
@@ -48,17 +53,17 @@ constexpr int kColAcc = 0;
 constexpr int kColSFA = 256;
 constexpr int kColSFB = 272;
 constexpr int kMaxE = 1024;
-constexpr int kSfLag = 2;          // stages the SF loader keeps in flight
 constexpr unsigned long long kWaitNs = 4000000000ull;
 
 template <int FMT>
 struct Cfg {
-    static constexpr int WORDS = (FMT == DS4G_MXFP4) ? 2 : 4;   // 4-scale words per row per stage
-    static constexpr int SFA_BYTES = WORDS * 512;
-    static constexpr int SFB_BYTES = WORDS * 1024;
-    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-    static constexpr int K_PER_WORD = (FMT == DS4G_MXFP4) ? 128 : 64;
-    static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + 256 + (kMaxE + 1) * 4;
+    static constexpr int WPS = (FMT == DS4G_MXFP4) ? 2 : 4;         // 4-scale words per row per K stage
+    static constexpr int SF_ROW = 2 * WPS * 4;                       // scale bytes per row per scale stage
+    static constexpr int SFA_BYTES = BM * SF_ROW;                    // one scale stage of A
+    static constexpr int SFB_BYTES = BN * SF_ROW;                    // one scale stage of W
+    static constexpr int DATA_BYTES = STAGES * (A_BYTES + B_BYTES);
+    static constexpr int SF_BYTES = SF_STAGES * (SFA_BYTES + SFB_BYTES);
+    static constexpr size_t SMEM = 1024 + (size_t)DATA_BYTES + SF_BYTES + 256 + (kMaxE + 1) * 4;
 };
 
 // ---- PTX wrappers ----------------------------------------------------------
@@ -96,10 +101,14 @@ __device__ __forceinline__ bool mbar_try(uint32_t a, uint32_t parity)
     return ok != 0;
 }
 
-// bounded wait; false when it gave up (or another role already gave up)
+// bounded wait; false when it gave up (or another role already gave up).
+// Spins without touching the timer first, so a wait that completes within a
+// few thousand polls costs nothing extra.
 __device__ __forceinline__ bool mbar_wait(uint32_t a, uint32_t parity, volatile int* abort_flag)
 {
-    if (mbar_try(a, parity)) return true;
+#pragma unroll 1
+    for (int i = 0; i < 4096; ++i)
+        if (mbar_try(a, parity)) return true;
     const uint64_t t0 = globaltimer();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try(a, parity)) return true;
@@ -126,14 +135,6 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
         ::"r"(dst), "l"((uint64_t)map), "r"(mbar), "r"(x), "r"(y)
         : "memory");
 }
-
-__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src, uint32_t src_size)
-{
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(src_size) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 // shared-memory matrix descriptor (tcgen05): K-major, 128-byte swizzle,
 // 8-row core groups 1024 bytes apart
@@ -215,6 +216,35 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v)
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// in-place transposition of one scale stage of `rows` rows (multiple of 128)
+// from row order [rows][words * 4 bytes] to the tcgen05.cp chunk order: for
+// 128-row group g and word c, a 512-byte chunk at ((c * groups) + g) * 512
+// whose 16-byte line l holds word c of rows l, l + 32, l + 64, l + 96.
+template <int WORDS, int GROUPS>
+__device__ __forceinline__ void sf_transpose(uint8_t* base, int lane)
+{
+    uint32_t v[GROUPS][4][WORDS];
+#pragma unroll
+    for (int g = 0; g < GROUPS; ++g)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint32_t* row = reinterpret_cast<const uint32_t*>(base + (size_t)(g * 128 + q * 32 + lane) * WORDS * 4);
+#pragma unroll
+            for (int c = 0; c < WORDS; c += 4) {
+                const uint4 x = *reinterpret_cast<const uint4*>(row + c);
+                v[g][q][c] = x.x; v[g][q][c + 1] = x.y; v[g][q][c + 2] = x.z; v[g][q][c + 3] = x.w;
+            }
+        }
+    __syncwarp();
+#pragma unroll
+    for (int g = 0; g < GROUPS; ++g)
+#pragma unroll
+        for (int c = 0; c < WORDS; ++c)
+            *reinterpret_cast<uint4*>(base + (size_t)((c * GROUPS + g) * 512 + lane * 16)) =
+                make_uint4(v[g][0][c], v[g][1][c], v[g][2][c], v[g][3][c]);
+    __syncwarp();
+}
+
 // ---- tile enumeration --------------------------------------------------------
 struct Tile {
     int e;        // expert
@@ -242,59 +272,76 @@ __device__ __forceinline__ Tile tile_of(int64_t t, const int32_t* prefix, const 
     return r;
 }
 
+// first weight rows of the two 128-row halves of the W tile
+template <int EPI>
+__device__ __forceinline__ void w_rows(const Tile& tl, int N, int I, int64_t& y0, int64_t& y1)
+{
+    const int64_t wbase = (int64_t)tl.e * N;
+    if (EPI == DS4G_EPI_SWIGLU_REQUANT) {
+        y0 = wbase + (int64_t)tl.nt * 128;          // gate rows
+        y1 = wbase + I + (int64_t)tl.nt * 128;      // up rows
+    } else {
+        y0 = wbase + (int64_t)tl.nt * BN;
+        y1 = y0 + 128;
+    }
+}
+
 template <int FMT, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
-k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b, const GemmArgs p)
+k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+          const __grid_constant__ CUtensorMap map_sfa, const __grid_constant__ CUtensorMap map_sfb, const GemmArgs p)
 {
     using C = Cfg<FMT>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;
     uint8_t* sB = sA + STAGES * A_BYTES;
-    uint8_t* sSFA = sB + STAGES * B_BYTES;
-    uint8_t* sSFB = sSFA + STAGES * C::SFA_BYTES;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sSFB + STAGES * C::SFB_BYTES);
-    uint64_t* full = bars;                    // [STAGES]
-    uint64_t* empty = bars + STAGES;          // [STAGES]
-    uint64_t* tmem_full = bars + 2 * STAGES;
+    uint8_t* sSFA = sB + STAGES * B_BYTES;                 // [SF_STAGES][SFA_BYTES]
+    uint8_t* sSFB = sSFA + SF_STAGES * C::SFA_BYTES;       // [SF_STAGES][SFB_BYTES]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sSFB + SF_STAGES * C::SFB_BYTES);
+    uint64_t* full = bars;                                 // [STAGES]  TMA data landed
+    uint64_t* empty = full + STAGES;                       // [STAGES]  MMAs done with the data
+    uint64_t* sf_full = empty + STAGES;                    // [SF_STAGES] TMA scales landed
+    uint64_t* sf_ready = sf_full + SF_STAGES;              // [SF_STAGES] scales transposed
+    uint64_t* sf_empty = sf_ready + SF_STAGES;             // [SF_STAGES] MMAs done with the scales
+    uint64_t* tmem_full = sf_empty + SF_STAGES;
     uint64_t* tmem_empty = tmem_full + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tmem_empty + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int32_t* total_tiles = reinterpret_cast<int32_t*>(tmem_slot + 2);
-    int32_t* prefix = reinterpret_cast<int32_t*>(smem + STAGES * C::STAGE_BYTES + 256);
+    int32_t* prefix = reinterpret_cast<int32_t*>(smem + C::DATA_BYTES + C::SF_BYTES + 256);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int E = p.E;
     const int64_t K = p.K;
     const int nks = (int)ceil_div(K, BK);
+    const int npairs = (nks + 1) / 2;
     const int I = p.N / 2;
     const int n_tiles = (EPI == DS4G_EPI_SWIGLU_REQUANT) ? (I / 128) : (p.N / BN);
 
     // ---- prologue
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(smem_u32(&full[s]), 2);
+            mbar_init(smem_u32(&full[s]), 1);
             mbar_init(smem_u32(&empty[s]), 1);
         }
+        for (int r = 0; r < SF_STAGES; ++r) {
+            mbar_init(smem_u32(&sf_full[r]), 1);
+            mbar_init(smem_u32(&sf_ready[r]), 1);
+            mbar_init(smem_u32(&sf_empty[r]), 1);
+        }
         mbar_init(smem_u32(tmem_full), 1);
-        mbar_init(smem_u32(tmem_empty), 128);
+        mbar_init(smem_u32(tmem_empty), 32 * kEpiWarps);
         *abort_flag = 0;
         fence_barrier_init();
     }
     if (warp == 0) {
         // tiles per expert, exclusive scan by one warp
         const int per = (E + 31) / 32;
-        int32_t local[32];
         int32_t sum = 0;
         for (int i = 0; i < per; ++i) {
             const int e = lane * per + i;
-            int32_t v = 0;
-            if (e < E) {
-                const int64_t rows = (int64_t)p.offsets[e + 1] - p.offsets[e];
-                v = (int32_t)(ceil_div(rows, BM) * n_tiles);
-            }
-            local[i < 32 ? i : 31] = v;
-            sum += v;
+            if (e < E) sum += (int32_t)(ceil_div((int64_t)p.offsets[e + 1] - p.offsets[e], BM) * n_tiles);
         }
         int32_t incl = sum;
 #pragma unroll
@@ -305,8 +352,10 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
         int32_t run = incl - sum;
         for (int i = 0; i < per; ++i) {
             const int e = lane * per + i;
-            if (e < E) prefix[e] = run;
-            run += local[i < 32 ? i : 31];
+            if (e < E) {
+                prefix[e] = run;
+                run += (int32_t)(ceil_div((int64_t)p.offsets[e + 1] - p.offsets[e], BM) * n_tiles);
+            }
         }
         if (lane == 31) {
             prefix[E] = incl;
@@ -320,6 +369,8 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
         if (lane == 0) {
             asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&map_a) : "memory");
             asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&map_b) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&map_sfa) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&map_sfb) : "memory");
         }
     }
     if (warp == 3) {
@@ -337,36 +388,40 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
     if (warp == 0) {
         // ================= TMA producer =================
         if (lane == 0) {
-            uint32_t it = 0;
+            uint32_t it = 0, sit = 0;
             bool ok = true;
             for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
                 const Tile tl = tile_of(t, prefix, p.offsets, E, n_tiles);
-                const int64_t wbase = (int64_t)tl.e * p.N;
-                int yb0, yb1;
-                if (EPI == DS4G_EPI_SWIGLU_REQUANT) {
-                    yb0 = (int)(wbase + (int64_t)tl.nt * 128);
-                    yb1 = (int)(wbase + I + (int64_t)tl.nt * 128);
-                } else {
-                    yb0 = (int)(wbase + (int64_t)tl.nt * BN);
-                    yb1 = yb0 + 128;
-                }
+                int64_t y0, y1;
+                w_rows<EPI>(tl, p.N, I, y0, y1);
                 for (int ks = 0; ks < nks; ++ks, ++it) {
+                    if ((ks & 1) == 0) {
+                        const int r = sit % SF_STAGES;
+                        if (!mbar_wait(smem_u32(&sf_empty[r]), ((sit / SF_STAGES) & 1) ^ 1, abort_flag)) { ok = false; break; }
+                        const uint32_t fb = smem_u32(&sf_full[r]);
+                        mbar_arrive_tx(fb, C::SFA_BYTES + C::SFB_BYTES);
+                        const int x = (ks >> 1) * C::SF_ROW;
+                        tma_load_2d(smem_u32(sSFA + r * C::SFA_BYTES), &map_sfa, fb, x, (int)tl.m0);
+                        tma_load_2d(smem_u32(sSFB + r * C::SFB_BYTES), &map_sfb, fb, x, (int)y0);
+                        tma_load_2d(smem_u32(sSFB + r * C::SFB_BYTES + C::SFB_BYTES / 2), &map_sfb, fb, x, (int)y1);
+                        ++sit;
+                    }
                     const int s = it % STAGES;
-                    const uint32_t ph = (it / STAGES) & 1;
-                    if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1, abort_flag)) { ok = false; break; }
+                    if (!mbar_wait(smem_u32(&empty[s]), ((it / STAGES) & 1) ^ 1, abort_flag)) { ok = false; break; }
                     const uint32_t fb = smem_u32(&full[s]);
                     mbar_arrive_tx(fb, A_BYTES + B_BYTES);
                     tma_load_2d(smem_u32(sA + s * A_BYTES), &map_a, fb, ks * BKB, (int)tl.m0);
-                    tma_load_2d(smem_u32(sB + s * B_BYTES), &map_b, fb, ks * BKB, yb0);
-                    tma_load_2d(smem_u32(sB + s * B_BYTES + B_BYTES / 2), &map_b, fb, ks * BKB, yb1);
+                    tma_load_2d(smem_u32(sB + s * B_BYTES), &map_b, fb, ks * BKB, (int)y0);
+                    tma_load_2d(smem_u32(sB + s * B_BYTES + B_BYTES / 2), &map_b, fb, ks * BKB, (int)y1);
                 }
             }
             if (!ok) {
-                // let copies already issued land before the CTA goes away
-                for (uint32_t j = (it > STAGES ? it - STAGES : 0); j < it; ++j) {
-                    volatile int dummy = 0;
-                    mbar_wait(smem_u32(&full[j % STAGES]), (j / STAGES) & 1, &dummy);
-                }
+                // let the copies already issued land before the CTA goes away
+                volatile int never = 0;
+                for (uint32_t j = (it > STAGES ? it - STAGES : 0); j < it; ++j)
+                    mbar_wait(smem_u32(&full[j % STAGES]), (j / STAGES) & 1, &never);
+                for (uint32_t j = (sit > SF_STAGES ? sit - SF_STAGES : 0); j < sit; ++j)
+                    mbar_wait(smem_u32(&sf_full[j % SF_STAGES]), (j / SF_STAGES) & 1, &never);
             }
         }
         __syncwarp();
@@ -374,24 +429,28 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
         // ================= MMA issuer =================
         if (lane == 0) {
             const uint32_t ibase = idesc_base<FMT>();
-            uint32_t it = 0, tcount = 0;
+            uint32_t it = 0, sit = 0, tcount = 0;
             bool ok = true;
             for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++tcount) {
                 if (!mbar_wait(smem_u32(tmem_empty), (tcount & 1) ^ 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 for (int ks = 0; ks < nks; ++ks, ++it) {
+                    const int r = sit % SF_STAGES;
+                    if ((ks & 1) == 0) {
+                        if (!mbar_wait(smem_u32(&sf_ready[r]), (sit / SF_STAGES) & 1, abort_flag)) { ok = false; break; }
+                    }
                     const int s = it % STAGES;
-                    const uint32_t ph = (it / STAGES) & 1;
-                    if (!mbar_wait(smem_u32(&full[s]), ph, abort_flag)) { ok = false; break; }
+                    if (!mbar_wait(smem_u32(&full[s]), (it / STAGES) & 1, abort_flag)) { ok = false; break; }
                     tc_fence_after();
-                    // scale factors of this stage -> TMEM
-                    const uint32_t sfa_s = smem_u32(sSFA + s * C::SFA_BYTES);
-                    const uint32_t sfb_s = smem_u32(sSFB + s * C::SFB_BYTES);
+                    // this K stage's scale words -> TMEM
+                    const int w0 = (ks & 1) * C::WPS;
+                    const uint32_t sfa_s = smem_u32(sSFA + r * C::SFA_BYTES);
+                    const uint32_t sfb_s = smem_u32(sSFB + r * C::SFB_BYTES);
 #pragma unroll
-                    for (int c = 0; c < C::WORDS; ++c) {
-                        utccp(tmem + kColSFA + 4 * c, desc_sf(sfa_s + c * 512));
-                        utccp(tmem + kColSFB + 8 * c, desc_sf(sfb_s + c * 1024));
-                        utccp(tmem + kColSFB + 8 * c + 4, desc_sf(sfb_s + c * 1024 + 512));
+                    for (int c = 0; c < C::WPS; ++c) {
+                        utccp(tmem + kColSFA + 4 * c, desc_sf(sfa_s + (w0 + c) * 512));
+                        utccp(tmem + kColSFB + 8 * c, desc_sf(sfb_s + ((w0 + c) * 2 + 0) * 512));
+                        utccp(tmem + kColSFB + 8 * c + 4, desc_sf(sfb_s + ((w0 + c) * 2 + 1) * 512));
                     }
                     const int64_t krem = K - (int64_t)ks * BK;
                     const int nmma = krem >= BK ? 4 : (int)(krem / 64);
@@ -408,6 +467,10 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
                         }
                     }
                     tc_commit(smem_u32(&empty[s]));
+                    if ((ks & 1) == 1 || ks == nks - 1) {
+                        tc_commit(smem_u32(&sf_empty[r]));
+                        ++sit;
+                    }
                 }
                 if (!ok) break;
                 tc_commit(smem_u32(tmem_full));
@@ -415,69 +478,27 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
         }
         __syncwarp();
     } else if (warp == 2) {
-        // ================= scale-factor loader =================
-        uint32_t it = 0, pending_from = 0;
-        bool ok = true;
-        const int64_t sa_row = K / ((FMT == DS4G_MXFP4) ? 32 : 16);   // scale bytes per row
-        for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-            const Tile tl = tile_of(t, prefix, p.offsets, E, n_tiles);
-            const int64_t wbase = (int64_t)tl.e * p.N;
-            for (int ks = 0; ks < nks; ++ks, ++it) {
-                const int s = it % STAGES;
-                const uint32_t ph = (it / STAGES) & 1;
+        // ================= scale transposer =================
+        uint32_t sit = 0;
+        for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x) {
+            bool ok = true;
+            for (int pr = 0; pr < npairs; ++pr, ++sit) {
+                const int r = sit % SF_STAGES;
                 bool w_ok = true;
-                if (lane == 0) w_ok = mbar_wait(smem_u32(&empty[s]), ph ^ 1, abort_flag);
-                w_ok = __shfl_sync(0xffffffffu, w_ok ? 1 : 0, 0) != 0;
-                if (!w_ok) { ok = false; break; }
-                const int64_t krem = K - (int64_t)ks * BK;
-                const int nw = (int)min((int64_t)C::WORDS, krem / C::K_PER_WORD);
-                const int64_t kb = (int64_t)ks * (C::WORDS * 4);          // first scale byte of the stage
-                const uint32_t sfa_s = smem_u32(sSFA + s * C::SFA_BYTES);
-                const uint32_t sfb_s = smem_u32(sSFB + s * C::SFB_BYTES);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int64_t row = tl.m0 + lane + 32 * q;
-                    const bool valid = row < p.S;
-                    for (int c = 0; c < nw; ++c) {
-                        const uint8_t* src = valid ? (p.a_scales + row * sa_row + kb + 4 * c) : p.a_scales;
-                        cp_async4(sfa_s + c * 512 + lane * 16 + q * 4, src, valid ? 4u : 0u);
-                    }
-                }
-#pragma unroll
-                for (int g = 0; g < 2; ++g) {
-                    int64_t brow0;
-                    if (EPI == DS4G_EPI_SWIGLU_REQUANT) brow0 = wbase + (g ? I : 0) + (int64_t)tl.nt * 128;
-                    else brow0 = wbase + (int64_t)tl.nt * BN + 128 * g;
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const int64_t row = brow0 + lane + 32 * q;
-                        for (int c = 0; c < nw; ++c)
-                            cp_async4(sfb_s + c * 1024 + g * 512 + lane * 16 + q * 4,
-                                      p.w_scales + row * sa_row + kb + 4 * c, 4u);
-                    }
-                }
-                cp_async_commit();
-                if (it >= pending_from + kSfLag) {
-                    cp_async_wait<kSfLag>();
-                    fence_proxy_async();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(smem_u32(&full[(it - kSfLag) % STAGES]));
-                }
-                if (it + 1 < pending_from + kSfLag) { /* still filling the lag window */ }
+                if (lane == 0) w_ok = mbar_wait(smem_u32(&sf_full[r]), (sit / SF_STAGES) & 1, abort_flag);
+                if (!__shfl_sync(0xffffffffu, w_ok ? 1 : 0, 0)) { ok = false; break; }
+                sf_transpose<2 * C::WPS, 1>(sSFA + r * C::SFA_BYTES, lane);
+                sf_transpose<2 * C::WPS, 2>(sSFB + r * C::SFB_BYTES, lane);
+                fence_proxy_async();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&sf_ready[r]));
             }
+            if (!ok) break;
         }
-        // publish the stages still in flight
-        cp_async_wait<0>();
-        fence_proxy_async();
-        __syncwarp();
-        if (lane == 0) {
-            const uint32_t first = it >= kSfLag ? it - kSfLag : 0;
-            for (uint32_t j = first; j < it; ++j) mbar_arrive(smem_u32(&full[j % STAGES]));
-        }
-        (void)pending_from;
     } else if (warp >= 4) {
         // ================= epilogue =================
-        const int ew = warp - 4;
+        const int q = warp & 3;                 // TMEM lane quarter this warp may access
+        const int half = (warp - 4) >> 2;       // which half of the tile's columns
         uint32_t tcount = 0;
         const float gh = (FMT == DS4G_NVFP4 && EPI == DS4G_EPI_SWIGLU_REQUANT) ? *p.oq_g : 1.0f;
         for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, ++tcount) {
@@ -485,16 +506,17 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
             tc_fence_after();
             const Tile tl = tile_of(t, prefix, p.offsets, E, n_tiles);
             const float gscale = (FMT == DS4G_NVFP4) ? __fmul_rn(p.a_g[0], p.w_g[tl.e]) : 1.0f;
-            const int64_t row = tl.m0 + 32 * ew + lane;
+            const int64_t row = tl.m0 + 32 * q + lane;
             const bool valid = row < tl.end;
-            const uint32_t tbase = tmem + kColAcc + ((uint32_t)(32 * ew) << 16);
+            const uint32_t tbase = tmem + kColAcc + ((uint32_t)(32 * q) << 16);
             if (EPI == DS4G_EPI_NONE) {
 #pragma unroll 1
-                for (int c8 = 0; c8 < BN / 32; ++c8) {
+                for (int c8 = 0; c8 < 4; ++c8) {
+                    const int col = half * 128 + 32 * c8;
                     float v[32];
-                    tmem_ld32(tbase + 32 * c8, v);
+                    tmem_ld32(tbase + col, v);
                     if (valid) {
-                        float4* dst = reinterpret_cast<float4*>(p.out + row * p.N + (int64_t)tl.nt * BN + 32 * c8);
+                        float4* dst = reinterpret_cast<float4*>(p.out + row * p.N + (int64_t)tl.nt * BN + col);
 #pragma unroll
                         for (int i = 0; i < 8; ++i)
                             dst[i] = make_float4(v[4 * i] * gscale, v[4 * i + 1] * gscale, v[4 * i + 2] * gscale,
@@ -503,11 +525,12 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
                 }
             } else {
 #pragma unroll 1
-                for (int j = 0; j < 4; ++j) {
+                for (int j = 0; j < 2; ++j) {
+                    const int gcol = half * 64 + 32 * j;            // gate column within the tile
                     float gv[32], uv[32];
-                    tmem_ld32(tbase + 32 * j, gv);
-                    tmem_ld32(tbase + 128 + 32 * j, uv);
-                    const int64_t col0 = (int64_t)tl.nt * 128 + 32 * j;
+                    tmem_ld32(tbase + gcol, gv);
+                    tmem_ld32(tbase + 128 + gcol, uv);
+                    const int64_t col0 = (int64_t)tl.nt * 128 + gcol;
                     float h[32];
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
@@ -591,46 +614,58 @@ static PFN_encodeTiled get_encode()
     return fn;
 }
 
-// 2-D map over a packed FP4 matrix [rows][K/2] bytes, box 128 bytes x 128 rows
-static bool make_map(CUtensorMap* m, const uint8_t* base, int64_t rows, int64_t K)
+// 2-D byte map over [rows][width] bytes with a box of box_w bytes x 128 rows
+static bool make_map(CUtensorMap* m, const uint8_t* base, int64_t rows, int64_t width, uint32_t box_w, bool swizzle)
 {
     PFN_encodeTiled enc = get_encode();
     if (!enc) return false;
-    cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
-    cuuint32_t box[2] = {128, 128};
+    cuuint64_t dims[2] = {(cuuint64_t)width, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)width};
+    cuuint32_t box[2] = {box_w, 128};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(base), dims, strides, box, estr,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
 template <int FMT, int EPI>
-static cudaError_t run_tc(const GemmArgs& a, const CUtensorMap& ma, const CUtensorMap& mb, cudaStream_t st)
+static cudaError_t run_tc(const GemmArgs& a, cudaStream_t st)
 {
+    using C = tc::Cfg<FMT>;
+    const int blk = (FMT == DS4G_MXFP4) ? 32 : 16;
+    CUtensorMap ma, mb, msa, msb;
+    if (!make_map(&ma, a.a_data, a.S, a.K / 2, 128, true) ||
+        !make_map(&mb, a.w_data, (int64_t)a.E * a.N, a.K / 2, 128, true) ||
+        !make_map(&msa, a.a_scales, a.S, a.K / blk, C::SF_ROW, false) ||
+        !make_map(&msb, a.w_scales, (int64_t)a.E * a.N, a.K / blk, C::SF_ROW, false))
+        return cudaErrorInvalidValue;
     auto kern = tc::k_gemm_tc<FMT, EPI>;
-    const size_t shm = tc::Cfg<FMT>::SMEM;
+    const size_t shm = C::SMEM;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)shm);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = kNumSMs;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    kern<<<sms, tc::kThreads, shm, st>>>(ma, mb, a);
+    kern<<<sms, tc::kThreads, shm, st>>>(ma, mb, msa, msb, a);
     return cudaGetLastError();
+}
+
+bool gemm_tc_supports(int fmt, int64_t K)
+{
+    // the scale rows are loaded by TMA in 16 (MX) / 32 (NV) byte boxes, whose
+    // row pitch K / block must be a multiple of 16 bytes
+    return fmt == DS4G_MXFP4 ? (K % 512 == 0) : (K % 256 == 0);
 }
 
 cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st)
 {
     if (a.S == 0) return cudaSuccess;
-    if (a.E > tc::kMaxE) return cudaErrorInvalidValue;
-    CUtensorMap ma, mb;
-    if (!make_map(&ma, a.a_data, a.S, a.K) || !make_map(&mb, a.w_data, (int64_t)a.E * a.N, a.K))
-        return cudaErrorInvalidValue;
+    if (a.E > tc::kMaxE || !gemm_tc_supports(a.fmt, a.K)) return cudaErrorInvalidValue;
     if (a.fmt == DS4G_MXFP4)
-        return a.epilogue == DS4G_EPI_NONE ? run_tc<DS4G_MXFP4, DS4G_EPI_NONE>(a, ma, mb, st)
-                                           : run_tc<DS4G_MXFP4, DS4G_EPI_SWIGLU_REQUANT>(a, ma, mb, st);
-    return a.epilogue == DS4G_EPI_NONE ? run_tc<DS4G_NVFP4, DS4G_EPI_NONE>(a, ma, mb, st)
-                                       : run_tc<DS4G_NVFP4, DS4G_EPI_SWIGLU_REQUANT>(a, ma, mb, st);
+        return a.epilogue == DS4G_EPI_NONE ? run_tc<DS4G_MXFP4, DS4G_EPI_NONE>(a, st)
+                                           : run_tc<DS4G_MXFP4, DS4G_EPI_SWIGLU_REQUANT>(a, st);
+    return a.epilogue == DS4G_EPI_NONE ? run_tc<DS4G_NVFP4, DS4G_EPI_NONE>(a, st)
+                                       : run_tc<DS4G_NVFP4, DS4G_EPI_SWIGLU_REQUANT>(a, st);
 }
 
 }  // namespace ds4g
