@@ -248,15 +248,16 @@ def run_ours(args, rank, world, local_rank):
                                    out=b["y2"])
         ds4g.ds4g_moe_combine(b["y2"], b["s2r"][:wl.S], b["w"], out=b["out"])
 
+    # the layer step as one CUDA graph (all seven library calls, no host work)
+    graph, gout = layer.capture(x, lg)
     for _ in range(args.warmup):
-        step()
+        graph.replay()
     torch.cuda.synchronize()
     ds4g.ds4g_check_device()
     offsets = b["offsets"].cpu().numpy()
     alg = algorithmic(wl, offsets)
     launches_per_step = (1 + (1 if wl.fmt == 0 else 3) + 4 + 1 + 1 + 1)
 
-    fc1_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
@@ -265,15 +266,22 @@ def run_ours(args, rank, world, local_rank):
                       int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local_rank])) as clk:
         e0.record(st)
         for i in range(args.steps):
-            step(fc1_ev[i])
+            graph.replay()
         e1.record(st)
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     ds4g.ds4g_check_device()
     ms_total = e0.elapsed_time(e1)
-    fc1_ms = float(np.mean([a.elapsed_time(c) for a, c in fc1_ev]))
     ms_total = max_over_ranks(ms_total, world, dev)
+
+    # the dominant kernel (FC1), timed with CUDA events on the launching
+    # stream over the same number of eager steps
+    fc1_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.steps):
+        step(fc1_ev[i])
+    torch.cuda.synchronize()
+    fc1_ms = float(np.mean([a.elapsed_time(c) for a, c in fc1_ev]))
 
     # end to end through the public API: pinned host inputs -> device, layer, result -> host
     xh = torch.empty((wl.T, wl.d), dtype=torch.bfloat16, pin_memory=True)
@@ -281,14 +289,12 @@ def run_ours(args, rank, world, local_rank):
     xh.copy_(x)
     lh.copy_(lg)
     oh = torch.empty((wl.T, wl.d), dtype=torch.float32, pin_memory=True)
-    xd = torch.empty_like(x)
-    ld = torch.empty_like(lg)
 
     def e2e_step():
-        xd.copy_(xh, non_blocking=True)
-        ld.copy_(lh, non_blocking=True)
-        out = layer.forward(xd, ld)
-        oh.copy_(out, non_blocking=True)
+        x.copy_(xh, non_blocking=True)
+        lg.copy_(lh, non_blocking=True)
+        graph.replay()
+        oh.copy_(gout, non_blocking=True)
 
     for _ in range(2):
         e2e_step()
@@ -347,6 +353,7 @@ def run_ours(args, rank, world, local_rank):
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": wl.T * wl.d * 2 + wl.T * wl.E * 4,
                 "d2h_bytes_per_step": wl.T * wl.d * 4},
         "gpu_launches": launches_per_step * args.steps,
+        "step_mode": "CUDA graph of the seven library calls",
         "clocks": clk.summary(),
     }
     return line

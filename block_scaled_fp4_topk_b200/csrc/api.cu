@@ -131,17 +131,20 @@ ds4g_status ds4g_grouped_gemm_fp4(const ds4g_fp4* a, const int32_t* offsets, int
     if (st != DS4G_OK) return st;
     st = check_fp4(w, (int64_t)E * N, K, fmt, true);
     if (st != DS4G_OK) return st;
-    // kernel choice: the weight-streaming GEMV for decode-sized segments (and
-    // for K the tensor-core kernel's scale loads cannot tile), else tcgen05
-    const bool gemv = max_rows_per_expert <= 8 || !gemm_tc_supports(fmt, K);
+    // kernel choice: the tcgen05 kernel for segments longer than 8 rows when
+    // its tiling fits (K for the scale loads, N / I for the 256-column tiles),
+    // else the weight-streaming GEMV kernel (any segment length)
+    const bool tc_shape = gemm_tc_supports(fmt, K) &&
+                          (epilogue == DS4G_EPI_NONE ? (N % 256 == 0) : (N % 2 == 0 && (N / 2) % 128 == 0));
+    const bool gemv = max_rows_per_expert <= 8 || !tc_shape;
     const int64_t Sr = a->rows;
     if (epilogue == DS4G_EPI_NONE) {
         if (Sr > 0 && (!out || !aligned16(out))) return DS4G_ERR_INVALID_ARG;
-        if (gemv ? (N % 64 != 0) : (N % 256 != 0)) return DS4G_ERR_SHAPE;
+        if (N % 64 != 0) return DS4G_ERR_SHAPE;
     } else {
         if (N % 2 != 0) return DS4G_ERR_SHAPE;
         const int I = N / 2;
-        if (gemv ? (I % 32 != 0) : (I % 128 != 0)) return DS4G_ERR_SHAPE;
+        if (I % 32 != 0) return DS4G_ERR_SHAPE;
         st = check_fp4(out_q, Sr, I, fmt, true);
         if (st != DS4G_OK) return st;
         if (h_debug && !aligned16(h_debug)) return DS4G_ERR_INVALID_ARG;

@@ -49,6 +49,17 @@ __device__ __forceinline__ uint32_t e2m1_code(float y)
     return e2m1_mag_code(fabsf(y)) | ((__float_as_uint(y) >> 28) & 8u);
 }
 
+// Two values at once with the hardware conversion (round to nearest even,
+// saturating to +-6, sign kept): low nibble = lo, high nibble = hi.
+__device__ __forceinline__ uint32_t e2m1x2(float lo, float hi)
+{
+    uint32_t d;
+    asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u32.u8 %0, t;\n\t}"
+        : "=r"(d)
+        : "f"(hi), "f"(lo));
+    return d;
+}
+
 // MX shared exponent X = floor(log2(amax)) - 2, clamped to [-127, 127]
 // (OCP MX rule with the E2M1 element's largest exponent 2), from the bits.
 __device__ __forceinline__ int mx_shared_exp(float amax)

@@ -535,7 +535,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
                         const float g = gv[i] * gscale, u = uv[i] * gscale;
-                        h[i] = __fmul_rn(__fdiv_rn(g, __fadd_rn(1.0f, expf(-g))), u);
+                        h[i] = __fdividef(g * u, 1.0f + __expf(-g));    // silu(g) * u
                     }
                     if (valid) {
                         if (p.h_debug) {
@@ -551,7 +551,8 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
                             const int X = mx_shared_exp(m);
                             const float inv = exp2i(-X);
 #pragma unroll
-                            for (int i = 0; i < 32; ++i) wq[i >> 3] |= e2m1_code(__fmul_rn(h[i], inv)) << (4 * (i & 7));
+                            for (int i = 0; i < 32; i += 2)
+                                wq[i >> 3] |= e2m1x2(__fmul_rn(h[i], inv), __fmul_rn(h[i + 1], inv)) << (4 * (i & 7));
                             p.oq_scales[row * (I / 32) + col0 / 32] = (uint8_t)(X + 127);
                         } else {
                             uint32_t sb[2];
@@ -562,13 +563,16 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
                                 for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(h[16 * hb + i]));
                                 const uint32_t s = ue4m3_encode(__fdiv_rn(m, __fmul_rn(6.0f, gh)));
                                 const float ds = ue4m3_value(s);
-                                const float den = __fmul_rn(ds, gh);
+                                if (ds == 0.0f) {
 #pragma unroll
-                                for (int i = 0; i < 16; ++i) {
-                                    const float x = h[16 * hb + i];
-                                    const uint32_t code =
-                                        (ds == 0.0f) ? ((__float_as_uint(x) >> 28) & 8u) : e2m1_code(__fdiv_rn(x, den));
-                                    wq[2 * hb + (i >> 3)] |= code << (4 * (i & 7));
+                                    for (int i = 0; i < 16; ++i)
+                                        wq[2 * hb + (i >> 3)] |= ((__float_as_uint(h[16 * hb + i]) >> 28) & 8u) << (4 * (i & 7));
+                                } else {
+                                    const float rcp = __frcp_rn(__fmul_rn(ds, gh));
+#pragma unroll
+                                    for (int i = 0; i < 16; i += 2)
+                                        wq[2 * hb + (i >> 3)] |= e2m1x2(h[16 * hb + i] * rcp, h[16 * hb + i + 1] * rcp)
+                                                                 << (4 * (i & 7));
                                 }
                                 sb[hb] = s;
                             }

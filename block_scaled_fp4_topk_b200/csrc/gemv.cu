@@ -24,8 +24,6 @@
 
 namespace ds4g {
 
-constexpr int kGemvThreads = 256;
-
 template <int FMT>
 struct BlockScale;
 
@@ -69,13 +67,19 @@ __device__ __forceinline__ void decode_word_signed(uint32_t x, uint32_t& lo, uin
     hi = out[1];
 }
 
-template <int FMT, int EPI, int MAXR, int RPW>
-__global__ void __launch_bounds__(kGemvThreads)
+// NW warps per CTA, NR weight rows per warp, activation rows handled MAXR at a
+// time (rows beyond the segment are skipped at run time, CTA-uniformly).
+// FC1 with the fused epilogue: a CTA owns 32 gate columns and the matching 32
+// up rows (NW * NR == 64), each warp NR/2 gate + NR/2 up rows.
+template <int FMT, int EPI, int MAXR, int NW, int NR>
+__global__ void __launch_bounds__(NW * 32)
 k_gemv(const GemmArgs p)
 {
     extern __shared__ __align__(16) uint8_t smem[];
     constexpr int BLK = (FMT == DS4G_MXFP4) ? 32 : 16;
     constexpr int NSB = 32 / BLK;                       // scales per 32-element chunk
+    constexpr int NT = NW * 32;
+    constexpr bool kSwiGLU = (EPI == DS4G_EPI_SWIGLU_REQUANT);
     const int64_t K = p.K;
     const int64_t nchunk = K / 32;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -98,38 +102,37 @@ k_gemv(const GemmArgs p)
     const float gscale = (FMT == DS4G_NVFP4) ? __fmul_rn(p.a_g[0], p.w_g[e]) : 1.0f;   // per-expert weight scale
     const int I = p.N / 2;
 
+    // this warp's weight rows
+    int64_t wrow[NR];
+#pragma unroll
+    for (int i = 0; i < NR; ++i) {
+        int n;
+        if (kSwiGLU) {
+            constexpr int H = NR / 2;
+            n = (i < H) ? (blockIdx.x * 32 + warp * H + i) : (I + blockIdx.x * 32 + warp * H + (i - H));
+        } else {
+            n = blockIdx.x * (NW * NR) + warp * NR + i;
+        }
+        wrow[i] = (int64_t)e * p.N + n;
+    }
+
     for (int64_t rg = r; rg < seg_end; rg += MAXR) {
         const int nr = (int)min((int64_t)MAXR, seg_end - rg);
         __syncthreads();
         // ---- activation rows -> int8 + float scales in shared memory
-        for (int64_t i = threadIdx.x; i < (int64_t)MAXR * (K / 8); i += kGemvThreads) {
+        for (int64_t i = threadIdx.x; i < (int64_t)nr * (K / 8); i += NT) {
             const int rr = (int)(i / (K / 8));
             const int64_t wd = i % (K / 8);
-            uint32_t lo8 = 0, hi8 = 0;
-            if (rr < nr) {
-                uint32_t x = reinterpret_cast<const uint32_t*>(p.a_data + (rg + rr) * (K / 2))[wd];
-                decode_word_signed(x, lo8, hi8);
-            }
+            uint32_t lo8, hi8;
+            const uint32_t x = reinterpret_cast<const uint32_t*>(p.a_data + (rg + rr) * (K / 2))[wd];
+            decode_word_signed(x, lo8, hi8);
             reinterpret_cast<uint2*>(a8)[i] = make_uint2(lo8, hi8);
         }
-        for (int64_t i = threadIdx.x; i < (int64_t)MAXR * (K / BLK); i += kGemvThreads) {
+        for (int64_t i = threadIdx.x; i < (int64_t)nr * (K / BLK); i += NT) {
             const int rr = (int)(i / (K / BLK));
-            asc[i] = (rr < nr) ? BlockScale<FMT>::a(p.a_scales[(rg + rr) * (K / BLK) + i % (K / BLK)]) : 0.f;
+            asc[i] = BlockScale<FMT>::a(p.a_scales[(rg + rr) * (K / BLK) + i % (K / BLK)]);
         }
         __syncthreads();
-
-        // ---- this warp's weight rows
-        constexpr int NR = (EPI == DS4G_EPI_SWIGLU_REQUANT) ? 8 : RPW;
-        int64_t wrow[NR];
-#pragma unroll
-        for (int i = 0; i < NR; ++i) {
-            int n;
-            if (EPI == DS4G_EPI_SWIGLU_REQUANT)
-                n = (i < 4) ? (blockIdx.x * 32 + warp * 4 + i) : (I + blockIdx.x * 32 + warp * 4 + (i - 4));
-            else
-                n = blockIdx.x * (8 * RPW) + warp * RPW + i;
-            wrow[i] = (int64_t)e * p.N + n;
-        }
 
         float acc[NR][MAXR];
 #pragma unroll
@@ -158,7 +161,6 @@ k_gemv(const GemmArgs p)
 #pragma unroll
             for (int i = 0; i < NR; ++i) { cv[i] = wv[i]; cs[i] = ws[i]; }
             load(c + 32);                                  // prefetch the next step
-            // activation int8 words of this chunk for every row
 #pragma unroll
             for (int i = 0; i < NR; ++i) {
                 uint32_t pp[8], pn[8];
@@ -173,31 +175,33 @@ k_gemv(const GemmArgs p)
                 }
 #pragma unroll
                 for (int rr = 0; rr < MAXR; ++rr) {
-                    const uint4* ap = reinterpret_cast<const uint4*>(a8 + (size_t)rr * K + c * 32);
-                    const uint4 a0 = ap[0], a1 = ap[1];
-                    const uint32_t av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-                    if (FMT == DS4G_MXFP4) {
-                        int dp = 0, dn = 0;
+                    if (rr < nr) {
+                        const uint4* ap = reinterpret_cast<const uint4*>(a8 + (size_t)rr * K + c * 32);
+                        const uint4 a0 = ap[0], a1 = ap[1];
+                        const uint32_t av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+                        if (FMT == DS4G_MXFP4) {
+                            int dp = 0, dn = 0;
 #pragma unroll
-                        for (int m = 0; m < 8; ++m) {
-                            dp = __dp4a((int)pp[m], (int)av[m], dp);
-                            dn = __dp4a((int)pn[m], (int)av[m], dn);
-                        }
-                        const float sa = asc[(size_t)rr * (K / BLK) + c];
-                        acc[i][rr] += ((float)(dp - dn) * sa) * BlockScale<FMT>::w(cs[i]);
-                    } else {
-                        int dp0 = 0, dn0 = 0, dp1 = 0, dn1 = 0;
+                            for (int m = 0; m < 8; ++m) {
+                                dp = __dp4a((int)pp[m], (int)av[m], dp);
+                                dn = __dp4a((int)pn[m], (int)av[m], dn);
+                            }
+                            const float sa = asc[(size_t)rr * (K / BLK) + c];
+                            acc[i][rr] += ((float)(dp - dn) * sa) * BlockScale<FMT>::w(cs[i]);
+                        } else {
+                            int dp0 = 0, dn0 = 0, dp1 = 0, dn1 = 0;
 #pragma unroll
-                        for (int m = 0; m < 4; ++m) {
-                            dp0 = __dp4a((int)pp[m], (int)av[m], dp0);
-                            dn0 = __dp4a((int)pn[m], (int)av[m], dn0);
-                            dp1 = __dp4a((int)pp[m + 4], (int)av[m + 4], dp1);
-                            dn1 = __dp4a((int)pn[m + 4], (int)av[m + 4], dn1);
+                            for (int m = 0; m < 4; ++m) {
+                                dp0 = __dp4a((int)pp[m], (int)av[m], dp0);
+                                dn0 = __dp4a((int)pn[m], (int)av[m], dn0);
+                                dp1 = __dp4a((int)pp[m + 4], (int)av[m + 4], dp1);
+                                dn1 = __dp4a((int)pn[m + 4], (int)av[m + 4], dn1);
+                            }
+                            const float sa0 = asc[(size_t)rr * (K / BLK) + 2 * c];
+                            const float sa1 = asc[(size_t)rr * (K / BLK) + 2 * c + 1];
+                            acc[i][rr] += ((float)(dp0 - dn0) * sa0) * BlockScale<FMT>::w(cs[i] & 0xFF);
+                            acc[i][rr] += ((float)(dp1 - dn1) * sa1) * BlockScale<FMT>::w(cs[i] >> 8);
                         }
-                        const float sa0 = asc[(size_t)rr * (K / BLK) + 2 * c];
-                        const float sa1 = asc[(size_t)rr * (K / BLK) + 2 * c + 1];
-                        acc[i][rr] += ((float)(dp0 - dn0) * sa0) * BlockScale<FMT>::w(cs[i] & 0xFF);
-                        acc[i][rr] += ((float)(dp1 - dn1) * sa1) * BlockScale<FMT>::w(cs[i] >> 8);
                     }
                 }
             }
@@ -208,37 +212,38 @@ k_gemv(const GemmArgs p)
         for (int i = 0; i < NR; ++i)
 #pragma unroll
             for (int rr = 0; rr < MAXR; ++rr) {
-                float v = acc[i][rr];
+                if (rr < nr) {
+                    float v = acc[i][rr];
 #pragma unroll
-                for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-                acc[i][rr] = v * gscale;
+                    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+                    acc[i][rr] = v * gscale;
+                }
             }
 
-        if (EPI == DS4G_EPI_NONE) {
-            if (lane < MAXR) {
+        if (!kSwiGLU) {
 #pragma unroll
-                for (int rr = 0; rr < MAXR; ++rr) {
-                    if (rr == lane && rr < nr) {
+            for (int rr = 0; rr < MAXR; ++rr) {
+                if (rr == lane && rr < nr) {
 #pragma unroll
-                        for (int i = 0; i < NR; ++i)
-                            p.out[(rg + rr) * p.N + (blockIdx.x * (8 * RPW) + warp * RPW + i)] = acc[i][rr];
-                    }
+                    for (int i = 0; i < NR; ++i)
+                        p.out[(rg + rr) * p.N + (blockIdx.x * (NW * NR) + warp * NR + i)] = acc[i][rr];
                 }
             }
         } else {
             // gate / up results of this CTA's 32 columns -> shared, then one
             // warp per activation row computes h and quantises its block(s)
+            constexpr int H = NR / 2;
             if (lane == 0) {
 #pragma unroll
                 for (int rr = 0; rr < MAXR; ++rr)
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        red[(0 * MAXR + rr) * 32 + warp * 4 + i] = acc[i][rr];
-                        red[(1 * MAXR + rr) * 32 + warp * 4 + i] = acc[i + 4][rr];
+                    for (int i = 0; i < H; ++i) {
+                        red[(0 * MAXR + rr) * 32 + warp * H + i] = acc[i][rr];
+                        red[(1 * MAXR + rr) * 32 + warp * H + i] = acc[i + H][rr];
                     }
             }
             __syncthreads();
-            for (int rr = warp; rr < nr; rr += 8) {
+            for (int rr = warp; rr < nr; rr += NW) {
                 const float g = red[(0 * MAXR + rr) * 32 + lane];
                 const float u = red[(1 * MAXR + rr) * 32 + lane];
                 const float h = __fmul_rn(__fdiv_rn(g, __fadd_rn(1.0f, expf(-g))), u);
@@ -272,42 +277,43 @@ k_gemv(const GemmArgs p)
     }
 }
 
-template <int FMT, int EPI, int MAXR, int RPW>
+template <int FMT, int EPI, int MAXR, int NW, int NR>
 static cudaError_t run(const GemmArgs& a, int gx, cudaStream_t st)
 {
     constexpr int BLK = (FMT == DS4G_MXFP4) ? 32 : 16;
     const size_t shm = (size_t)MAXR * a.K + (size_t)MAXR * (a.K / BLK) * 4 + 2 * MAXR * 32 * 4;
-    auto kern = k_gemv<FMT, EPI, MAXR, RPW>;
+    auto kern = k_gemv<FMT, EPI, MAXR, NW, NR>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)shm);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)gx, (unsigned)a.S);
-    kern<<<grid, kGemvThreads, shm, st>>>(a);
+    kern<<<grid, NW * 32, shm, st>>>(a);
     return cudaGetLastError();
 }
 
 template <int FMT, int EPI, int MAXR>
-static cudaError_t pick_rpw(const GemmArgs& a, cudaStream_t st)
+static cudaError_t pick_shape(const GemmArgs& a, cudaStream_t st)
 {
-    if (EPI == DS4G_EPI_SWIGLU_REQUANT) return run<FMT, EPI, MAXR, 8>(a, a.N / 2 / 32, st);
-    // enough CTAs in flight: aim for >= 4 waves of column tiles per touched expert
+    constexpr int NRMAX = MAXR >= 4 ? 4 : 8;     // keeps the accumulators in registers
+    if (EPI == DS4G_EPI_SWIGLU_REQUANT) return run<FMT, EPI, MAXR, 64 / NRMAX, NRMAX>(a, a.N / 2 / 32, st);
+    // enough CTAs in flight: aim for >= 4 CTAs per SM over the touched experts
     const int64_t experts = a.S < a.E ? a.S : a.E;
-    int rpw = 8;
+    int rpw = NRMAX;
     while (rpw > 1 && (int64_t)(a.N / (8 * rpw)) * experts < 4 * kNumSMs) rpw >>= 1;
     switch (rpw) {
-    case 8: return run<FMT, EPI, MAXR, 8>(a, a.N / 64, st);
-    case 4: return run<FMT, EPI, MAXR, 4>(a, a.N / 32, st);
-    case 2: return run<FMT, EPI, MAXR, 2>(a, a.N / 16, st);
-    default: return run<FMT, EPI, MAXR, 1>(a, a.N / 8, st);
+    case 8: return run<FMT, EPI, MAXR, 8, (NRMAX >= 8 ? 8 : 4)>(a, a.N / (8 * (NRMAX >= 8 ? 8 : 4)), st);
+    case 4: return run<FMT, EPI, MAXR, 8, 4>(a, a.N / 32, st);
+    case 2: return run<FMT, EPI, MAXR, 8, 2>(a, a.N / 16, st);
+    default: return run<FMT, EPI, MAXR, 8, 1>(a, a.N / 8, st);
     }
 }
 
 template <int FMT, int EPI>
 static cudaError_t pick_rows(const GemmArgs& a, cudaStream_t st)
 {
-    if (a.max_rows <= 1) return pick_rpw<FMT, EPI, 1>(a, st);
-    if (a.max_rows <= 2) return pick_rpw<FMT, EPI, 2>(a, st);
-    if (a.max_rows <= 4) return pick_rpw<FMT, EPI, 4>(a, st);
-    return pick_rpw<FMT, EPI, 8>(a, st);
+    if (a.max_rows <= 1) return pick_shape<FMT, EPI, 1>(a, st);
+    if (a.max_rows <= 2) return pick_shape<FMT, EPI, 2>(a, st);
+    if (a.max_rows <= 4) return pick_shape<FMT, EPI, 4>(a, st);
+    return pick_shape<FMT, EPI, 8>(a, st);
 }
 
 cudaError_t launch_gemv(const GemmArgs& a, cudaStream_t st)

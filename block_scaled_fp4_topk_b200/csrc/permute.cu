@@ -117,6 +117,86 @@ __global__ void k_perm_gather(const uint8_t* __restrict__ xd, const uint8_t* __r
     for (int64_t i = lane; i < ns / 2; i += 32) sd[i] = ss[i];
 }
 
+// Small slot counts (decode): the whole permutation in one CTA -- counts,
+// scan, stable ranks and the row gather -- so a decode step pays one launch.
+constexpr int kSmallS = 512;
+
+__global__ void __launch_bounds__(512)
+k_perm_small(const int32_t* __restrict__ idx, int S, int E, int k, int64_t K, int blk,
+             const uint8_t* __restrict__ xd, const uint8_t* __restrict__ xs, const float* __restrict__ xg,
+             int32_t* __restrict__ offsets, int32_t* __restrict__ row_to_slot, int32_t* __restrict__ slot_to_row,
+             uint8_t* __restrict__ ad, uint8_t* __restrict__ as, float* __restrict__ ag)
+{
+    extern __shared__ int32_t sh[];
+    int32_t* cnt = sh;                 // [E]
+    int32_t* off = sh + E;             // [E + 1]
+    int32_t* r2s = off + E + 1;        // [S]
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (ag && tid == 0) *ag = *xg;
+    for (int e = tid; e < E; e += blockDim.x) cnt[e] = 0;
+    __syncthreads();
+    for (int s = tid; s < S; s += blockDim.x) atomicAdd(&cnt[idx[s]], 1);
+    __syncthreads();
+    if (warp == 0) {
+        const int per = (E + 31) / 32;
+        int32_t sum = 0;
+        for (int i = 0; i < per; ++i) {
+            const int e = lane * per + i;
+            if (e < E) sum += cnt[e];
+        }
+        int32_t incl = sum;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        int32_t run = incl - sum;
+        for (int i = 0; i < per; ++i) {
+            const int e = lane * per + i;
+            if (e < E) {
+                off[e] = run;
+                offsets[e] = run;
+                run += cnt[e];
+                cnt[e] = 0;            // reused as the running rank of each expert
+            }
+        }
+        if (lane == 31) {
+            off[E] = incl;
+            offsets[E] = incl;
+        }
+        __syncwarp();
+        for (int g = 0; g < S; g += 32) {
+            const int s = g + lane;
+            const bool valid = s < S;
+            const int e = valid ? idx[s] : -1 - lane;
+            const unsigned peers = __match_any_sync(0xffffffffu, e);
+            const int rank = __popc(peers & ((1u << lane) - 1u));
+            int32_t pos = 0;
+            if (valid) pos = off[e] + cnt[e] + rank;
+            __syncwarp();
+            if (valid && rank == 0) cnt[e] += __popc(peers);
+            __syncwarp();
+            if (valid) {
+                r2s[pos] = s;
+                row_to_slot[pos] = s;
+                slot_to_row[s] = pos;
+            }
+        }
+    }
+    __syncthreads();
+    // gather: one warp per permuted row
+    const int64_t nvec = K / 32;
+    const int64_t ns = K / blk;
+    for (int r = warp; r < S; r += blockDim.x / 32) {
+        const int64_t t = r2s[r] / k;
+        const uint4* src = reinterpret_cast<const uint4*>(xd + t * (K / 2));
+        uint4* dst = reinterpret_cast<uint4*>(ad + (int64_t)r * (K / 2));
+        for (int64_t i = lane; i < nvec; i += 32) dst[i] = src[i];
+        const uint16_t* ss = reinterpret_cast<const uint16_t*>(xs + t * ns);
+        uint16_t* sd = reinterpret_cast<uint16_t*>(as + (int64_t)r * ns);
+        for (int64_t i = lane; i < ns / 2; i += 32) sd[i] = ss[i];
+    }
+}
+
 cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, const uint8_t* xd, const uint8_t* xs,
                            const float* xg, int64_t K, int fmt, int32_t* offsets, int32_t* row_to_slot,
                            int32_t* slot_to_row, uint8_t* ad, uint8_t* as, float* ag, void* ws_,
@@ -131,6 +211,13 @@ cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, const uint8_
         if (e != cudaSuccess) return e;
         if (fmt == DS4G_NVFP4 && ag) return cudaMemcpyAsync(ag, xg, sizeof(float), cudaMemcpyDeviceToDevice, st);
         return cudaSuccess;
+    }
+    const int blk0 = (fmt == DS4G_MXFP4) ? 32 : 16;
+    if (S <= kSmallS) {
+        const size_t shs = (size_t)(2 * E + 1 + S) * sizeof(int32_t);
+        k_perm_small<<<1, 512, shs, st>>>(idx, (int)S, E, k, K, blk0, xd, xs, xg, offsets, row_to_slot, slot_to_row,
+                                          ad, as, fmt == DS4G_NVFP4 ? ag : nullptr);
+        return cudaGetLastError();
     }
     k_perm_hist<<<B, 256, shm, st>>>(idx, S, E, B, ws);
     k_perm_scan<<<1, 1024, 0, st>>>(ws, E * B, E, B, S, offsets);

@@ -48,10 +48,8 @@ __device__ __forceinline__ void quant_mx_block(const float* v, uint4& packed, ui
     float inv = exp2i(-X);
     uint32_t w[4] = {0, 0, 0, 0};
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-        uint32_t c = e2m1_code(__fmul_rn(v[i], inv));
-        w[i >> 3] |= c << (4 * (i & 7));
-    }
+    for (int i = 0; i < 32; i += 2)
+        w[i >> 3] |= e2m1x2(__fmul_rn(v[i], inv), __fmul_rn(v[i + 1], inv)) << (4 * (i & 7));
     packed = make_uint4(w[0], w[1], w[2], w[3]);
 }
 
@@ -67,11 +65,13 @@ __device__ __forceinline__ void quant_nv_block(const float* v, float g, uint2& p
     float ds = ue4m3_value(s);
     float denom = __fmul_rn(ds, g);
     uint32_t w[2] = {0, 0};
+    if (ds == 0.0f) {
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        uint32_t c = (ds == 0.0f) ? ((__float_as_uint(v[i]) >> 28) & 8u)
-                                  : e2m1_code(__fdiv_rn(v[i], denom));
-        w[i >> 3] |= c << (4 * (i & 7));
+        for (int i = 0; i < 16; ++i) w[i >> 3] |= ((__float_as_uint(v[i]) >> 28) & 8u) << (4 * (i & 7));
+    } else {
+#pragma unroll
+        for (int i = 0; i < 16; i += 2)
+            w[i >> 3] |= e2m1x2(__fdiv_rn(v[i], denom), __fdiv_rn(v[i + 1], denom)) << (4 * (i & 7));
     }
     packed = make_uint2(w[0], w[1]);
 }

@@ -69,6 +69,20 @@ class MoeLayer:
         ds4g.ds4g_moe_combine(b["y2"], b["s2r"][:T * self.k], b["w"], out=b["out"])
         return b["out"]
 
+    def capture(self, x, logits):
+        """Records forward(x, logits) on these (static) input buffers as a CUDA
+        graph; returns (graph, out).  Replaying the graph re-runs the whole
+        layer on whatever x / logits hold at that time."""
+        side = torch.cuda.Stream(device=x.device)
+        side.wait_stream(torch.cuda.current_stream(x.device))
+        with torch.cuda.stream(side):
+            self.forward(x, logits)            # first call sets kernel attributes, buffers
+        torch.cuda.current_stream(x.device).wait_stream(side)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            out = self.forward(x, logits)
+        return graph, out
+
     # -- synthetic weights -----------------------------------------------------
     @staticmethod
     def synthetic_weights(E, d, I, fmt, seed=0, device="cuda", rows_w1=None, chunk=8):

@@ -151,12 +151,12 @@ ds4g_status ds4g_moe_permute(const int32_t* idx, int T, int k, int E, const ds4g
  *   ds4g_quantize_mx; for NVFP4 *out_q->g is the caller's static tensor
  *   scale of h, read, not written); h_debug (nullable) receives h fp32 [S][I].
  * max_rows_per_expert: an upper bound on any segment length (T for top-k
- *   routing).  The tcgen05 tensor-core kernel runs when it is > 8 and K is a
- *   multiple of 512 (MXFP4) / 256 (NVFP4); otherwise the weight-streaming
+ *   routing).  The tcgen05 tensor-core kernel runs when it is > 8 and the
+ *   shape tiles: K a multiple of 512 (MXFP4) / 256 (NVFP4), and N % 256 == 0
+ *   (NONE) or I % 128 == 0 (SWIGLU_REQUANT); otherwise the weight-streaming
  *   GEMV kernel runs (any segment length, processed 8 rows at a time).
- * Shapes: K % 64 == 0; NONE needs N % 256 == 0 (tensor-core kernel) or
- *   N % 64 == 0 (GEMV kernel); SWIGLU_REQUANT needs I % 128 == 0
- *   (tensor-core) or I % 32 == 0 (GEMV).  offsets[E] must equal S. */
+ * Shapes: K % 64 == 0; NONE needs N % 64 == 0; SWIGLU_REQUANT needs
+ *   I % 32 == 0.  offsets[E] must equal S. */
 ds4g_status ds4g_grouped_gemm_fp4(const ds4g_fp4* a, const int32_t* offsets, int E,
                                   int max_rows_per_expert, const ds4g_fp4* w, int N, int epilogue,
                                   float* out, ds4g_fp4* out_q, float* h_debug, void* stream);

@@ -1,0 +1,48 @@
+"""The C-ABI library loads on a machine without a GPU and exports every
+function include/ds4g.h declares; the host-only helpers answer without a
+device (no compute call is made here)."""
+import ctypes
+import os
+import re
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "ds4g.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(ds4g_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_path_calls():
+    names = _declared()
+    for n in ("ds4g_quantize_mx", "ds4g_route_topk", "ds4g_moe_permute", "ds4g_grouped_gemm_fp4",
+              "ds4g_swiglu_requant", "ds4g_moe_combine"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    from block_scaled_fp4_topk_b200 import build
+    build.build()
+    lib = ctypes.CDLL(build.LIB)
+    missing = [n for n in _declared() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_host_only_helpers():
+    from block_scaled_fp4_topk_b200 import ds4g
+    L = ds4g._lib
+    assert L.ds4g_status_str(0) == b"ok"
+    assert b"64" in L.ds4g_status_str(2)
+    assert L.ds4g_quantize_workspace_bytes(1, 0) >= 4 and L.ds4g_quantize_workspace_bytes(0, 0) == 0
+    assert L.ds4g_permute_workspace_bytes(2048, 6, 256) == 256 * 12 * 4
+
+
+def test_bad_arguments_rejected_before_any_launch():
+    # shape / argument validation happens on the host and needs no device
+    from block_scaled_fp4_topk_b200 import ds4g
+    L = ds4g._lib
+    assert L.ds4g_route_topk(None, 4, 8, 9, None, None, None) == 1          # k > E
+    assert L.ds4g_moe_combine(None, None, None, 2, 2, 6, None, None) == 2   # d % 4 != 0
+    out = ds4g._Fp4C(None, None, None, 4, 96, 0, 0)
+    assert L.ds4g_quantize_mx(None, 0, 4, 96, 0, None, ctypes.byref(out), None, 0, None) == 2   # K % 64
