@@ -9,3 +9,4 @@
 #include "gemm_tc.cu"
 #include "swiglu.cu"
 #include "combine.cu"
+#include "noalloc.cu"

@@ -53,6 +53,8 @@ _SIGS = {
     "ds4g_grouped_gemm_fp4": ([_P, _vp, _i32, _i32, _P, _i32, _i32, _vp, _P, _vp, _vp], _i32),
     "ds4g_swiglu_requant": ([_vp, _i64, _i32, _i32, _P, _vp, _vp], _i32),
     "ds4g_moe_combine": ([_vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp], _i32),
+    "ds4g_permute_static_max_bytes": ([], _sz),
+    "ds4g_moe_permute_static": ([_vp, _i32, _i32, _i32, _P, _vp, _vp, _vp, _P, _vp], _i32),
 }
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -160,6 +162,26 @@ def ds4g_moe_permute(idx, E, x_q, offsets=None, row_to_slot=None, slot_to_row=No
     _check("ds4g_moe_permute", _lib.ds4g_moe_permute(idx.data_ptr(), T, k, E, ctypes.byref(xc), offsets.data_ptr(),
                                                      row_to_slot.data_ptr(), slot_to_row.data_ptr(), ctypes.byref(ac),
                                                      workspace.data_ptr(), workspace.numel(), _stream()))
+    return offsets, row_to_slot[:S], slot_to_row[:S], a_perm
+
+
+def ds4g_moe_permute_static(idx, E, x_q, offsets=None, row_to_slot=None, slot_to_row=None, a_perm=None):
+    """ds4g_moe_permute with the library's own static scratch (no workspace)."""
+    T, k = idx.shape
+    S = T * k
+    dev = idx.device
+    if offsets is None:
+        offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    if row_to_slot is None:
+        row_to_slot = torch.empty(max(S, 1), dtype=torch.int32, device=dev)
+    if slot_to_row is None:
+        slot_to_row = torch.empty(max(S, 1), dtype=torch.int32, device=dev)
+    if a_perm is None:
+        a_perm = Fp4Tensor.empty(S, x_q.K, x_q.fmt, dev)
+    xc, ac = x_q.c(), a_perm.c()
+    _check("ds4g_moe_permute_static",
+           _lib.ds4g_moe_permute_static(idx.data_ptr(), T, k, E, ctypes.byref(xc), offsets.data_ptr(),
+                                        row_to_slot.data_ptr(), slot_to_row.data_ptr(), ctypes.byref(ac), _stream()))
     return offsets, row_to_slot[:S], slot_to_row[:S], a_perm
 
 

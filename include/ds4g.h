@@ -176,6 +176,25 @@ ds4g_status ds4g_swiglu_requant(const float* y1, int64_t rows, int I, int fmt, d
 ds4g_status ds4g_moe_combine(const float* y2, const int32_t* slot_to_row, const float* w, int T,
                              int k, int d, float* out, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * ds4g_moe_permute_static: ds4g_moe_permute without a caller workspace, for
+ * callers that cannot allocate device memory at all (a runtime that owns all
+ * device memory through its own pool, a plug-in restricted to the buffers it
+ * is handed).  The pages have no counterpart; this is a library convenience.
+ * Arguments, results and errors are those of ds4g_moe_permute.  The scratch is
+ * a file-scope device array of ds4g_permute_static_max_bytes() bytes (256 KiB)
+ * that every GPU loading the library keeps until the process exits; a problem
+ * whose ds4g_permute_workspace_bytes(T, k, E) exceeds it returns
+ * DS4G_ERR_WORKSPACE.  The first call on a device looks the array's device
+ * address up for that device (make that first call before any stream
+ * capture).  All calls share the one array: calls that overlap on the GPU
+ * (concurrent streams, or several host threads) race on it and must be
+ * serialised by the caller. */
+size_t ds4g_permute_static_max_bytes(void);
+ds4g_status ds4g_moe_permute_static(const int32_t* idx, int T, int k, int E, const ds4g_fp4* x_q,
+                                    int32_t* offsets, int32_t* row_to_slot, int32_t* slot_to_row,
+                                    ds4g_fp4* a_perm, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -36,6 +36,7 @@ def test_host_only_helpers():
     assert b"64" in L.ds4g_status_str(2)
     assert L.ds4g_quantize_workspace_bytes(1, 0) >= 4 and L.ds4g_quantize_workspace_bytes(0, 0) == 0
     assert L.ds4g_permute_workspace_bytes(2048, 6, 256) == 256 * 12 * 4
+    assert L.ds4g_permute_static_max_bytes() == 256 * 1024
 
 
 def test_bad_arguments_rejected_before_any_launch():
