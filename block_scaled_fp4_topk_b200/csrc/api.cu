@@ -131,12 +131,14 @@ ds4g_status ds4g_grouped_gemm_fp4(const ds4g_fp4* a, const int32_t* offsets, int
     if (st != DS4G_OK) return st;
     st = check_fp4(w, (int64_t)E * N, K, fmt, true);
     if (st != DS4G_OK) return st;
-    // kernel choice: the tcgen05 kernel for segments longer than 8 rows when
-    // its tiling fits (K for the scale loads, N / I for the 256-column tiles),
-    // else the weight-streaming GEMV kernel (any segment length)
+    // kernel choice: decode-sized segments (<= 16 rows) take the swapped
+    // tensor-core kernel (weights as the MMA's M side) when the tiling fits;
+    // longer segments the 128 x 256 tensor-core kernel; shapes neither fits
+    // take the dp4a GEMV kernel (any segment length)
     const bool tc_shape = gemm_tc_supports(fmt, K) &&
                           (epilogue == DS4G_EPI_NONE ? (N % 256 == 0) : (N % 2 == 0 && (N / 2) % 128 == 0));
-    const bool gemv = max_rows_per_expert <= 8 || !tc_shape;
+    const bool dtc = max_rows_per_expert <= 16 && gemv_tc_supports(fmt, K, N, epilogue);
+    const bool gemv = !dtc && (max_rows_per_expert <= 8 || !tc_shape);
     const int64_t Sr = a->rows;
     if (epilogue == DS4G_EPI_NONE) {
         if (Sr > 0 && (!out || !aligned16(out))) return DS4G_ERR_INVALID_ARG;
@@ -170,7 +172,7 @@ ds4g_status ds4g_grouped_gemm_fp4(const ds4g_fp4* a, const int32_t* offsets, int
     g.oq_g = out_q ? out_q->g : nullptr;
     g.h_debug = h_debug;
     g.max_rows = max_rows_per_expert;
-    return cuda_status(gemv ? launch_gemv(g, S(stream)) : launch_gemm_tc(g, S(stream)));
+    return cuda_status(dtc ? launch_gemv_tc(g, S(stream)) : gemv ? launch_gemv(g, S(stream)) : launch_gemm_tc(g, S(stream)));
 }
 
 ds4g_status ds4g_swiglu_requant(const float* y1, int64_t rows, int I, int fmt, ds4g_fp4* h_q, float* h_debug,

@@ -1,8 +1,9 @@
 // combine.cu -- MoE combine ("Moore Threads full-link adaptation of
 // DeepSeek-V4": MoE routing / dispatch / combine operators): each token's
 // output row is the routing-weighted sum of its k expert output rows, summed
-// in j = 0..k-1 order (a gather per token, no atomics, deterministic).  One
-// CTA per token; 16-byte loads and stores.
+// in j = 0..k-1 order (a gather per token, no atomics, deterministic).  A 2-D
+// grid (token, 1024-column slice) keeps a few-token decode step from running
+// on a handful of CTAs; 16-byte loads and stores.
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -13,7 +14,7 @@ __global__ void k_combine(const float* __restrict__ y2, const int32_t* __restric
 {
     const int64_t t = blockIdx.x;
     const int nv = d / 4;
-    for (int c = threadIdx.x; c < nv; c += blockDim.x) {
+    for (int c = blockIdx.y * blockDim.x + threadIdx.x; c < nv; c += gridDim.y * blockDim.x) {
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int j = 0; j < k; ++j) {
             const int64_t row = slot_to_row[t * k + j];
@@ -34,7 +35,9 @@ cudaError_t launch_combine(const float* y2, const int32_t* slot_to_row, const fl
     if (T == 0) return cudaSuccess;
     int threads = d / 4 < 256 ? ((d / 4 + 31) / 32) * 32 : 256;
     if (threads < 32) threads = 32;
-    k_combine<<<T, threads, 0, st>>>(y2, slot_to_row, w, k, d, out);
+    // few tokens: spread each row over several CTAs so enough loads are in flight
+    const int slices = T >= 2 * kNumSMs ? 1 : (int)ceil_div(d / 4, threads);
+    k_combine<<<dim3(T, slices), threads, 0, st>>>(y2, slot_to_row, w, k, d, out);
     return cudaGetLastError();
 }
 

@@ -618,14 +618,15 @@ static PFN_encodeTiled get_encode()
     return fn;
 }
 
-// 2-D byte map over [rows][width] bytes with a box of box_w bytes x 128 rows
-static bool make_map(CUtensorMap* m, const uint8_t* base, int64_t rows, int64_t width, uint32_t box_w, bool swizzle)
+// 2-D byte map over [rows][width] bytes with a box of box_w bytes x box_h rows
+static bool make_map(CUtensorMap* m, const uint8_t* base, int64_t rows, int64_t width, uint32_t box_w,
+                     uint32_t box_h, bool swizzle)
 {
     PFN_encodeTiled enc = get_encode();
     if (!enc) return false;
     cuuint64_t dims[2] = {(cuuint64_t)width, (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)width};
-    cuuint32_t box[2] = {box_w, 128};
+    cuuint32_t box[2] = {box_w, box_h};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(base), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -639,10 +640,10 @@ static cudaError_t run_tc(const GemmArgs& a, cudaStream_t st)
     using C = tc::Cfg<FMT>;
     const int blk = (FMT == DS4G_MXFP4) ? 32 : 16;
     CUtensorMap ma, mb, msa, msb;
-    if (!make_map(&ma, a.a_data, a.S, a.K / 2, 128, true) ||
-        !make_map(&mb, a.w_data, (int64_t)a.E * a.N, a.K / 2, 128, true) ||
-        !make_map(&msa, a.a_scales, a.S, a.K / blk, C::SF_ROW, false) ||
-        !make_map(&msb, a.w_scales, (int64_t)a.E * a.N, a.K / blk, C::SF_ROW, false))
+    if (!make_map(&ma, a.a_data, a.S, a.K / 2, 128, 128, true) ||
+        !make_map(&mb, a.w_data, (int64_t)a.E * a.N, a.K / 2, 128, 128, true) ||
+        !make_map(&msa, a.a_scales, a.S, a.K / blk, C::SF_ROW, 128, false) ||
+        !make_map(&msb, a.w_scales, (int64_t)a.E * a.N, a.K / blk, C::SF_ROW, 128, false))
         return cudaErrorInvalidValue;
     auto kern = tc::k_gemm_tc<FMT, EPI>;
     const size_t shm = C::SMEM;

@@ -1,0 +1,456 @@
+// gemv_tc.cu -- decode-sized grouped block-scaled FP4 GEMM on the tensor
+// cores, operands swapped: the 128 weight rows of a tile are the MMA's M side
+// and the (at most 16) activation rows of the expert are its N side.
+//
+// At decode sizes ("[DeepSeek V4] Triton FP4 optimisation in practice":
+// moving fewer bytes beats faster math) the work is streaming the touched
+// experts' packed weights from HBM once.  Doing the dot products on the tensor
+// cores (tcgen05.mma kind::mxf4 / kind::mxf4nvf4, M128 N16 K64, the same
+// block-scaled MMA as the prefill kernel) leaves the SMs nothing to do but
+// keep TMA copies in flight, so the kernel runs at the rate weights arrive.
+//
+// Roles (one persistent CTA per SM, 256 threads):
+//   warp 0  TMA producer: weight tile (128 rows x 256 K) and the expert's
+//           activation rows (16 rows x 256 K), 8 stages; row-major scale
+//           boxes of both (512 K per scale stage, 4 scale stages)
+//   warp 1  MMA issuer: scales -> TMEM (tcgen05.cp), 4 MMAs per stage,
+//           double-buffered 16-column accumulators
+//   warp 2  scale transposer (weights in place; activations into zeroed
+//           128-line chunks of which lines 0..15 carry the 16 rows)
+//   warp 3  TMEM allocator
+//   warps 4-7  epilogue: thread = weight row, 16 token columns; the plain
+//           fp32 store is coalesced along the weight rows; FC1 exchanges the up
+//           rows through shared memory and quantises h along 32-column blocks
+// Items (expert, group of 16 activation rows, weight tile) come from the
+// expert offsets on the device; empty experts have none.  Every mbarrier
+// wait is bounded.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace ds4g {
+
+namespace dtc {
+
+using namespace tc;   // PTX wrappers and the scale transposer of gemm_tc.cu
+
+constexpr int BMW = 128;           // weight rows per tile (MMA M)
+constexpr int BNT = 16;            // activation rows per tile (MMA N)
+constexpr int BKB = 128;
+constexpr int BK = 256;
+constexpr int STAGES = 8;
+constexpr int SF_STAGES = 4;
+constexpr int kThreads = 256;
+constexpr int W_BYTES = BMW * BKB;   // 16 KB
+constexpr int X_BYTES = BNT * BKB;   // 2 KB
+constexpr int kTmemCols = 128;
+constexpr int kColAcc = 0;         // two 16-column accumulators
+constexpr int kColSFW = 32;
+constexpr int kColSFX = 64;
+constexpr int kMaxE = 1024;
+
+template <int FMT>
+struct Cfg {
+    static constexpr int WPS = (FMT == DS4G_MXFP4) ? 2 : 4;    // 4-scale words per row per K stage
+    static constexpr int SF_ROW = 2 * WPS * 4;                  // scale bytes per row per scale stage
+    static constexpr int SFW_BYTES = BMW * SF_ROW;              // weights, transposed in place
+    static constexpr int SFXR_BYTES = BNT * SF_ROW;             // activations, as loaded
+    static constexpr int SFXC_BYTES = 2 * WPS * 512;            // activations, chunk order
+    static constexpr int DATA_BYTES = STAGES * (W_BYTES + X_BYTES);
+    static constexpr int SF_BYTES = SF_STAGES * (SFW_BYTES + SFXR_BYTES + SFXC_BYTES);
+    static constexpr size_t SMEM = 1024 + (size_t)DATA_BYTES + SF_BYTES + 512 + 64 * 16 * 4 + (kMaxE + 1) * 4;
+};
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v)
+{
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+struct Item {
+    int e;
+    int wt;        // weight tile
+    int64_t x0;    // first activation row
+    int nr;        // activation rows in the group (<= 16)
+};
+
+__device__ __forceinline__ Item item_of(int64_t it, const int32_t* prefix, const int32_t* offsets, int E, int wtiles)
+{
+    int lo = 0, hi = E - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (prefix[mid] <= it) lo = mid; else hi = mid - 1;
+    }
+    Item r;
+    r.e = lo;
+    const int64_t local = it - prefix[lo];
+    r.wt = (int)(local % wtiles);
+    r.x0 = offsets[lo] + (local / wtiles) * BNT;
+    r.nr = (int)min((int64_t)BNT, (int64_t)offsets[lo + 1] - r.x0);
+    return r;
+}
+
+template <int EPI>
+__device__ __forceinline__ void w_rows(const Item& itm, int N, int I, int64_t& y0, int64_t& y1)
+{
+    const int64_t wbase = (int64_t)itm.e * N;
+    if (EPI == DS4G_EPI_SWIGLU_REQUANT) {
+        y0 = wbase + (int64_t)itm.wt * 64;
+        y1 = wbase + I + (int64_t)itm.wt * 64;
+    } else {
+        y0 = wbase + (int64_t)itm.wt * BMW;
+        y1 = y0;
+    }
+}
+
+// activation scales: 16 row-major rows of SF_ROW bytes -> zeroed 128-line
+// chunks (one per word) whose line l < 16 holds word c of row l in its first
+// 4 bytes (rows 32.. of the chunk do not exist at N = 16)
+template <int WORDS>
+__device__ __forceinline__ void sfx_transpose(const uint8_t* raw, uint8_t* chunks, int lane)
+{
+#pragma unroll
+    for (int c = 0; c < WORDS; ++c) {
+        uint32_t w0 = 0;
+        if (lane < BNT) w0 = reinterpret_cast<const uint32_t*>(raw + lane * WORDS * 4)[c];
+        *reinterpret_cast<uint4*>(chunks + c * 512 + lane * 16) = make_uint4(w0, 0u, 0u, 0u);
+    }
+    __syncwarp();
+}
+
+template <int FMT, int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+k_gemv_tc(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x,
+          const __grid_constant__ CUtensorMap map_sfw, const __grid_constant__ CUtensorMap map_sfx, const GemmArgs p)
+{
+    using C = Cfg<FMT>;
+    constexpr bool kSwiGLU = (EPI == DS4G_EPI_SWIGLU_REQUANT);
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sW = smem;
+    uint8_t* sX = sW + STAGES * W_BYTES;
+    uint8_t* sSFW = sX + STAGES * X_BYTES;                    // [SF_STAGES][SFW_BYTES]
+    uint8_t* sSFXC = sSFW + SF_STAGES * C::SFW_BYTES;         // [SF_STAGES][SFXC_BYTES]
+    uint8_t* sSFXR = sSFXC + SF_STAGES * C::SFXC_BYTES;       // [SF_STAGES][SFXR_BYTES]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sSFXR + SF_STAGES * C::SFXR_BYTES);
+    uint64_t* full = bars;
+    uint64_t* empty = full + STAGES;
+    uint64_t* sf_full = empty + STAGES;
+    uint64_t* sf_ready = sf_full + SF_STAGES;
+    uint64_t* sf_empty = sf_ready + SF_STAGES;
+    uint64_t* tmem_full = sf_empty + SF_STAGES;
+    uint64_t* tmem_empty = tmem_full + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tmem_empty + 2);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    int32_t* total_items = reinterpret_cast<int32_t*>(tmem_slot + 2);
+    float* xch = reinterpret_cast<float*>(smem + C::DATA_BYTES + C::SF_BYTES + 512);   // [64][16] up rows
+    int32_t* prefix = reinterpret_cast<int32_t*>(xch + 64 * 16);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int E = p.E;
+    const int64_t K = p.K;
+    const int nks = (int)ceil_div(K, BK);
+    const int npairs = (nks + 1) / 2;
+    const int I = p.N / 2;
+    const int wtiles = kSwiGLU ? (I / 64) : (p.N / BMW);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(smem_u32(&full[s]), 1);
+            mbar_init(smem_u32(&empty[s]), 1);
+        }
+        for (int r = 0; r < SF_STAGES; ++r) {
+            mbar_init(smem_u32(&sf_full[r]), 1);
+            mbar_init(smem_u32(&sf_ready[r]), 1);
+            mbar_init(smem_u32(&sf_empty[r]), 1);
+        }
+        for (int b2 = 0; b2 < 2; ++b2) {
+            mbar_init(smem_u32(&tmem_full[b2]), 1);
+            mbar_init(smem_u32(&tmem_empty[b2]), 128);
+        }
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        const int per = (E + 31) / 32;
+        int32_t sum = 0;
+        for (int i = 0; i < per; ++i) {
+            const int e = lane * per + i;
+            if (e < E) sum += (int32_t)(ceil_div((int64_t)p.offsets[e + 1] - p.offsets[e], BNT) * wtiles);
+        }
+        int32_t incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        int32_t run = incl - sum;
+        for (int i = 0; i < per; ++i) {
+            const int e = lane * per + i;
+            if (e < E) {
+                prefix[e] = run;
+                run += (int32_t)(ceil_div((int64_t)p.offsets[e + 1] - p.offsets[e], BNT) * wtiles);
+            }
+        }
+        if (lane == 31) {
+            prefix[E] = incl;
+            int32_t tot = incl;
+            if ((int64_t)p.offsets[E] > p.S) {
+                raise_error(kErrBadOffsets);
+                tot = 0;
+            }
+            *total_items = tot;
+        }
+        if (lane == 0) {
+            asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&map_w) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&map_x) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&map_sfw) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&map_sfx) : "memory");
+        }
+    }
+    if (warp == 3) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int64_t nitems = *total_items;
+
+    if (warp == 0) {
+        // ================= TMA producer =================
+        if (lane == 0) {
+            uint32_t it = 0, sit = 0;
+            bool ok = true;
+            for (int64_t t = blockIdx.x; t < nitems && ok; t += gridDim.x) {
+                const Item itm = item_of(t, prefix, p.offsets, E, wtiles);
+                int64_t y0, y1;
+                w_rows<EPI>(itm, p.N, I, y0, y1);
+                for (int ks = 0; ks < nks; ++ks, ++it) {
+                    if ((ks & 1) == 0) {
+                        const int r = sit % SF_STAGES;
+                        if (!mbar_wait(smem_u32(&sf_empty[r]), ((sit / SF_STAGES) & 1) ^ 1, abort_flag)) { ok = false; break; }
+                        const uint32_t fb = smem_u32(&sf_full[r]);
+                        mbar_arrive_tx(fb, C::SFW_BYTES + C::SFXR_BYTES);
+                        const int x = (ks >> 1) * C::SF_ROW;
+                        tma_load_2d(smem_u32(sSFW + r * C::SFW_BYTES), &map_sfw, fb, x, (int)y0);
+                        if (kSwiGLU) tma_load_2d(smem_u32(sSFW + r * C::SFW_BYTES + C::SFW_BYTES / 2), &map_sfw, fb, x, (int)y1);
+                        tma_load_2d(smem_u32(sSFXR + r * C::SFXR_BYTES), &map_sfx, fb, x, (int)itm.x0);
+                        ++sit;
+                    }
+                    const int s = it % STAGES;
+                    if (!mbar_wait(smem_u32(&empty[s]), ((it / STAGES) & 1) ^ 1, abort_flag)) { ok = false; break; }
+                    const uint32_t fb = smem_u32(&full[s]);
+                    mbar_arrive_tx(fb, W_BYTES + X_BYTES);
+                    tma_load_2d(smem_u32(sW + s * W_BYTES), &map_w, fb, ks * BKB, (int)y0);
+                    if (kSwiGLU) tma_load_2d(smem_u32(sW + s * W_BYTES + W_BYTES / 2), &map_w, fb, ks * BKB, (int)y1);
+                    tma_load_2d(smem_u32(sX + s * X_BYTES), &map_x, fb, ks * BKB, (int)itm.x0);
+                }
+            }
+            if (!ok) {
+                volatile int never = 0;
+                for (uint32_t j = (it > STAGES ? it - STAGES : 0); j < it; ++j)
+                    mbar_wait(smem_u32(&full[j % STAGES]), (j / STAGES) & 1, &never);
+                for (uint32_t j = (sit > SF_STAGES ? sit - SF_STAGES : 0); j < sit; ++j)
+                    mbar_wait(smem_u32(&sf_full[j % SF_STAGES]), (j / SF_STAGES) & 1, &never);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ================= MMA issuer =================
+        if (lane == 0) {
+            const uint32_t ibase = (1u << 7) | (1u << 10) | ((uint32_t)(BNT >> 3) << 17) |
+                                   ((FMT == DS4G_MXFP4 ? 1u : 0u) << 23) | ((uint32_t)(BMW >> 4) << 24);
+            uint32_t it = 0, sit = 0, tcount = 0;
+            bool ok = true;
+            for (int64_t t = blockIdx.x; t < nitems && ok; t += gridDim.x, ++tcount) {
+                const int buf = tcount & 1;
+                if (!mbar_wait(smem_u32(&tmem_empty[buf]), ((tcount >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t acc = tmem + kColAcc + buf * BNT;
+                for (int ks = 0; ks < nks; ++ks, ++it) {
+                    const int r = sit % SF_STAGES;
+                    if ((ks & 1) == 0) {
+                        if (!mbar_wait(smem_u32(&sf_ready[r]), (sit / SF_STAGES) & 1, abort_flag)) { ok = false; break; }
+                    }
+                    const int s = it % STAGES;
+                    if (!mbar_wait(smem_u32(&full[s]), (it / STAGES) & 1, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    const int w0 = (ks & 1) * C::WPS;
+                    const uint32_t sfw_s = smem_u32(sSFW + r * C::SFW_BYTES);
+                    const uint32_t sfx_s = smem_u32(sSFXC + r * C::SFXC_BYTES);
+#pragma unroll
+                    for (int c = 0; c < C::WPS; ++c) {
+                        utccp(tmem + kColSFW + 4 * c, desc_sf(sfw_s + (w0 + c) * 512));
+                        utccp(tmem + kColSFX + 4 * c, desc_sf(sfx_s + (w0 + c) * 512));
+                    }
+                    const int64_t krem = K - (int64_t)ks * BK;
+                    const int nmma = krem >= BK ? 4 : (int)(krem / 64);
+                    const uint32_t w_s = smem_u32(sW + s * W_BYTES);
+                    const uint32_t x_s = smem_u32(sX + s * X_BYTES);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        if (j < nmma) {
+                            const int c = (FMT == DS4G_MXFP4) ? (j >> 1) : j;
+                            const uint32_t sfid = (FMT == DS4G_MXFP4) ? (uint32_t)((j & 1) * 2) : 0u;
+                            const uint32_t idesc = ibase | (sfid << 4) | (sfid << 29);
+                            mma<FMT>(acc, desc_sw128(w_s + 32 * j), desc_sw128(x_s + 32 * j), idesc,
+                                     (ks > 0 || j > 0) ? 1u : 0u, tmem + kColSFW + 4 * c, tmem + kColSFX + 4 * c);
+                        }
+                    }
+                    tc_commit(smem_u32(&empty[s]));
+                    if ((ks & 1) == 1 || ks == nks - 1) {
+                        tc_commit(smem_u32(&sf_empty[r]));
+                        ++sit;
+                    }
+                }
+                if (!ok) break;
+                tc_commit(smem_u32(&tmem_full[buf]));
+            }
+        }
+        __syncwarp();
+    } else if (warp == 2) {
+        // ================= scale transposer =================
+        uint32_t sit = 0;
+        for (int64_t t = blockIdx.x; t < nitems; t += gridDim.x) {
+            bool ok = true;
+            for (int pr = 0; pr < npairs; ++pr, ++sit) {
+                const int r = sit % SF_STAGES;
+                bool w_ok = true;
+                if (lane == 0) w_ok = mbar_wait(smem_u32(&sf_full[r]), (sit / SF_STAGES) & 1, abort_flag);
+                if (!__shfl_sync(0xffffffffu, w_ok ? 1 : 0, 0)) { ok = false; break; }
+                sf_transpose<2 * C::WPS, 1>(sSFW + r * C::SFW_BYTES, lane);
+                sfx_transpose<2 * C::WPS>(sSFXR + r * C::SFXR_BYTES, sSFXC + r * C::SFXC_BYTES, lane);
+                fence_proxy_async();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&sf_ready[r]));
+            }
+            if (!ok) break;
+        }
+    } else if (warp >= 4) {
+        // ================= epilogue =================
+        const int q = warp & 3;                  // weight rows 32q .. 32q + 31 of the tile
+        uint32_t tcount = 0;
+        const float gh = (FMT == DS4G_NVFP4 && kSwiGLU) ? *p.oq_g : 1.0f;
+        for (int64_t t = blockIdx.x; t < nitems; t += gridDim.x, ++tcount) {
+            const int buf = tcount & 1;
+            if (!mbar_wait(smem_u32(&tmem_full[buf]), (tcount >> 1) & 1, abort_flag)) break;
+            tc_fence_after();
+            const Item itm = item_of(t, prefix, p.offsets, E, wtiles);
+            const float gscale = (FMT == DS4G_NVFP4) ? __fmul_rn(p.a_g[0], p.w_g[itm.e]) : 1.0f;
+            float v[16];
+            tmem_ld16(tmem + kColAcc + buf * BNT + ((uint32_t)(32 * q) << 16), v);
+            tc_fence_before();
+            mbar_arrive(smem_u32(&tmem_empty[buf]));          // accumulator drained into registers
+            if (!kSwiGLU) {
+                const int64_t n = (int64_t)itm.wt * BMW + 32 * q + lane;
+#pragma unroll
+                for (int tt = 0; tt < BNT; ++tt)
+                    if (tt < itm.nr) p.out[(itm.x0 + tt) * p.N + n] = v[tt] * gscale;
+            } else {
+                // up rows (warps with q >= 2) -> shared; gate rows compute h
+                asm volatile("bar.sync 1, 128;" ::: "memory");
+                if (q >= 2) {
+#pragma unroll
+                    for (int tt = 0; tt < BNT; ++tt) xch[((q - 2) * 32 + lane) * BNT + tt] = v[tt];
+                }
+                asm volatile("bar.sync 1, 128;" ::: "memory");
+                if (q < 2) {
+                    const int col = itm.wt * 64 + 32 * q + lane;    // h column (gate row within I)
+#pragma unroll 1
+                    for (int tt = 0; tt < itm.nr; ++tt) {
+                        const float g = v[tt] * gscale;
+                        const float u = xch[(q * 32 + lane) * BNT + tt] * gscale;
+                        const float h = __fdividef(g * u, 1.0f + __expf(-g));
+                        const int64_t row = itm.x0 + tt;
+                        if (p.h_debug) p.h_debug[row * I + col] = h;
+                        uint32_t code;
+                        if (FMT == DS4G_MXFP4) {
+                            float m = fabsf(h);
+#pragma unroll
+                            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+                            const int X = mx_shared_exp(m);
+                            code = e2m1_code(__fmul_rn(h, exp2i(-X)));
+                            if (lane == 0) p.oq_scales[row * (I / 32) + col / 32] = (uint8_t)(X + 127);
+                        } else {
+                            float m = fabsf(h);
+#pragma unroll
+                            for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+                            const uint32_t s = ue4m3_encode(__fdiv_rn(m, __fmul_rn(6.0f, gh)));
+                            const float ds = ue4m3_value(s);
+                            code = (ds == 0.0f) ? ((__float_as_uint(h) >> 28) & 8u)
+                                                : e2m1_code(h * __frcp_rn(__fmul_rn(ds, gh)));
+                            if ((lane & 15) == 0) p.oq_scales[row * (I / 16) + col / 16] = (uint8_t)s;
+                        }
+                        const uint32_t hi_code = __shfl_down_sync(0xffffffffu, code, 1);
+                        if ((lane & 1) == 0) p.oq_data[row * (I / 2) + col / 2] = (uint8_t)(code | (hi_code << 4));
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 3) {
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+    }
+}
+
+}  // namespace dtc
+
+template <int FMT, int EPI>
+static cudaError_t run_dtc(const GemmArgs& a, cudaStream_t st)
+{
+    using C = dtc::Cfg<FMT>;
+    const int blk = (FMT == DS4G_MXFP4) ? 32 : 16;
+    const uint32_t wbox = (EPI == DS4G_EPI_SWIGLU_REQUANT) ? 64 : 128;
+    CUtensorMap mw, mx, msw, msx;
+    if (!make_map(&mw, a.w_data, (int64_t)a.E * a.N, a.K / 2, 128, wbox, true) ||
+        !make_map(&mx, a.a_data, a.S, a.K / 2, 128, dtc::BNT, true) ||
+        !make_map(&msw, a.w_scales, (int64_t)a.E * a.N, a.K / blk, C::SF_ROW, wbox, false) ||
+        !make_map(&msx, a.a_scales, a.S, a.K / blk, C::SF_ROW, dtc::BNT, false))
+        return cudaErrorInvalidValue;
+    auto kern = dtc::k_gemv_tc<FMT, EPI>;
+    const size_t shm = C::SMEM;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)shm);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = kNumSMs;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    kern<<<sms, dtc::kThreads, shm, st>>>(mw, mx, msw, msx, a);
+    return cudaGetLastError();
+}
+
+bool gemv_tc_supports(int fmt, int64_t K, int N, int epilogue)
+{
+    if (!gemm_tc_supports(fmt, K)) return false;
+    return epilogue == DS4G_EPI_NONE ? (N % 128 == 0) : (N % 2 == 0 && (N / 2) % 64 == 0);
+}
+
+cudaError_t launch_gemv_tc(const GemmArgs& a, cudaStream_t st)
+{
+    if (a.S == 0) return cudaSuccess;
+    if (a.E > dtc::kMaxE || !gemv_tc_supports(a.fmt, a.K, a.N, a.epilogue)) return cudaErrorInvalidValue;
+    if (a.fmt == DS4G_MXFP4)
+        return a.epilogue == DS4G_EPI_NONE ? run_dtc<DS4G_MXFP4, DS4G_EPI_NONE>(a, st)
+                                           : run_dtc<DS4G_MXFP4, DS4G_EPI_SWIGLU_REQUANT>(a, st);
+    return a.epilogue == DS4G_EPI_NONE ? run_dtc<DS4G_NVFP4, DS4G_EPI_NONE>(a, st)
+                                       : run_dtc<DS4G_NVFP4, DS4G_EPI_SWIGLU_REQUANT>(a, st);
+}
+
+}  // namespace ds4g

@@ -7,6 +7,7 @@
 #include "permute.cu"
 #include "gemv.cu"
 #include "gemm_tc.cu"
+#include "gemv_tc.cu"
 #include "swiglu.cu"
 #include "combine.cu"
 #include "noalloc.cu"

@@ -151,10 +151,13 @@ ds4g_status ds4g_moe_permute(const int32_t* idx, int T, int k, int E, const ds4g
  *   ds4g_quantize_mx; for NVFP4 *out_q->g is the caller's static tensor
  *   scale of h, read, not written); h_debug (nullable) receives h fp32 [S][I].
  * max_rows_per_expert: an upper bound on any segment length (T for top-k
- *   routing).  The tcgen05 tensor-core kernel runs when it is > 8 and the
- *   shape tiles: K a multiple of 512 (MXFP4) / 256 (NVFP4), and N % 256 == 0
- *   (NONE) or I % 128 == 0 (SWIGLU_REQUANT); otherwise the weight-streaming
- *   GEMV kernel runs (any segment length, processed 8 rows at a time).
+ *   routing); it selects the kernel:
+ *   <= 16 rows, K a multiple of 512 (MXFP4) / 256 (NVFP4), N % 128 == 0
+ *     (NONE) or I % 64 == 0 (SWIGLU_REQUANT): tensor-core kernel with the
+ *     weights as the MMA's M side (decode);
+ *   > 16 rows and the same K rule, N % 256 == 0 (NONE) or I % 128 == 0
+ *     (SWIGLU_REQUANT): tensor-core kernel with 128-row x 256-column tiles;
+ *   otherwise: a dp4a weight-streaming kernel (any segment length).
  * Shapes: K % 64 == 0; NONE needs N % 64 == 0; SWIGLU_REQUANT needs
  *   I % 32 == 0.  offsets[E] must equal S. */
 ds4g_status ds4g_grouped_gemm_fp4(const ds4g_fp4* a, const int32_t* offsets, int E,

@@ -169,8 +169,10 @@ def _ref_gemm(a, offsets, w, gw, N):
     return out, ab
 
 
+# decode-sized segments: the swapped tensor-core kernel where the tiling fits
+# (K % 512 MX / % 256 NV), the dp4a kernel otherwise
 GEMV_CASES = [([3, 0, 1, 8, 5], 512, 7168), ([1, 1, 1, 1, 1, 1], 256, 2048), ([2, 0, 0, 7], 256, 256),
-              ([8], 4096, 256), ([1], 128, 128)]
+              ([8], 4096, 256), ([1], 128, 128), ([16, 9, 0, 13], 256, 1024), ([1, 2], 384, 1024)]
 # tensor-core kernel cases (MX needs K % 512, NV K % 256; others take the
 # GEMV kernel with long segments, which is covered as well)
 TC_CASES = [([300, 0, 1, 129, 77], 512, 512), ([256, 128], 256, 1024), ([9, 200, 0, 0, 1000], 256, 512),
@@ -208,7 +210,7 @@ def _h_bound(y1_ref, ab1, I):
 @pytest.mark.parametrize("fmt", [MX, NV])
 @pytest.mark.parametrize("case", [([3, 0, 1, 8, 5], 256, 7168), ([300, 0, 1, 129, 77], 256, 512),
                                   ([2, 1], 64, 256), ([131], 128, 2048), ([20, 0, 150], 128, 768),
-                                  ([200, 9], 384, 1024), ([100, 30], 96, 1024)])
+                                  ([200, 9], 384, 1024), ([100, 30], 96, 1024), ([5, 16, 2], 192, 1024)])
 def test_fc1_fused_swiglu_requant(fmt, case):
     seg, I, K = case
     offsets, a, w, gw = _grouped_problem(seg, 2 * I, K, fmt, stream=21)
