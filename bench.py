@@ -4,7 +4,7 @@ weights on B200 (sm_100a), through the library's C ABI.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
 A step is one whole layer (route -> quantise -> permute -> FC1 + SwiGLU +
-requantise -> FC2 -> combine) over one batch of T synthetic tokens.  Default
+requantise -> FC2 + weighted combine) over one batch of T synthetic tokens.  Default
 workload: the prefill layer (T = 2048, E = 256, top-6, d = 7168, I = 2048,
 MXFP4, skewed router bias).  Under torchrun every rank runs its own replica
 on its own GPU (independent token shards, no data-path collective; weak
@@ -244,11 +244,10 @@ def run_ours(args, rank, world, local_rank):
                                    ds4g.EPI_SWIGLU_REQUANT, out_q=b["hq"])
         if ev is not None:
             ev[1].record(st)
-        ds4g.ds4g_grouped_gemm_fp4(b["hq"], b["offsets"], layer.E, wl.T, layer.w2, layer.d, ds4g.EPI_NONE,
-                                   out=b["y2"])
-        ds4g.ds4g_moe_combine(b["y2"], b["s2r"][:wl.S], b["w"], out=b["out"])
+        ds4g.ds4g_grouped_gemm_fp4_combine(b["hq"], b["offsets"], layer.E, wl.T, layer.w2, layer.d, b["r2s"], b["w"],
+                                           out=b["out"])
 
-    # the layer step as one CUDA graph (all seven library calls, no host work)
+    # the layer step as one CUDA graph (all its library calls, no host work)
     graph, gout = layer.capture(x, lg)
     for _ in range(args.warmup):
         graph.replay()
@@ -256,7 +255,9 @@ def run_ours(args, rank, world, local_rank):
     ds4g.ds4g_check_device()
     offsets = b["offsets"].cpu().numpy()
     alg = algorithmic(wl, offsets)
-    launches_per_step = (1 + (1 if wl.fmt == 0 else 3) + 4 + 1 + 1 + 1)
+    # route, quantise (NV: amax, g, quantise), permute (1 CTA kernel up to 512
+    # slots, else 4), FC1 + SwiGLU/requant, FC2 + combine
+    launches_per_step = 1 + (1 if wl.fmt == 0 else 3) + (1 if wl.S <= 512 else 4) + 1 + 1
 
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
@@ -353,7 +354,7 @@ def run_ours(args, rank, world, local_rank):
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": wl.T * wl.d * 2 + wl.T * wl.E * 4,
                 "d2h_bytes_per_step": wl.T * wl.d * 4},
         "gpu_launches": launches_per_step * args.steps,
-        "step_mode": "CUDA graph of the seven library calls",
+        "step_mode": "CUDA graph of the layer's library calls",
         "clocks": clk.summary(),
     }
     return line

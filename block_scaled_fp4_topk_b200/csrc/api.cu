@@ -117,12 +117,11 @@ ds4g_status ds4g_moe_permute(const int32_t* idx, int T, int k, int E, const ds4g
                                       S(stream)));
 }
 
-ds4g_status ds4g_grouped_gemm_fp4(const ds4g_fp4* a, const int32_t* offsets, int E, int max_rows_per_expert,
-                                  const ds4g_fp4* w, int N, int epilogue, float* out, ds4g_fp4* out_q,
-                                  float* h_debug, void* stream)
+static ds4g_status grouped_gemm(const ds4g_fp4* a, const int32_t* offsets, int E, int max_rows_per_expert,
+                                const ds4g_fp4* w, int N, int epilogue, float* out, ds4g_fp4* out_q, float* h_debug,
+                                const int32_t* row_to_slot, const float* route_w, int k, int T, void* stream)
 {
     if (!a || !w || !offsets || E < 1 || N < 1 || max_rows_per_expert < 0) return DS4G_ERR_INVALID_ARG;
-    if (epilogue != DS4G_EPI_NONE && epilogue != DS4G_EPI_SWIGLU_REQUANT) return DS4G_ERR_INVALID_ARG;
     const int fmt = a->fmt;
     if (fmt != DS4G_MXFP4 && fmt != DS4G_NVFP4) return DS4G_ERR_INVALID_ARG;
     const int64_t K = a->K;
@@ -135,12 +134,12 @@ ds4g_status ds4g_grouped_gemm_fp4(const ds4g_fp4* a, const int32_t* offsets, int
     // tensor-core kernel (weights as the MMA's M side) when the tiling fits;
     // longer segments the 128 x 256 tensor-core kernel; shapes neither fits
     // take the dp4a GEMV kernel (any segment length)
-    const bool tc_shape = gemm_tc_supports(fmt, K) &&
-                          (epilogue == DS4G_EPI_NONE ? (N % 256 == 0) : (N % 2 == 0 && (N / 2) % 128 == 0));
+    const bool swiglu = epilogue == DS4G_EPI_SWIGLU_REQUANT;
+    const bool tc_shape = gemm_tc_supports(fmt, K) && (!swiglu ? (N % 256 == 0) : (N % 2 == 0 && (N / 2) % 128 == 0));
     const bool dtc = max_rows_per_expert <= 16 && gemv_tc_supports(fmt, K, N, epilogue);
     const bool gemv = !dtc && (max_rows_per_expert <= 8 || !tc_shape);
     const int64_t Sr = a->rows;
-    if (epilogue == DS4G_EPI_NONE) {
+    if (!swiglu) {
         if (Sr > 0 && (!out || !aligned16(out))) return DS4G_ERR_INVALID_ARG;
         if (N % 64 != 0) return DS4G_ERR_SHAPE;
     } else {
@@ -172,7 +171,34 @@ ds4g_status ds4g_grouped_gemm_fp4(const ds4g_fp4* a, const int32_t* offsets, int
     g.oq_g = out_q ? out_q->g : nullptr;
     g.h_debug = h_debug;
     g.max_rows = max_rows_per_expert;
+    g.r2s = row_to_slot;
+    g.route_w = route_w;
+    g.topk = k;
+    if (epilogue == kEpiCombine && T > 0) {
+        cudaError_t e = cudaMemsetAsync(out, 0, sizeof(float) * (size_t)T * N, S(stream));
+        if (e != cudaSuccess) return DS4G_ERR_CUDA;
+    }
     return cuda_status(dtc ? launch_gemv_tc(g, S(stream)) : gemv ? launch_gemv(g, S(stream)) : launch_gemm_tc(g, S(stream)));
+}
+
+ds4g_status ds4g_grouped_gemm_fp4(const ds4g_fp4* a, const int32_t* offsets, int E, int max_rows_per_expert,
+                                  const ds4g_fp4* w, int N, int epilogue, float* out, ds4g_fp4* out_q,
+                                  float* h_debug, void* stream)
+{
+    if (epilogue != DS4G_EPI_NONE && epilogue != DS4G_EPI_SWIGLU_REQUANT) return DS4G_ERR_INVALID_ARG;
+    return grouped_gemm(a, offsets, E, max_rows_per_expert, w, N, epilogue, out, out_q, h_debug, nullptr, nullptr, 0,
+                        0, stream);
+}
+
+ds4g_status ds4g_grouped_gemm_fp4_combine(const ds4g_fp4* a, const int32_t* offsets, int E, int max_rows_per_expert,
+                                          const ds4g_fp4* w, int N, const int32_t* row_to_slot, const float* route_w,
+                                          int T, int k, float* out, void* stream)
+{
+    if (T < 0 || k < 1) return DS4G_ERR_INVALID_ARG;
+    if (a && a->rows != (int64_t)T * k) return DS4G_ERR_SHAPE;
+    if (T > 0 && (!row_to_slot || !route_w || !out)) return DS4G_ERR_INVALID_ARG;
+    return grouped_gemm(a, offsets, E, max_rows_per_expert, w, N, kEpiCombine, out, nullptr, nullptr, row_to_slot,
+                        route_w, k, T, stream);
 }
 
 ds4g_status ds4g_swiglu_requant(const float* y1, int64_t rows, int I, int fmt, ds4g_fp4* h_q, float* h_debug,

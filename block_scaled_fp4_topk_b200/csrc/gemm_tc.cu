@@ -509,18 +509,30 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
             const int64_t row = tl.m0 + 32 * q + lane;
             const bool valid = row < tl.end;
             const uint32_t tbase = tmem + kColAcc + ((uint32_t)(32 * q) << 16);
-            if (EPI == DS4G_EPI_NONE) {
+            if (EPI != DS4G_EPI_SWIGLU_REQUANT) {
+                // plain: store the row; combine: add w * row into its token's output
+                float* dst_row = p.out + row * p.N;
+                float wr = gscale;
+                if (EPI == kEpiCombine && valid) {
+                    const int32_t s = p.r2s[row];
+                    dst_row = p.out + (int64_t)(s / p.topk) * p.N;
+                    wr = p.route_w[s] * gscale;
+                }
 #pragma unroll 1
                 for (int c8 = 0; c8 < 4; ++c8) {
                     const int col = half * 128 + 32 * c8;
                     float v[32];
                     tmem_ld32(tbase + col, v);
                     if (valid) {
-                        float4* dst = reinterpret_cast<float4*>(p.out + row * p.N + (int64_t)tl.nt * BN + col);
+                        float* dst = dst_row + (int64_t)tl.nt * BN + col;
 #pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            dst[i] = make_float4(v[4 * i] * gscale, v[4 * i + 1] * gscale, v[4 * i + 2] * gscale,
-                                                 v[4 * i + 3] * gscale);
+                        for (int i = 0; i < 8; ++i) {
+                            if (EPI == kEpiCombine)
+                                red_add_v4(dst + 4 * i, v[4 * i] * wr, v[4 * i + 1] * wr, v[4 * i + 2] * wr, v[4 * i + 3] * wr);
+                            else
+                                reinterpret_cast<float4*>(dst)[i] =
+                                    make_float4(v[4 * i] * wr, v[4 * i + 1] * wr, v[4 * i + 2] * wr, v[4 * i + 3] * wr);
+                        }
                     }
                 }
             } else {
@@ -668,8 +680,10 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st)
     if (a.E > tc::kMaxE || !gemm_tc_supports(a.fmt, a.K)) return cudaErrorInvalidValue;
     if (a.fmt == DS4G_MXFP4)
         return a.epilogue == DS4G_EPI_NONE ? run_tc<DS4G_MXFP4, DS4G_EPI_NONE>(a, st)
+             : a.epilogue == kEpiCombine   ? run_tc<DS4G_MXFP4, kEpiCombine>(a, st)
                                            : run_tc<DS4G_MXFP4, DS4G_EPI_SWIGLU_REQUANT>(a, st);
     return a.epilogue == DS4G_EPI_NONE ? run_tc<DS4G_NVFP4, DS4G_EPI_NONE>(a, st)
+         : a.epilogue == kEpiCombine   ? run_tc<DS4G_NVFP4, kEpiCombine>(a, st)
                                        : run_tc<DS4G_NVFP4, DS4G_EPI_SWIGLU_REQUANT>(a, st);
 }
 

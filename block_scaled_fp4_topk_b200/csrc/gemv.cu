@@ -225,8 +225,15 @@ k_gemv(const GemmArgs p)
             for (int rr = 0; rr < MAXR; ++rr) {
                 if (rr == lane && rr < nr) {
 #pragma unroll
-                    for (int i = 0; i < NR; ++i)
-                        p.out[(rg + rr) * p.N + (blockIdx.x * (NW * NR) + warp * NR + i)] = acc[i][rr];
+                    for (int i = 0; i < NR; ++i) {
+                        const int64_t n = blockIdx.x * (NW * NR) + warp * NR + i;
+                        if (EPI == kEpiCombine) {
+                            const int32_t s = p.r2s[rg + rr];
+                            atomicAdd(p.out + (int64_t)(s / p.topk) * p.N + n, acc[i][rr] * p.route_w[s]);
+                        } else {
+                            p.out[(rg + rr) * p.N + n] = acc[i][rr];
+                        }
+                    }
                 }
             }
         } else {
@@ -321,8 +328,10 @@ cudaError_t launch_gemv(const GemmArgs& a, cudaStream_t st)
     if (a.S == 0) return cudaSuccess;
     if (a.fmt == DS4G_MXFP4)
         return a.epilogue == DS4G_EPI_NONE ? pick_rows<DS4G_MXFP4, DS4G_EPI_NONE>(a, st)
+             : a.epilogue == kEpiCombine   ? pick_rows<DS4G_MXFP4, kEpiCombine>(a, st)
                                            : pick_rows<DS4G_MXFP4, DS4G_EPI_SWIGLU_REQUANT>(a, st);
     return a.epilogue == DS4G_EPI_NONE ? pick_rows<DS4G_NVFP4, DS4G_EPI_NONE>(a, st)
+         : a.epilogue == kEpiCombine   ? pick_rows<DS4G_NVFP4, kEpiCombine>(a, st)
                                        : pick_rows<DS4G_NVFP4, DS4G_EPI_SWIGLU_REQUANT>(a, st);
 }
 

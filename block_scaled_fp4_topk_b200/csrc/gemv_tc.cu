@@ -359,8 +359,17 @@ k_gemv_tc(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUt
             if (!kSwiGLU) {
                 const int64_t n = (int64_t)itm.wt * BMW + 32 * q + lane;
 #pragma unroll
-                for (int tt = 0; tt < BNT; ++tt)
-                    if (tt < itm.nr) p.out[(itm.x0 + tt) * p.N + n] = v[tt] * gscale;
+                for (int tt = 0; tt < BNT; ++tt) {
+                    if (tt < itm.nr) {
+                        if (EPI == kEpiCombine) {
+                            // add w * row into its token's output (coalesced along n)
+                            const int32_t s = p.r2s[itm.x0 + tt];
+                            atomicAdd(p.out + (int64_t)(s / p.topk) * p.N + n, v[tt] * gscale * p.route_w[s]);
+                        } else {
+                            p.out[(itm.x0 + tt) * p.N + n] = v[tt] * gscale;
+                        }
+                    }
+                }
             } else {
                 // up rows (warps with q >= 2) -> shared; gate rows compute h
                 asm volatile("bar.sync 1, 128;" ::: "memory");
@@ -439,7 +448,7 @@ static cudaError_t run_dtc(const GemmArgs& a, cudaStream_t st)
 bool gemv_tc_supports(int fmt, int64_t K, int N, int epilogue)
 {
     if (!gemm_tc_supports(fmt, K)) return false;
-    return epilogue == DS4G_EPI_NONE ? (N % 128 == 0) : (N % 2 == 0 && (N / 2) % 64 == 0);
+    return epilogue != DS4G_EPI_SWIGLU_REQUANT ? (N % 128 == 0) : (N % 2 == 0 && (N / 2) % 64 == 0);
 }
 
 cudaError_t launch_gemv_tc(const GemmArgs& a, cudaStream_t st)
@@ -448,8 +457,10 @@ cudaError_t launch_gemv_tc(const GemmArgs& a, cudaStream_t st)
     if (a.E > dtc::kMaxE || !gemv_tc_supports(a.fmt, a.K, a.N, a.epilogue)) return cudaErrorInvalidValue;
     if (a.fmt == DS4G_MXFP4)
         return a.epilogue == DS4G_EPI_NONE ? run_dtc<DS4G_MXFP4, DS4G_EPI_NONE>(a, st)
+             : a.epilogue == kEpiCombine   ? run_dtc<DS4G_MXFP4, kEpiCombine>(a, st)
                                            : run_dtc<DS4G_MXFP4, DS4G_EPI_SWIGLU_REQUANT>(a, st);
     return a.epilogue == DS4G_EPI_NONE ? run_dtc<DS4G_NVFP4, DS4G_EPI_NONE>(a, st)
+         : a.epilogue == kEpiCombine   ? run_dtc<DS4G_NVFP4, kEpiCombine>(a, st)
                                        : run_dtc<DS4G_NVFP4, DS4G_EPI_SWIGLU_REQUANT>(a, st);
 }
 

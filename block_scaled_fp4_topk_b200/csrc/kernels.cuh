@@ -39,6 +39,9 @@ struct GemmArgs {
     const float* oq_g;
     float* h_debug;
     int max_rows;
+    const int32_t* r2s;      // combine epilogue: row -> slot, routing weights, k
+    const float* route_w;
+    int topk;
 };
 
 cudaError_t launch_gemv(const GemmArgs& a, cudaStream_t st);

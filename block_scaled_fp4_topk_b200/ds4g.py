@@ -52,6 +52,7 @@ _SIGS = {
     "ds4g_moe_permute": ([_vp, _i32, _i32, _i32, _P, _vp, _vp, _vp, _P, _vp, _sz, _vp], _i32),
     "ds4g_grouped_gemm_fp4": ([_P, _vp, _i32, _i32, _P, _i32, _i32, _vp, _P, _vp, _vp], _i32),
     "ds4g_swiglu_requant": ([_vp, _i64, _i32, _i32, _P, _vp, _vp], _i32),
+    "ds4g_grouped_gemm_fp4_combine": ([_P, _vp, _i32, _i32, _P, _i32, _vp, _vp, _i32, _i32, _vp, _vp], _i32),
     "ds4g_moe_combine": ([_vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp], _i32),
     "ds4g_permute_static_max_bytes": ([], _sz),
     "ds4g_moe_permute_static": ([_vp, _i32, _i32, _i32, _P, _vp, _vp, _vp, _P, _vp], _i32),
@@ -199,6 +200,19 @@ def ds4g_grouped_gemm_fp4(a, offsets, E, max_rows_per_expert, w, N, epilogue=EPI
                                       N, epilogue, _ptr(out), ctypes.byref(qc) if qc is not None else None,
                                       _ptr(h_debug), _stream()))
     return out if epilogue == EPI_NONE else out_q
+
+
+def ds4g_grouped_gemm_fp4_combine(a, offsets, E, max_rows_per_expert, w, N, row_to_slot, route_w, out=None):
+    """FC2 with the weighted combine fused: out [T][N] (zeroed by the call)."""
+    T, k = route_w.shape
+    if out is None:
+        out = torch.empty((T, N), dtype=torch.float32, device=a.data.device)
+    ac, wc = a.c(), w.c()
+    _check("ds4g_grouped_gemm_fp4_combine",
+           _lib.ds4g_grouped_gemm_fp4_combine(ctypes.byref(ac), offsets.data_ptr(), E, max_rows_per_expert,
+                                              ctypes.byref(wc), N, row_to_slot.data_ptr(), route_w.data_ptr(), T, k,
+                                              out.data_ptr(), _stream()))
+    return out
 
 
 def ds4g_swiglu_requant(y1, fmt, h_q=None, h_debug=None, g_h=None):

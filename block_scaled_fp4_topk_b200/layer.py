@@ -1,6 +1,7 @@
 """One routed-expert MoE FFN layer with block-scaled FP4 expert weights,
 run as the sequence of libds4g calls (route -> quantise -> permute -> FC1
-with fused SwiGLU + requantisation -> FC2 -> combine) on one stream.
+with fused SwiGLU + requantisation -> FC2 with the weighted combine fused;
+the unfused SwiGLU and combine steps are available as options) on one stream.
 
 All arithmetic happens in the library's kernels; this module only owns the
 device buffers and issues the calls.
@@ -12,13 +13,14 @@ from .ds4g import EPI_NONE, EPI_SWIGLU_REQUANT, NVFP4, Fp4Tensor
 
 
 class MoeLayer:
-    def __init__(self, w1, w2, E, k, d, I, fmt, g_h=None, fused=True):
+    def __init__(self, w1, w2, E, k, d, I, fmt, g_h=None, fused=True, fused_combine=True):
         """w1: Fp4Tensor [E*2I][d] (gate rows then up rows per expert),
         w2: Fp4Tensor [E*d][I]; NVFP4 weights carry one tensor scale per
         expert (w.g has E floats); g_h: the static NVFP4 tensor scale of h."""
         self.w1, self.w2 = w1, w2
         self.E, self.k, self.d, self.I, self.fmt = E, k, d, I, fmt
         self.fused = fused
+        self.fused_combine = fused_combine
         self.g_h = None
         if fmt == NVFP4:
             dev = w1.data.device
@@ -39,7 +41,6 @@ class MoeLayer:
                 s2r=torch.empty(max(S, 1), dtype=torch.int32, device=device),
                 a=Fp4Tensor.empty(S, self.d, self.fmt, device),
                 hq=Fp4Tensor.empty(S, self.I, self.fmt, device),
-                y2=torch.empty((S, self.d), dtype=torch.float32, device=device),
                 out=torch.empty((T, self.d), dtype=torch.float32, device=device),
                 pws=ds4g.permute_workspace(T, self.k, self.E, device),
                 qws=torch.empty(16, dtype=torch.uint8, device=device),
@@ -48,6 +49,8 @@ class MoeLayer:
                 b["hq"].g = self.g_h
             if not self.fused:
                 b["y1"] = torch.empty((S, 2 * self.I), dtype=torch.float32, device=device)
+            if not self.fused_combine:
+                b["y2"] = torch.empty((S, self.d), dtype=torch.float32, device=device)
             self._bufs[key] = b
         return b
 
@@ -65,8 +68,12 @@ class MoeLayer:
         else:
             ds4g.ds4g_grouped_gemm_fp4(b["a"], b["offsets"], self.E, T, self.w1, 2 * self.I, EPI_NONE, out=b["y1"])
             ds4g.ds4g_swiglu_requant(b["y1"], self.fmt, h_q=b["hq"], h_debug=h_debug)
-        ds4g.ds4g_grouped_gemm_fp4(b["hq"], b["offsets"], self.E, T, self.w2, self.d, EPI_NONE, out=b["y2"])
-        ds4g.ds4g_moe_combine(b["y2"], b["s2r"][:T * self.k], b["w"], out=b["out"])
+        if self.fused_combine:
+            ds4g.ds4g_grouped_gemm_fp4_combine(b["hq"], b["offsets"], self.E, T, self.w2, self.d, b["r2s"],
+                                               b["w"], out=b["out"])
+        else:
+            ds4g.ds4g_grouped_gemm_fp4(b["hq"], b["offsets"], self.E, T, self.w2, self.d, EPI_NONE, out=b["y2"])
+            ds4g.ds4g_moe_combine(b["y2"], b["s2r"][:T * self.k], b["w"], out=b["out"])
         return b["out"]
 
     def capture(self, x, logits):

@@ -165,6 +165,21 @@ ds4g_status ds4g_grouped_gemm_fp4(const ds4g_fp4* a, const int32_t* offsets, int
                                   float* out, ds4g_fp4* out_q, float* h_debug, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * FC2 with the combine fused ("Moore Threads ..." MoE combine, folded into
+ * the GEMM's epilogue): the same grouped GEMM as ds4g_grouped_gemm_fp4 (a has
+ * S = T*k rows), but instead of storing y[r][:] each row adds
+ * route_w[s] * y[r][:] into out[s / k][:], s = row_to_slot[r].  out fp32
+ * [T][N] is zeroed by the call first.  The adds are fp32 atomics, so the
+ * order in which a token's k rows are summed is not fixed (results can
+ * differ in the last bits from run to run; ds4g_moe_combine is the
+ * deterministic alternative).  Kernel choice and shapes as for
+ * ds4g_grouped_gemm_fp4 with DS4G_EPI_NONE. */
+ds4g_status ds4g_grouped_gemm_fp4_combine(const ds4g_fp4* a, const int32_t* offsets, int E,
+                                          int max_rows_per_expert, const ds4g_fp4* w, int N,
+                                          const int32_t* row_to_slot, const float* route_w, int T, int k,
+                                          float* out, void* stream);
+
+/* ---------------------------------------------------------------------------
  * The SwiGLU + requantisation epilogue as its own step ("Moore Threads ..."
  * fused SwiGLU + quant pattern): y1 fp32 [rows][2I] -> h_q (fmt, [rows][I]);
  * h_debug (nullable) receives h fp32.  For NVFP4 *h_q->g is the static

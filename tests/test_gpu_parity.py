@@ -246,6 +246,37 @@ def test_swiglu_requant(fmt):
     check_requant(from_dev(hq), h_ref, dh, fmt, g=g_h, min_exact=0.9999)
 
 
+# ---- FC2 with the combine fused --------------------------------------------------------
+
+@pytest.mark.parametrize("fmt", [MX, NV])
+@pytest.mark.parametrize("T,k,E,N,K", [(300, 6, 16, 512, 1024),    # tensor-core kernel
+                                       (3, 6, 64, 256, 1024),      # decode tensor-core kernel
+                                       (4, 2, 8, 128, 256)])       # dp4a kernel (MX) / decode tc (NV)
+def test_fc2_combine_fused(fmt, T, k, E, N, K):
+    lg = synth.logits(T, E, 0, 1.5)
+    idx, w = oracle.route_topk(lg, k)
+    offsets, r2s, s2r = oracle.moe_permute(idx, E)
+    S = T * k
+    a = oracle.quantize(_x_f32(S, K, 51), fmt)
+    wf = synth.normal_f32((E * N, K), 0, 52, 0.02)
+    if fmt == NV:
+        ws = [oracle.quantize(wf[e * N:(e + 1) * N], NV) for e in range(E)]
+        W = oracle.Fp4(np.concatenate([t.data for t in ws]), np.concatenate([t.scales for t in ws]), 1.0, NV)
+        gw = [t.g for t in ws]
+    else:
+        W, gw = oracle.quantize(wf, MX), None
+    w32 = w.astype(np.float32)
+    out = ds4g.ds4g_grouped_gemm_fp4_combine(to_dev(a), torch.from_numpy(offsets).to(dev()), E, T,
+                                             to_dev(W, g_per_expert=gw), N, torch.from_numpy(r2s).to(dev()), torch.from_numpy(w32).to(dev()))
+    ds4g.ds4g_check_device()
+    y2, ab = _ref_gemm(a, offsets, W, gw, N)
+    ref = oracle.moe_combine(y2, s2r, w32.astype(np.float64))
+    bound = (oracle.moe_combine(1e-5 * ab + 1e-6, s2r, np.abs(w32.astype(np.float64))) +
+             1e-6 * oracle.moe_combine(np.abs(y2), s2r, np.abs(w32.astype(np.float64))) + 1e-7)
+    got = out.cpu().numpy()
+    assert np.all(np.abs(got - ref) <= bound), f"worst excess {(np.abs(got - ref) - bound).max():.3e}"
+
+
 # ---- combine -----------------------------------------------------------------------
 
 def test_combine():
@@ -264,13 +295,13 @@ def test_combine():
 
 # ---- full layer --------------------------------------------------------------------
 
-@pytest.mark.parametrize("fused", [True, False])
-def test_layer_tiny(fused):
+@pytest.mark.parametrize("fused,fused_combine", [(True, True), (False, False), (True, False)])
+def test_layer_tiny(fused, fused_combine):
     from synth import workloads
     from block_scaled_fp4_topk_b200.layer import MoeLayer
     wl = workloads.WORKLOADS["tiny"]
     w1, w2 = MoeLayer.synthetic_weights(wl.E, wl.d, wl.I, wl.fmt, device=dev())
-    layer = MoeLayer(w1, w2, wl.E, wl.k, wl.d, wl.I, wl.fmt, fused=fused)
+    layer = MoeLayer(w1, w2, wl.E, wl.k, wl.d, wl.I, wl.fmt, fused=fused, fused_combine=fused_combine)
     xb = workloads.host_x_bits(wl)
     lg = workloads.host_logits(wl)
     out = layer.forward(bf16_dev(xb), torch.from_numpy(lg).to(dev())).cpu().numpy()
