@@ -267,7 +267,8 @@ def test_fc2_combine_fused(fmt, T, k, E, N, K):
         W, gw = oracle.quantize(wf, MX), None
     w32 = w.astype(np.float32)
     out = ds4g.ds4g_grouped_gemm_fp4_combine(to_dev(a), torch.from_numpy(offsets).to(dev()), E, T,
-                                             to_dev(W, g_per_expert=gw), N, torch.from_numpy(r2s).to(dev()), torch.from_numpy(w32).to(dev()))
+                                             to_dev(W, g_per_expert=gw), N, torch.from_numpy(r2s).to(dev()),
+                                             torch.from_numpy(w32).to(dev()))
     ds4g.ds4g_check_device()
     y2, ab = _ref_gemm(a, offsets, W, gw, N)
     ref = oracle.moe_combine(y2, s2r, w32.astype(np.float64))
