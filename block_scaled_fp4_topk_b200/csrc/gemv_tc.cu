@@ -13,11 +13,11 @@
 //   warp 0  TMA producer: weight tile (128 rows x 256 K) and the expert's
 //           activation rows (16 rows x 256 K), 8 stages; row-major scale
 //           boxes of both (512 K per scale stage, 4 scale stages)
-//   warp 1  MMA issuer: scales -> TMEM (tcgen05.cp), 4 MMAs per stage,
-//           double-buffered 16-column accumulators
+//   warps 1, 3  MMA issuers, alternate K stages: scales -> TMEM (tcgen05.cp),
+//           4 MMAs per stage, double-buffered 16-column accumulators each
+//           (the epilogue adds the two); warp 3 also allocates TMEM
 //   warp 2  scale transposer (weights in place; activations into zeroed
 //           128-line chunks of which lines 0..15 carry the 16 rows)
-//   warp 3  TMEM allocator
 //   warps 4-7  epilogue: thread = weight row, 16 token columns; the plain
 //           fp32 store is coalesced along the weight rows; FC1 exchanges the up
 //           rows through shared memory and quantises h along 32-column blocks
@@ -46,9 +46,8 @@ constexpr int kThreads = 256;
 constexpr int W_BYTES = BMW * BKB;   // 16 KB
 constexpr int X_BYTES = BNT * BKB;   // 2 KB
 constexpr int kTmemCols = 128;
-constexpr int kColAcc = 0;         // two 16-column accumulators
-constexpr int kColSFW = 32;
-constexpr int kColSFX = 64;
+constexpr int kColAcc = 0;         // [issuer][buffer] 16-column accumulators: 64 columns
+constexpr int kColSF = 64;         // [issuer] 16 weight-scale then 16 activation-scale columns
 constexpr int kMaxE = 1024;
 
 template <int FMT>
@@ -173,10 +172,10 @@ k_gemv_tc(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUt
         for (int r = 0; r < SF_STAGES; ++r) {
             mbar_init(smem_u32(&sf_full[r]), 1);
             mbar_init(smem_u32(&sf_ready[r]), 1);
-            mbar_init(smem_u32(&sf_empty[r]), 1);
+            mbar_init(smem_u32(&sf_empty[r]), 2);
         }
         for (int b2 = 0; b2 < 2; ++b2) {
-            mbar_init(smem_u32(&tmem_full[b2]), 1);
+            mbar_init(smem_u32(&tmem_full[b2]), 2);
             mbar_init(smem_u32(&tmem_empty[b2]), 128);
         }
         *abort_flag = 0;
@@ -270,23 +269,33 @@ k_gemv_tc(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUt
             }
         }
         __syncwarp();
-    } else if (warp == 1) {
-        // ================= MMA issuer =================
+    } else if (warp == 1 || warp == 3) {
+        // ================= MMA issuers =================
+        // Two threads share the K stages of every item, even and odd global
+        // stage index, each with its own accumulators and scale columns.  A
+        // thread that has issued tensor-core work and then waits on a barrier
+        // (or reads anything it branches on) first waits for that work to
+        // complete, so a single issuer leaves the tensor pipe idle at every
+        // stage boundary; with two, one issues while the other drains.
         if (lane == 0) {
+            const int pi = (warp == 1) ? 0 : 1;
             const uint32_t ibase = (1u << 7) | (1u << 10) | ((uint32_t)(BNT >> 3) << 17) |
                                    ((FMT == DS4G_MXFP4 ? 1u : 0u) << 23) | ((uint32_t)(BMW >> 4) << 24);
-            uint32_t it = 0, sit = 0, tcount = 0;
+            const uint32_t col_sfw = tmem + kColSF + pi * 32, col_sfx = col_sfw + 16;
+            uint32_t tcount = 0;
             bool ok = true;
             for (int64_t t = blockIdx.x; t < nitems && ok; t += gridDim.x, ++tcount) {
                 const int buf = tcount & 1;
                 if (!mbar_wait(smem_u32(&tmem_empty[buf]), ((tcount >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t acc = tmem + kColAcc + buf * BNT;
-                for (int ks = 0; ks < nks; ++ks, ++it) {
+                const uint32_t acc = tmem + kColAcc + pi * 32 + buf * BNT;
+                const uint32_t it0 = tcount * (uint32_t)nks;       // global index of the item's first stage
+                const uint32_t sit0 = tcount * (uint32_t)npairs;
+                bool first = true;
+                for (int ks = pi ^ (int)(it0 & 1); ks < nks; ks += 2) {
+                    const uint32_t it = it0 + ks, sit = sit0 + ks / 2;
                     const int r = sit % SF_STAGES;
-                    if ((ks & 1) == 0) {
-                        if (!mbar_wait(smem_u32(&sf_ready[r]), (sit / SF_STAGES) & 1, abort_flag)) { ok = false; break; }
-                    }
+                    if (!mbar_wait(smem_u32(&sf_ready[r]), (sit / SF_STAGES) & 1, abort_flag)) { ok = false; break; }
                     const int s = it % STAGES;
                     if (!mbar_wait(smem_u32(&full[s]), (it / STAGES) & 1, abort_flag)) { ok = false; break; }
                     tc_fence_after();
@@ -295,8 +304,8 @@ k_gemv_tc(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUt
                     const uint32_t sfx_s = smem_u32(sSFXC + r * C::SFXC_BYTES);
 #pragma unroll
                     for (int c = 0; c < C::WPS; ++c) {
-                        utccp(tmem + kColSFW + 4 * c, desc_sf(sfw_s + (w0 + c) * 512));
-                        utccp(tmem + kColSFX + 4 * c, desc_sf(sfx_s + (w0 + c) * 512));
+                        utccp(col_sfw + 4 * c, desc_sf(sfw_s + (w0 + c) * 512));
+                        utccp(col_sfx + 4 * c, desc_sf(sfx_s + (w0 + c) * 512));
                     }
                     const int64_t krem = K - (int64_t)ks * BK;
                     const int nmma = krem >= BK ? 4 : (int)(krem / 64);
@@ -309,17 +318,18 @@ k_gemv_tc(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUt
                             const uint32_t sfid = (FMT == DS4G_MXFP4) ? (uint32_t)((j & 1) * 2) : 0u;
                             const uint32_t idesc = ibase | (sfid << 4) | (sfid << 29);
                             mma<FMT>(acc, desc_sw128(w_s + 32 * j), desc_sw128(x_s + 32 * j), idesc,
-                                     (ks > 0 || j > 0) ? 1u : 0u, tmem + kColSFW + 4 * c, tmem + kColSFX + 4 * c);
+                                     (!first || j > 0) ? 1u : 0u, col_sfw + 4 * c, col_sfx + 4 * c);
                         }
                     }
+                    first = false;
                     tc_commit(smem_u32(&empty[s]));
-                    if ((ks & 1) == 1 || ks == nks - 1) {
-                        tc_commit(smem_u32(&sf_empty[r]));
-                        ++sit;
-                    }
+                    // the scale stage is released by two commits: one per data
+                    // stage it covers, twice when it covers only one
+                    tc_commit(smem_u32(&sf_empty[r]));
+                    if ((ks & 1) == 0 && ks == nks - 1) tc_commit(smem_u32(&sf_empty[r]));
                 }
                 if (!ok) break;
-                tc_commit(smem_u32(&tmem_full[buf]));
+                tc_commit(smem_u32(&tmem_full[buf]));             // also when this issuer had no stage
             }
         }
         __syncwarp();
@@ -352,8 +362,19 @@ k_gemv_tc(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUt
             tc_fence_after();
             const Item itm = item_of(t, prefix, p.offsets, E, wtiles);
             const float gscale = (FMT == DS4G_NVFP4) ? __fmul_rn(p.a_g[0], p.w_g[itm.e]) : 1.0f;
+            // issuer i holds the sum over the stages of parity i (global index)
+            const uint32_t it0 = tcount * (uint32_t)nks;
+            const uint32_t lanes = (uint32_t)(32 * q) << 16;
             float v[16];
-            tmem_ld16(tmem + kColAcc + buf * BNT + ((uint32_t)(32 * q) << 16), v);
+            if (nks >= 2) {
+                float v1[16];
+                tmem_ld16(tmem + kColAcc + buf * BNT + lanes, v);
+                tmem_ld16(tmem + kColAcc + 32 + buf * BNT + lanes, v1);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) v[i] += v1[i];
+            } else {
+                tmem_ld16(tmem + kColAcc + (it0 & 1) * 32 + buf * BNT + lanes, v);
+            }
             tc_fence_before();
             mbar_arrive(smem_u32(&tmem_empty[buf]));          // accumulator drained into registers
             if (!kSwiGLU) {

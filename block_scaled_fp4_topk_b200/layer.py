@@ -58,16 +58,28 @@ class MoeLayer:
         """x: bf16 [T][d] (device), logits: fp32 [T][E] (device) -> fp32 [T][d]"""
         T = x.shape[0]
         b = self.buffers(T, x.device)
+        self.dispatch(x, logits, b)
+        self.fc1(b, T, h_debug)
+        return self.fc2(b, T)
+
+    def dispatch(self, x, logits, b):
+        """routing, activation quantisation and the expert-contiguous permutation"""
         ds4g.ds4g_route_topk(logits, self.k, idx=b["idx"], w=b["w"])
         ds4g.ds4g_quantize_mx(x, self.fmt, out=b["xq"], workspace=b["qws"])
         ds4g.ds4g_moe_permute(b["idx"], self.E, b["xq"], offsets=b["offsets"], row_to_slot=b["r2s"],
                               slot_to_row=b["s2r"], a_perm=b["a"], workspace=b["pws"])
+
+    def fc1(self, b, T, h_debug=None):
+        """grouped FC1 with SwiGLU and the FP4 requantisation of h"""
         if self.fused:
             ds4g.ds4g_grouped_gemm_fp4(b["a"], b["offsets"], self.E, T, self.w1, 2 * self.I, EPI_SWIGLU_REQUANT,
                                        out_q=b["hq"], h_debug=h_debug)
         else:
             ds4g.ds4g_grouped_gemm_fp4(b["a"], b["offsets"], self.E, T, self.w1, 2 * self.I, EPI_NONE, out=b["y1"])
             ds4g.ds4g_swiglu_requant(b["y1"], self.fmt, h_q=b["hq"], h_debug=h_debug)
+
+    def fc2(self, b, T):
+        """grouped FC2 and the routing-weighted combine into out [T][d]"""
         if self.fused_combine:
             ds4g.ds4g_grouped_gemm_fp4_combine(b["hq"], b["offsets"], self.E, T, self.w2, self.d, b["r2s"],
                                                b["w"], out=b["out"])
@@ -76,19 +88,38 @@ class MoeLayer:
             ds4g.ds4g_moe_combine(b["y2"], b["s2r"][:T * self.k], b["w"], out=b["out"])
         return b["out"]
 
-    def capture(self, x, logits):
-        """Records forward(x, logits) on these (static) input buffers as a CUDA
-        graph; returns (graph, out).  Replaying the graph re-runs the whole
-        layer on whatever x / logits hold at that time."""
+    def _warm(self, x, logits):
         side = torch.cuda.Stream(device=x.device)
         side.wait_stream(torch.cuda.current_stream(x.device))
         with torch.cuda.stream(side):
             self.forward(x, logits)            # first call sets kernel attributes, buffers
         torch.cuda.current_stream(x.device).wait_stream(side)
+
+    def capture(self, x, logits):
+        """Records forward(x, logits) on these (static) input buffers as a CUDA
+        graph; returns (graph, out).  Replaying the graph re-runs the whole
+        layer on whatever x / logits hold at that time."""
+        self._warm(x, logits)
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph):
             out = self.forward(x, logits)
         return graph, out
+
+    def capture_stages(self, x, logits):
+        """The same layer as three graphs replayed in order: dispatch, FC1,
+        FC2 + combine (so that FC1 can be bracketed by events); returns
+        ([g_dispatch, g_fc1, g_fc2], out)."""
+        self._warm(x, logits)
+        T = x.shape[0]
+        b = self.buffers(T, x.device)
+        graphs = [torch.cuda.CUDAGraph() for _ in range(3)]
+        with torch.cuda.graph(graphs[0]):
+            self.dispatch(x, logits, b)
+        with torch.cuda.graph(graphs[1]):
+            self.fc1(b, T)
+        with torch.cuda.graph(graphs[2]):
+            out = self.fc2(b, T)
+        return graphs, out
 
     # -- synthetic weights -----------------------------------------------------
     @staticmethod
