@@ -9,13 +9,15 @@
 // block-scaled MMA as the prefill kernel) leaves the SMs nothing to do but
 // keep TMA copies in flight, so the kernel runs at the rate weights arrive.
 //
-// Roles (one persistent CTA per SM, 256 threads):
-//   warp 0  TMA producer: weight tile (128 rows x 256 K) and the expert's
-//           activation rows (16 rows x 256 K), 8 stages; row-major scale
-//           boxes of both (512 K per scale stage, 4 scale stages)
-//   warps 1, 3  MMA issuers, alternate K stages: scales -> TMEM (tcgen05.cp),
-//           4 MMAs per stage, double-buffered 16-column accumulators each
-//           (the epilogue adds the two); warp 3 also allocates TMEM
+// Roles (one persistent CTA per SM, 288 threads):
+//   warps 0, 8  TMA producers, alternate scale stages: weight tile (128 rows
+//           x 256 K) and the expert's activation rows (16 rows x 256 K), 8
+//           stages; row-major scale boxes of both (512 K per scale stage, 4
+//           scale stages)
+//   warps 1, 3  MMA issuers, alternate scale stages: scales -> TMEM
+//           (tcgen05.cp), 4 MMAs per data stage, double-buffered 16-column
+//           accumulators each (the epilogue adds the two); warp 3 also
+//           allocates TMEM
 //   warp 2  scale transposer (weights in place; activations into zeroed
 //           128-line chunks of which lines 0..15 carry the 16 rows)
 //   warps 4-7  epilogue: thread = weight row, 16 token columns; the plain
@@ -42,7 +44,7 @@ constexpr int BKB = 128;
 constexpr int BK = 256;
 constexpr int STAGES = 8;
 constexpr int SF_STAGES = 4;
-constexpr int kThreads = 256;
+constexpr int kThreads = 288;
 constexpr int W_BYTES = BMW * BKB;   // 16 KB
 constexpr int X_BYTES = BNT * BKB;   // 2 KB
 constexpr int kTmemCols = 128;
@@ -172,7 +174,7 @@ k_gemv_tc(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUt
         for (int r = 0; r < SF_STAGES; ++r) {
             mbar_init(smem_u32(&sf_full[r]), 1);
             mbar_init(smem_u32(&sf_ready[r]), 1);
-            mbar_init(smem_u32(&sf_empty[r]), 2);
+            mbar_init(smem_u32(&sf_empty[r]), 1);
         }
         for (int b2 = 0; b2 < 2; ++b2) {
             mbar_init(smem_u32(&tmem_full[b2]), 2);
@@ -230,53 +232,70 @@ k_gemv_tc(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUt
     const uint32_t tmem = *tmem_slot;
     const int64_t nitems = *total_items;
 
-    if (warp == 0) {
-        // ================= TMA producer =================
+    // A thread that has issued asynchronous work (TMA copies, tensor-core
+    // instructions) and then waits on a barrier, or branches on anything it
+    // reads, first waits for that work to drain.  So producers and MMA
+    // issuers come in pairs that take alternate scale stages (each with its
+    // one or two data stages), and each waits for all the barriers of a scale
+    // stage before issuing any of its work: one drain per scale stage, while
+    // the other thread of the pair keeps the copy engine or the tensor pipe
+    // busy.
+    if (warp == 0 || warp == 8) {
+        // ================= TMA producers =================
         if (lane == 0) {
-            uint32_t it = 0, sit = 0;
+            const int pi = (warp == 0) ? 0 : 1;
+            uint32_t tcount = 0, it_next = 0, sit_next = 0;
             bool ok = true;
-            for (int64_t t = blockIdx.x; t < nitems && ok; t += gridDim.x) {
+            for (int64_t t = blockIdx.x; t < nitems && ok; t += gridDim.x, ++tcount) {
                 const Item itm = item_of(t, prefix, p.offsets, E, wtiles);
                 int64_t y0, y1;
                 w_rows<EPI>(itm, p.N, I, y0, y1);
-                for (int ks = 0; ks < nks; ++ks, ++it) {
-                    if ((ks & 1) == 0) {
-                        const int r = sit % SF_STAGES;
-                        if (!mbar_wait(smem_u32(&sf_empty[r]), ((sit / SF_STAGES) & 1) ^ 1, abort_flag)) { ok = false; break; }
-                        const uint32_t fb = smem_u32(&sf_full[r]);
-                        mbar_arrive_tx(fb, C::SFW_BYTES + C::SFXR_BYTES);
-                        const int x = (ks >> 1) * C::SF_ROW;
-                        tma_load_2d(smem_u32(sSFW + r * C::SFW_BYTES), &map_sfw, fb, x, (int)y0);
-                        if (kSwiGLU) tma_load_2d(smem_u32(sSFW + r * C::SFW_BYTES + C::SFW_BYTES / 2), &map_sfw, fb, x, (int)y1);
-                        tma_load_2d(smem_u32(sSFXR + r * C::SFXR_BYTES), &map_sfx, fb, x, (int)itm.x0);
-                        ++sit;
+                const uint32_t it0 = tcount * (uint32_t)nks, sit0 = tcount * (uint32_t)npairs;
+                for (int j = pi ^ (int)(sit0 & 1); j < npairs; j += 2) {
+                    const uint32_t sit = sit0 + j, ita = it0 + 2 * j;
+                    const int nd = min(2, nks - 2 * j);
+                    const int r = sit % SF_STAGES;
+                    if (!mbar_wait(smem_u32(&sf_empty[r]), ((sit / SF_STAGES) & 1) ^ 1, abort_flag)) { ok = false; break; }
+                    for (int d = 0; d < nd && ok; ++d)
+                        ok = mbar_wait(smem_u32(&empty[(ita + d) % STAGES]), (((ita + d) / STAGES) & 1) ^ 1, abort_flag);
+                    if (!ok) break;
+                    const uint32_t sfb = smem_u32(&sf_full[r]);
+                    mbar_arrive_tx(sfb, C::SFW_BYTES + C::SFXR_BYTES);
+                    const int x = j * C::SF_ROW;
+                    tma_load_2d(smem_u32(sSFW + r * C::SFW_BYTES), &map_sfw, sfb, x, (int)y0);
+                    if (kSwiGLU) tma_load_2d(smem_u32(sSFW + r * C::SFW_BYTES + C::SFW_BYTES / 2), &map_sfw, sfb, x, (int)y1);
+                    tma_load_2d(smem_u32(sSFXR + r * C::SFXR_BYTES), &map_sfx, sfb, x, (int)itm.x0);
+                    for (int d = 0; d < nd; ++d) {
+                        const int s = (ita + d) % STAGES;
+                        const int ks = 2 * j + d;
+                        const uint32_t fb = smem_u32(&full[s]);
+                        mbar_arrive_tx(fb, W_BYTES + X_BYTES);
+                        tma_load_2d(smem_u32(sW + s * W_BYTES), &map_w, fb, ks * BKB, (int)y0);
+                        if (kSwiGLU) tma_load_2d(smem_u32(sW + s * W_BYTES + W_BYTES / 2), &map_w, fb, ks * BKB, (int)y1);
+                        tma_load_2d(smem_u32(sX + s * X_BYTES), &map_x, fb, ks * BKB, (int)itm.x0);
                     }
-                    const int s = it % STAGES;
-                    if (!mbar_wait(smem_u32(&empty[s]), ((it / STAGES) & 1) ^ 1, abort_flag)) { ok = false; break; }
-                    const uint32_t fb = smem_u32(&full[s]);
-                    mbar_arrive_tx(fb, W_BYTES + X_BYTES);
-                    tma_load_2d(smem_u32(sW + s * W_BYTES), &map_w, fb, ks * BKB, (int)y0);
-                    if (kSwiGLU) tma_load_2d(smem_u32(sW + s * W_BYTES + W_BYTES / 2), &map_w, fb, ks * BKB, (int)y1);
-                    tma_load_2d(smem_u32(sX + s * X_BYTES), &map_x, fb, ks * BKB, (int)itm.x0);
+                    it_next = ita + nd;
+                    sit_next = sit + 1;
                 }
             }
             if (!ok) {
+                // let this thread's copies in flight land before the CTA goes
+                // away (stop at the first wait that gives up)
                 volatile int never = 0;
-                for (uint32_t j = (it > STAGES ? it - STAGES : 0); j < it; ++j)
-                    mbar_wait(smem_u32(&full[j % STAGES]), (j / STAGES) & 1, &never);
-                for (uint32_t j = (sit > SF_STAGES ? sit - SF_STAGES : 0); j < sit; ++j)
-                    mbar_wait(smem_u32(&sf_full[j % SF_STAGES]), (j / SF_STAGES) & 1, &never);
+                bool go = true;
+                for (uint32_t j = (it_next > STAGES + 2 ? it_next - STAGES - 2 : 0); j < it_next && go; ++j) {
+                    const uint32_t owner = ((j / nks) * npairs + (j % nks) / 2) & 1;
+                    if ((int)owner == pi) go = mbar_wait(smem_u32(&full[j % STAGES]), (j / STAGES) & 1, &never);
+                }
+                for (uint32_t j = (sit_next > SF_STAGES + 1 ? sit_next - SF_STAGES - 1 : 0); j < sit_next && go; ++j)
+                    if ((int)(j & 1) == pi) go = mbar_wait(smem_u32(&sf_full[j % SF_STAGES]), (j / SF_STAGES) & 1, &never);
             }
         }
         __syncwarp();
     } else if (warp == 1 || warp == 3) {
         // ================= MMA issuers =================
-        // Two threads share the K stages of every item, even and odd global
-        // stage index, each with its own accumulators and scale columns.  A
-        // thread that has issued tensor-core work and then waits on a barrier
-        // (or reads anything it branches on) first waits for that work to
-        // complete, so a single issuer leaves the tensor pipe idle at every
-        // stage boundary; with two, one issues while the other drains.
+        // each with its own accumulators and scale columns; the epilogue adds
+        // the two partial sums
         if (lane == 0) {
             const int pi = (warp == 1) ? 0 : 1;
             const uint32_t ibase = (1u << 7) | (1u << 10) | ((uint32_t)(BNT >> 3) << 17) |
@@ -289,44 +308,46 @@ k_gemv_tc(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUt
                 if (!mbar_wait(smem_u32(&tmem_empty[buf]), ((tcount >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t acc = tmem + kColAcc + pi * 32 + buf * BNT;
-                const uint32_t it0 = tcount * (uint32_t)nks;       // global index of the item's first stage
-                const uint32_t sit0 = tcount * (uint32_t)npairs;
+                const uint32_t it0 = tcount * (uint32_t)nks, sit0 = tcount * (uint32_t)npairs;
                 bool first = true;
-                for (int ks = pi ^ (int)(it0 & 1); ks < nks; ks += 2) {
-                    const uint32_t it = it0 + ks, sit = sit0 + ks / 2;
+                for (int j = pi ^ (int)(sit0 & 1); j < npairs; j += 2) {
+                    const uint32_t sit = sit0 + j, ita = it0 + 2 * j;
+                    const int nd = min(2, nks - 2 * j);
                     const int r = sit % SF_STAGES;
                     if (!mbar_wait(smem_u32(&sf_ready[r]), (sit / SF_STAGES) & 1, abort_flag)) { ok = false; break; }
-                    const int s = it % STAGES;
-                    if (!mbar_wait(smem_u32(&full[s]), (it / STAGES) & 1, abort_flag)) { ok = false; break; }
+                    for (int d = 0; d < nd && ok; ++d)
+                        ok = mbar_wait(smem_u32(&full[(ita + d) % STAGES]), ((ita + d) / STAGES) & 1, abort_flag);
+                    if (!ok) break;
                     tc_fence_after();
-                    const int w0 = (ks & 1) * C::WPS;
                     const uint32_t sfw_s = smem_u32(sSFW + r * C::SFW_BYTES);
                     const uint32_t sfx_s = smem_u32(sSFXC + r * C::SFXC_BYTES);
+                    for (int d = 0; d < nd; ++d) {
+                        const int s = (ita + d) % STAGES;
+                        const int ks = 2 * j + d;
+                        const int w0 = d * C::WPS;
 #pragma unroll
-                    for (int c = 0; c < C::WPS; ++c) {
-                        utccp(col_sfw + 4 * c, desc_sf(sfw_s + (w0 + c) * 512));
-                        utccp(col_sfx + 4 * c, desc_sf(sfx_s + (w0 + c) * 512));
-                    }
-                    const int64_t krem = K - (int64_t)ks * BK;
-                    const int nmma = krem >= BK ? 4 : (int)(krem / 64);
-                    const uint32_t w_s = smem_u32(sW + s * W_BYTES);
-                    const uint32_t x_s = smem_u32(sX + s * X_BYTES);
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        if (j < nmma) {
-                            const int c = (FMT == DS4G_MXFP4) ? (j >> 1) : j;
-                            const uint32_t sfid = (FMT == DS4G_MXFP4) ? (uint32_t)((j & 1) * 2) : 0u;
-                            const uint32_t idesc = ibase | (sfid << 4) | (sfid << 29);
-                            mma<FMT>(acc, desc_sw128(w_s + 32 * j), desc_sw128(x_s + 32 * j), idesc,
-                                     (!first || j > 0) ? 1u : 0u, col_sfw + 4 * c, col_sfx + 4 * c);
+                        for (int c = 0; c < C::WPS; ++c) {
+                            utccp(col_sfw + 4 * c, desc_sf(sfw_s + (w0 + c) * 512));
+                            utccp(col_sfx + 4 * c, desc_sf(sfx_s + (w0 + c) * 512));
                         }
+                        const int64_t krem = K - (int64_t)ks * BK;
+                        const int nmma = krem >= BK ? 4 : (int)(krem / 64);
+                        const uint32_t w_s = smem_u32(sW + s * W_BYTES);
+                        const uint32_t x_s = smem_u32(sX + s * X_BYTES);
+#pragma unroll
+                        for (int jj = 0; jj < 4; ++jj) {
+                            if (jj < nmma) {
+                                const int c = (FMT == DS4G_MXFP4) ? (jj >> 1) : jj;
+                                const uint32_t sfid = (FMT == DS4G_MXFP4) ? (uint32_t)((jj & 1) * 2) : 0u;
+                                const uint32_t idesc = ibase | (sfid << 4) | (sfid << 29);
+                                mma<FMT>(acc, desc_sw128(w_s + 32 * jj), desc_sw128(x_s + 32 * jj), idesc,
+                                         (!first || jj > 0) ? 1u : 0u, col_sfw + 4 * c, col_sfx + 4 * c);
+                            }
+                        }
+                        first = false;
+                        tc_commit(smem_u32(&empty[s]));
                     }
-                    first = false;
-                    tc_commit(smem_u32(&empty[s]));
-                    // the scale stage is released by two commits: one per data
-                    // stage it covers, twice when it covers only one
                     tc_commit(smem_u32(&sf_empty[r]));
-                    if ((ks & 1) == 0 && ks == nks - 1) tc_commit(smem_u32(&sf_empty[r]));
                 }
                 if (!ok) break;
                 tc_commit(smem_u32(&tmem_full[buf]));             // also when this issuer had no stage
@@ -362,18 +383,18 @@ k_gemv_tc(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUt
             tc_fence_after();
             const Item itm = item_of(t, prefix, p.offsets, E, wtiles);
             const float gscale = (FMT == DS4G_NVFP4) ? __fmul_rn(p.a_g[0], p.w_g[itm.e]) : 1.0f;
-            // issuer i holds the sum over the stages of parity i (global index)
-            const uint32_t it0 = tcount * (uint32_t)nks;
+            // issuer i holds the sum over the scale stages of parity i
+            const uint32_t sit0 = tcount * (uint32_t)npairs;
             const uint32_t lanes = (uint32_t)(32 * q) << 16;
             float v[16];
-            if (nks >= 2) {
+            if (npairs >= 2) {
                 float v1[16];
                 tmem_ld16(tmem + kColAcc + buf * BNT + lanes, v);
                 tmem_ld16(tmem + kColAcc + 32 + buf * BNT + lanes, v1);
 #pragma unroll
                 for (int i = 0; i < 16; ++i) v[i] += v1[i];
             } else {
-                tmem_ld16(tmem + kColAcc + (it0 & 1) * 32 + buf * BNT + lanes, v);
+                tmem_ld16(tmem + kColAcc + (sit0 & 1) * 32 + buf * BNT + lanes, v);
             }
             tc_fence_before();
             mbar_arrive(smem_u32(&tmem_empty[buf]));          // accumulator drained into registers
