@@ -11,9 +11,9 @@
 //
 // Roles (one persistent CTA per SM, 288 threads):
 //   warps 0, 8  TMA producers, alternate scale stages: weight tile (128 rows
-//           x 256 K) and the expert's activation rows (16 rows x 256 K), 8
-//           stages; row-major scale boxes of both (512 K per scale stage, 4
-//           scale stages)
+//           x 256 K) and the expert's activation rows (16 rows x 256 K), 10
+//           stages; row-major scale boxes of both (512 K per scale stage, 5
+//           scale stages for MXFP4, 4 for NVFP4)
 //   warps 1, 3  MMA issuers, alternate scale stages: scales -> TMEM
 //           (tcgen05.cp), 4 MMAs per data stage, double-buffered 16-column
 //           accumulators each (the epilogue adds the two); warp 3 also
@@ -42,8 +42,6 @@ constexpr int BMW = 128;           // weight rows per tile (MMA M)
 constexpr int BNT = 16;            // activation rows per tile (MMA N)
 constexpr int BKB = 128;
 constexpr int BK = 256;
-constexpr int STAGES = 8;
-constexpr int SF_STAGES = 4;
 constexpr int kThreads = 288;
 constexpr int W_BYTES = BMW * BKB;   // 16 KB
 constexpr int X_BYTES = BNT * BKB;   // 2 KB
@@ -54,6 +52,10 @@ constexpr int kMaxE = 1024;
 
 template <int FMT>
 struct Cfg {
+    // ring depths: as many 18 KB data stages as shared memory holds next to
+    // the scale stages (each scale stage covers two data stages)
+    static constexpr int STAGES = 10;
+    static constexpr int SF_STAGES = (FMT == DS4G_MXFP4) ? 5 : 4;
     static constexpr int WPS = (FMT == DS4G_MXFP4) ? 2 : 4;    // 4-scale words per row per K stage
     static constexpr int SF_ROW = 2 * WPS * 4;                  // scale bytes per row per scale stage
     static constexpr int SFW_BYTES = BMW * SF_ROW;              // weights, transposed in place
@@ -62,6 +64,8 @@ struct Cfg {
     static constexpr int DATA_BYTES = STAGES * (W_BYTES + X_BYTES);
     static constexpr int SF_BYTES = SF_STAGES * (SFW_BYTES + SFXR_BYTES + SFXC_BYTES);
     static constexpr size_t SMEM = 1024 + (size_t)DATA_BYTES + SF_BYTES + 512 + 64 * 16 * 4 + (kMaxE + 1) * 4;
+    static_assert((2 * STAGES + 3 * SF_STAGES + 4) * 8 + 16 <= 512, "barrier block");
+    static_assert(SMEM <= 232448, "shared memory per CTA");
 };
 
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v)
@@ -136,6 +140,8 @@ k_gemv_tc(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUt
           const __grid_constant__ CUtensorMap map_sfw, const __grid_constant__ CUtensorMap map_sfx, const GemmArgs p)
 {
     using C = Cfg<FMT>;
+    constexpr int STAGES = C::STAGES;
+    constexpr int SF_STAGES = C::SF_STAGES;
     constexpr bool kSwiGLU = (EPI == DS4G_EPI_SWIGLU_REQUANT);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
