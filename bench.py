@@ -284,18 +284,19 @@ def run_ours(args, rank, world, local_rank):
 
     # FC1 timed over the same number of whole steps, bracketed by events on
     # the launching stream between the dispatch and FC2 graphs
-    fc1_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    # (events between all three stage graphs: dispatch, FC1, FC2 + combine)
+    st_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     for i in range(args.steps):
         if flush:
             fbuf.fill_(i & 0xFF)
-        stages[0].replay()
-        fc1_ev[i][0].record(st)
-        stages[1].replay()
-        fc1_ev[i][1].record(st)
-        stages[2].replay()
+        st_ev[i][0].record(st)
+        for g in range(3):
+            stages[g].replay()
+            st_ev[i][g + 1].record(st)
     torch.cuda.synchronize()
     ds4g.ds4g_check_device()
-    fc1_ms = float(np.mean([a.elapsed_time(c) for a, c in fc1_ev]))
+    stage_ms = [float(np.mean([ev[g].elapsed_time(ev[g + 1]) for ev in st_ev])) for g in range(3)]
+    fc1_ms = stage_ms[1]
 
     # end to end through the public API: pinned host inputs -> device, layer, result -> host
     xh = torch.empty((wl.T, wl.d), dtype=torch.bfloat16, pin_memory=True)
@@ -370,6 +371,8 @@ def run_ours(args, rank, world, local_rank):
                 "d2h_bytes_per_step": wl.T * wl.d * 4},
         "gpu_launches": launches_per_step * args.steps,
         "step_mode": "CUDA graph of the layer's library calls",
+        "stage_ms": {"dispatch": stage_ms[0], "fc1_swiglu": stage_ms[1], "fc2_combine": stage_ms[2],
+                     "note": "each stage as its own graph, events between them"},
         "clocks": clk.summary(),
     }
     return line

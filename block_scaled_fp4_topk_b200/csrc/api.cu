@@ -132,16 +132,17 @@ static ds4g_status grouped_gemm(const ds4g_fp4* a, const int32_t* offsets, int E
     if (st != DS4G_OK) return st;
     // kernel choice: decode-sized segments (<= 16 rows) take the swapped
     // tensor-core kernel (weights as the MMA's M side) when the tiling fits;
-    // longer segments the 128 x 256 tensor-core kernel; shapes neither fits
+    // longer segments the 128 x 224 / 128 x 256 tensor-core kernel; shapes neither fits
     // take the dp4a GEMV kernel (any segment length)
     const bool swiglu = epilogue == DS4G_EPI_SWIGLU_REQUANT;
-    const bool tc_shape = gemm_tc_supports(fmt, K) && (!swiglu ? (N % 256 == 0) : (N % 2 == 0 && (N / 2) % 128 == 0));
+    const bool tc_shape = gemm_tc_supports(fmt, K) &&
+                          (!swiglu ? (N % 256 == 0 || N % 224 == 0) : (N % 2 == 0 && (N / 2) % 128 == 0));
     const bool dtc = max_rows_per_expert <= 16 && gemv_tc_supports(fmt, K, N, epilogue);
     const bool gemv = !dtc && (max_rows_per_expert <= 8 || !tc_shape);
     const int64_t Sr = a->rows;
     if (!swiglu) {
         if (Sr > 0 && (!out || !aligned16(out))) return DS4G_ERR_INVALID_ARG;
-        if (N % 64 != 0) return DS4G_ERR_SHAPE;
+        if (gemv && N % 64 != 0) return DS4G_ERR_SHAPE;      // the dp4a kernel's column tiles
     } else {
         if (N % 2 != 0) return DS4G_ERR_SHAPE;
         const int I = N / 2;

@@ -39,7 +39,6 @@ namespace ds4g {
 namespace tc {
 
 constexpr int BM = 128;            // tile rows (tokens)
-constexpr int BN = 256;            // tile columns (weight rows)
 constexpr int BKB = 128;           // bytes of K per stage per row (256 FP4)
 constexpr int BK = 256;            // K elements per stage
 constexpr int STAGES = 4;
@@ -47,20 +46,28 @@ constexpr int SF_STAGES = 2;       // scale stages, each covering two K stages (
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = 32 * (4 + kEpiWarps);
 constexpr int A_BYTES = BM * BKB;  // 16 KB
-constexpr int B_BYTES = BN * BKB;  // 32 KB
 constexpr int kTmemCols = 512;
 constexpr int kColAcc = 0;
-constexpr int kColSFA = 256;
-constexpr int kColSFB = 272;
 constexpr int kMaxE = 1024;
 constexpr unsigned long long kWaitNs = 4000000000ull;
 
-template <int FMT>
+// TBN: tile columns (weight rows).  256 with one accumulator; 224 (for N a
+// multiple of 224, e.g. FC2 with N = 7168) with two, so that the epilogue of
+// one tile overlaps the MMAs of the next: 2 x 224 accumulator columns plus
+// the scale columns fit the 512 TMEM columns, 2 x 256 do not.
+template <int FMT, int TBN>
 struct Cfg {
+    static_assert(TBN == 256 || TBN == 224, "tile width");
+    static constexpr int NACC = (TBN == 256) ? 1 : 2;               // accumulator buffers
+    static constexpr int HALF = TBN / 2;                             // weight rows per TMA box
+    static constexpr int B_BYTES = TBN * BKB;
+    static constexpr int COL_SFA = NACC * TBN;                       // TMEM columns of the scales
+    static constexpr int COL_SFB = COL_SFA + 16;
     static constexpr int WPS = (FMT == DS4G_MXFP4) ? 2 : 4;         // 4-scale words per row per K stage
     static constexpr int SF_ROW = 2 * WPS * 4;                       // scale bytes per row per scale stage
     static constexpr int SFA_BYTES = BM * SF_ROW;                    // one scale stage of A
-    static constexpr int SFB_BYTES = BN * SF_ROW;                    // one scale stage of W
+    static constexpr int SFB_BYTES = 256 * SF_ROW;                   // one scale stage of W (two 128-row groups)
+    static_assert(COL_SFB + 8 * WPS <= kTmemCols, "TMEM columns");
     static constexpr int DATA_BYTES = STAGES * (A_BYTES + B_BYTES);
     static constexpr int SF_BYTES = SF_STAGES * (SFA_BYTES + SFB_BYTES);
     static constexpr size_t SMEM = 1024 + (size_t)DATA_BYTES + SF_BYTES + 256 + (kMaxE + 1) * 4;
@@ -160,11 +167,11 @@ __device__ __forceinline__ uint64_t desc_sf(uint32_t saddr)
 }
 
 // instruction descriptor: E2M1 x E2M1, fp32 accumulate, K-major A and B,
-// N = 256, M = 128; scale format UE8M0 (MX) or UE4M3 (NV)
-template <int FMT>
+// N = TBN, M = 128; scale format UE8M0 (MX) or UE4M3 (NV)
+template <int FMT, int TBN>
 __device__ __forceinline__ uint32_t idesc_base()
 {
-    return (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((FMT == DS4G_MXFP4 ? 1u : 0u) << 23) |
+    return (1u << 7) | (1u << 10) | ((uint32_t)(TBN >> 3) << 17) | ((FMT == DS4G_MXFP4 ? 1u : 0u) << 23) |
            ((uint32_t)(BM >> 4) << 24);
 }
 
@@ -196,6 +203,21 @@ __device__ __forceinline__ void tc_commit(uint32_t mbar)
 {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(mbar)
                  : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v)
+{
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v)
@@ -272,8 +294,8 @@ __device__ __forceinline__ Tile tile_of(int64_t t, const int32_t* prefix, const 
     return r;
 }
 
-// first weight rows of the two 128-row halves of the W tile
-template <int EPI>
+// first weight rows of the two halves of the W tile
+template <int EPI, int TBN>
 __device__ __forceinline__ void w_rows(const Tile& tl, int N, int I, int64_t& y0, int64_t& y1)
 {
     const int64_t wbase = (int64_t)tl.e * N;
@@ -281,17 +303,20 @@ __device__ __forceinline__ void w_rows(const Tile& tl, int N, int I, int64_t& y0
         y0 = wbase + (int64_t)tl.nt * 128;          // gate rows
         y1 = wbase + I + (int64_t)tl.nt * 128;      // up rows
     } else {
-        y0 = wbase + (int64_t)tl.nt * BN;
-        y1 = y0 + 128;
+        y0 = wbase + (int64_t)tl.nt * TBN;
+        y1 = y0 + TBN / 2;
     }
 }
 
-template <int FMT, int EPI>
+template <int FMT, int EPI, int TBN>
 __global__ void __launch_bounds__(kThreads, 1)
 k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
           const __grid_constant__ CUtensorMap map_sfa, const __grid_constant__ CUtensorMap map_sfb, const GemmArgs p)
 {
-    using C = Cfg<FMT>;
+    using C = Cfg<FMT, TBN>;
+    static_assert(EPI != DS4G_EPI_SWIGLU_REQUANT || TBN == 256, "SwiGLU tiles pair 128 gate and 128 up rows");
+    constexpr int NACC = C::NACC;
+    constexpr int B_BYTES = C::B_BYTES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;
@@ -304,9 +329,9 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
     uint64_t* sf_full = empty + STAGES;                    // [SF_STAGES] TMA scales landed
     uint64_t* sf_ready = sf_full + SF_STAGES;              // [SF_STAGES] scales transposed
     uint64_t* sf_empty = sf_ready + SF_STAGES;             // [SF_STAGES] MMAs done with the scales
-    uint64_t* tmem_full = sf_empty + SF_STAGES;
-    uint64_t* tmem_empty = tmem_full + 1;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tmem_empty + 1);
+    uint64_t* tmem_full = sf_empty + SF_STAGES;            // [NACC] accumulator complete
+    uint64_t* tmem_empty = tmem_full + 2;                  // [NACC] accumulator drained
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tmem_empty + 2);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int32_t* total_tiles = reinterpret_cast<int32_t*>(tmem_slot + 2);
     int32_t* prefix = reinterpret_cast<int32_t*>(smem + C::DATA_BYTES + C::SF_BYTES + 256);
@@ -317,7 +342,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
     const int nks = (int)ceil_div(K, BK);
     const int npairs = (nks + 1) / 2;
     const int I = p.N / 2;
-    const int n_tiles = (EPI == DS4G_EPI_SWIGLU_REQUANT) ? (I / 128) : (p.N / BN);
+    const int n_tiles = (EPI == DS4G_EPI_SWIGLU_REQUANT) ? (I / 128) : (p.N / TBN);
 
     // ---- prologue
     if (threadIdx.x == 0) {
@@ -330,8 +355,10 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
             mbar_init(smem_u32(&sf_ready[r]), 1);
             mbar_init(smem_u32(&sf_empty[r]), 1);
         }
-        mbar_init(smem_u32(tmem_full), 1);
-        mbar_init(smem_u32(tmem_empty), 32 * kEpiWarps);
+        for (int b2 = 0; b2 < NACC; ++b2) {
+            mbar_init(smem_u32(&tmem_full[b2]), 1);
+            mbar_init(smem_u32(&tmem_empty[b2]), 32 * kEpiWarps);
+        }
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -393,17 +420,17 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
             for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
                 const Tile tl = tile_of(t, prefix, p.offsets, E, n_tiles);
                 int64_t y0, y1;
-                w_rows<EPI>(tl, p.N, I, y0, y1);
+                w_rows<EPI, TBN>(tl, p.N, I, y0, y1);
                 for (int ks = 0; ks < nks; ++ks, ++it) {
                     if ((ks & 1) == 0) {
                         const int r = sit % SF_STAGES;
                         if (!mbar_wait(smem_u32(&sf_empty[r]), ((sit / SF_STAGES) & 1) ^ 1, abort_flag)) { ok = false; break; }
                         const uint32_t fb = smem_u32(&sf_full[r]);
-                        mbar_arrive_tx(fb, C::SFA_BYTES + C::SFB_BYTES);
+                        mbar_arrive_tx(fb, C::SFA_BYTES + TBN * C::SF_ROW);
                         const int x = (ks >> 1) * C::SF_ROW;
                         tma_load_2d(smem_u32(sSFA + r * C::SFA_BYTES), &map_sfa, fb, x, (int)tl.m0);
                         tma_load_2d(smem_u32(sSFB + r * C::SFB_BYTES), &map_sfb, fb, x, (int)y0);
-                        tma_load_2d(smem_u32(sSFB + r * C::SFB_BYTES + C::SFB_BYTES / 2), &map_sfb, fb, x, (int)y1);
+                        tma_load_2d(smem_u32(sSFB + r * C::SFB_BYTES + C::HALF * C::SF_ROW), &map_sfb, fb, x, (int)y1);
                         ++sit;
                     }
                     const int s = it % STAGES;
@@ -428,11 +455,13 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
     } else if (warp == 1) {
         // ================= MMA issuer =================
         if (lane == 0) {
-            const uint32_t ibase = idesc_base<FMT>();
+            const uint32_t ibase = idesc_base<FMT, TBN>();
             uint32_t it = 0, sit = 0, tcount = 0;
             bool ok = true;
             for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++tcount) {
-                if (!mbar_wait(smem_u32(tmem_empty), (tcount & 1) ^ 1, abort_flag)) { ok = false; break; }
+                const int buf = (int)(tcount % NACC);
+                if (!mbar_wait(smem_u32(&tmem_empty[buf]), ((tcount / NACC) & 1) ^ 1, abort_flag)) { ok = false; break; }
+                const uint32_t acc = tmem + kColAcc + buf * TBN;
                 tc_fence_after();
                 for (int ks = 0; ks < nks; ++ks, ++it) {
                     const int r = sit % SF_STAGES;
@@ -448,9 +477,9 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
                     const uint32_t sfb_s = smem_u32(sSFB + r * C::SFB_BYTES);
 #pragma unroll
                     for (int c = 0; c < C::WPS; ++c) {
-                        utccp(tmem + kColSFA + 4 * c, desc_sf(sfa_s + (w0 + c) * 512));
-                        utccp(tmem + kColSFB + 8 * c, desc_sf(sfb_s + ((w0 + c) * 2 + 0) * 512));
-                        utccp(tmem + kColSFB + 8 * c + 4, desc_sf(sfb_s + ((w0 + c) * 2 + 1) * 512));
+                        utccp(tmem + C::COL_SFA + 4 * c, desc_sf(sfa_s + (w0 + c) * 512));
+                        utccp(tmem + C::COL_SFB + 8 * c, desc_sf(sfb_s + ((w0 + c) * 2 + 0) * 512));
+                        utccp(tmem + C::COL_SFB + 8 * c + 4, desc_sf(sfb_s + ((w0 + c) * 2 + 1) * 512));
                     }
                     const int64_t krem = K - (int64_t)ks * BK;
                     const int nmma = krem >= BK ? 4 : (int)(krem / 64);
@@ -462,8 +491,8 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
                             const int c = (FMT == DS4G_MXFP4) ? (j >> 1) : j;
                             const uint32_t sfid = (FMT == DS4G_MXFP4) ? (uint32_t)((j & 1) * 2) : 0u;
                             const uint32_t idesc = ibase | (sfid << 4) | (sfid << 29);
-                            mma<FMT>(tmem + kColAcc, desc_sw128(a_s + 32 * j), desc_sw128(b_s + 32 * j), idesc,
-                                     (ks > 0 || j > 0) ? 1u : 0u, tmem + kColSFA + 4 * c, tmem + kColSFB + 8 * c);
+                            mma<FMT>(acc, desc_sw128(a_s + 32 * j), desc_sw128(b_s + 32 * j), idesc,
+                                     (ks > 0 || j > 0) ? 1u : 0u, tmem + C::COL_SFA + 4 * c, tmem + C::COL_SFB + 8 * c);
                         }
                     }
                     tc_commit(smem_u32(&empty[s]));
@@ -473,7 +502,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
                     }
                 }
                 if (!ok) break;
-                tc_commit(smem_u32(tmem_full));
+                tc_commit(smem_u32(&tmem_full[buf]));
             }
         }
         __syncwarp();
@@ -502,13 +531,14 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
         uint32_t tcount = 0;
         const float gh = (FMT == DS4G_NVFP4 && EPI == DS4G_EPI_SWIGLU_REQUANT) ? *p.oq_g : 1.0f;
         for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, ++tcount) {
-            if (!mbar_wait(smem_u32(tmem_full), tcount & 1, abort_flag)) break;
+            const int buf = (int)(tcount % NACC);
+            if (!mbar_wait(smem_u32(&tmem_full[buf]), (tcount / NACC) & 1, abort_flag)) break;
             tc_fence_after();
             const Tile tl = tile_of(t, prefix, p.offsets, E, n_tiles);
             const float gscale = (FMT == DS4G_NVFP4) ? __fmul_rn(p.a_g[0], p.w_g[tl.e]) : 1.0f;
             const int64_t row = tl.m0 + 32 * q + lane;
             const bool valid = row < tl.end;
-            const uint32_t tbase = tmem + kColAcc + ((uint32_t)(32 * q) << 16);
+            const uint32_t tbase = tmem + kColAcc + buf * TBN + ((uint32_t)(32 * q) << 16);
             if (EPI != DS4G_EPI_SWIGLU_REQUANT) {
                 // plain: store the row; combine: add w * row into its token's output
                 float* dst_row = p.out + row * p.N;
@@ -518,15 +548,33 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
                     dst_row = p.out + (int64_t)(s / p.topk) * p.N;
                     wr = p.route_w[s] * gscale;
                 }
+                // this warp's half of the columns: 32-column pieces (and a
+                // 16-column one when the half is 112 wide)
 #pragma unroll 1
-                for (int c8 = 0; c8 < 4; ++c8) {
-                    const int col = half * 128 + 32 * c8;
+                for (int c8 = 0; c8 < C::HALF / 32; ++c8) {
+                    const int col = half * C::HALF + 32 * c8;
                     float v[32];
                     tmem_ld32(tbase + col, v);
                     if (valid) {
-                        float* dst = dst_row + (int64_t)tl.nt * BN + col;
+                        float* dst = dst_row + (int64_t)tl.nt * TBN + col;
 #pragma unroll
                         for (int i = 0; i < 8; ++i) {
+                            if (EPI == kEpiCombine)
+                                red_add_v4(dst + 4 * i, v[4 * i] * wr, v[4 * i + 1] * wr, v[4 * i + 2] * wr, v[4 * i + 3] * wr);
+                            else
+                                reinterpret_cast<float4*>(dst)[i] =
+                                    make_float4(v[4 * i] * wr, v[4 * i + 1] * wr, v[4 * i + 2] * wr, v[4 * i + 3] * wr);
+                        }
+                    }
+                }
+                if (C::HALF % 32 != 0) {
+                    const int col = half * C::HALF + 32 * (C::HALF / 32);
+                    float v[16];
+                    tmem_ld16(tbase + col, v);
+                    if (valid) {
+                        float* dst = dst_row + (int64_t)tl.nt * TBN + col;
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
                             if (EPI == kEpiCombine)
                                 red_add_v4(dst + 4 * i, v[4 * i] * wr, v[4 * i + 1] * wr, v[4 * i + 2] * wr, v[4 * i + 3] * wr);
                             else
@@ -597,7 +645,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
                 }
             }
             tc_fence_before();
-            mbar_arrive(smem_u32(tmem_empty));
+            mbar_arrive(smem_u32(&tmem_empty[buf]));
         }
     }
 
@@ -646,18 +694,18 @@ static bool make_map(CUtensorMap* m, const uint8_t* base, int64_t rows, int64_t 
     return r == CUDA_SUCCESS;
 }
 
-template <int FMT, int EPI>
+template <int FMT, int EPI, int TBN>
 static cudaError_t run_tc(const GemmArgs& a, cudaStream_t st)
 {
-    using C = tc::Cfg<FMT>;
+    using C = tc::Cfg<FMT, TBN>;
     const int blk = (FMT == DS4G_MXFP4) ? 32 : 16;
     CUtensorMap ma, mb, msa, msb;
     if (!make_map(&ma, a.a_data, a.S, a.K / 2, 128, 128, true) ||
-        !make_map(&mb, a.w_data, (int64_t)a.E * a.N, a.K / 2, 128, 128, true) ||
+        !make_map(&mb, a.w_data, (int64_t)a.E * a.N, a.K / 2, 128, C::HALF, true) ||
         !make_map(&msa, a.a_scales, a.S, a.K / blk, C::SF_ROW, 128, false) ||
-        !make_map(&msb, a.w_scales, (int64_t)a.E * a.N, a.K / blk, C::SF_ROW, 128, false))
+        !make_map(&msb, a.w_scales, (int64_t)a.E * a.N, a.K / blk, C::SF_ROW, C::HALF, false))
         return cudaErrorInvalidValue;
-    auto kern = tc::k_gemm_tc<FMT, EPI>;
+    auto kern = tc::k_gemm_tc<FMT, EPI, TBN>;
     const size_t shm = C::SMEM;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)shm);
     if (e != cudaSuccess) return e;
@@ -665,6 +713,14 @@ static cudaError_t run_tc(const GemmArgs& a, cudaStream_t st)
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     kern<<<sms, tc::kThreads, shm, st>>>(ma, mb, msa, msb, a);
     return cudaGetLastError();
+}
+
+// plain and combine epilogues: 224-column tiles with two accumulators when N
+// allows, else 256-column tiles
+template <int FMT, int EPI>
+static cudaError_t run_tc_plain(const GemmArgs& a, cudaStream_t st)
+{
+    return (a.N % 224 == 0) ? run_tc<FMT, EPI, 224>(a, st) : run_tc<FMT, EPI, 256>(a, st);
 }
 
 bool gemm_tc_supports(int fmt, int64_t K)
@@ -679,12 +735,12 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st)
     if (a.S == 0) return cudaSuccess;
     if (a.E > tc::kMaxE || !gemm_tc_supports(a.fmt, a.K)) return cudaErrorInvalidValue;
     if (a.fmt == DS4G_MXFP4)
-        return a.epilogue == DS4G_EPI_NONE ? run_tc<DS4G_MXFP4, DS4G_EPI_NONE>(a, st)
-             : a.epilogue == kEpiCombine   ? run_tc<DS4G_MXFP4, kEpiCombine>(a, st)
-                                           : run_tc<DS4G_MXFP4, DS4G_EPI_SWIGLU_REQUANT>(a, st);
-    return a.epilogue == DS4G_EPI_NONE ? run_tc<DS4G_NVFP4, DS4G_EPI_NONE>(a, st)
-         : a.epilogue == kEpiCombine   ? run_tc<DS4G_NVFP4, kEpiCombine>(a, st)
-                                       : run_tc<DS4G_NVFP4, DS4G_EPI_SWIGLU_REQUANT>(a, st);
+        return a.epilogue == DS4G_EPI_NONE ? run_tc_plain<DS4G_MXFP4, DS4G_EPI_NONE>(a, st)
+             : a.epilogue == kEpiCombine   ? run_tc_plain<DS4G_MXFP4, kEpiCombine>(a, st)
+                                           : run_tc<DS4G_MXFP4, DS4G_EPI_SWIGLU_REQUANT, 256>(a, st);
+    return a.epilogue == DS4G_EPI_NONE ? run_tc_plain<DS4G_NVFP4, DS4G_EPI_NONE>(a, st)
+         : a.epilogue == kEpiCombine   ? run_tc_plain<DS4G_NVFP4, kEpiCombine>(a, st)
+                                       : run_tc<DS4G_NVFP4, DS4G_EPI_SWIGLU_REQUANT, 256>(a, st);
 }
 
 }  // namespace ds4g

@@ -155,11 +155,14 @@ ds4g_status ds4g_moe_permute(const int32_t* idx, int T, int k, int E, const ds4g
  *   <= 16 rows, K a multiple of 512 (MXFP4) / 256 (NVFP4), N % 128 == 0
  *     (NONE) or I % 64 == 0 (SWIGLU_REQUANT): tensor-core kernel with the
  *     weights as the MMA's M side (decode);
- *   > 16 rows and the same K rule, N % 256 == 0 (NONE) or I % 128 == 0
- *     (SWIGLU_REQUANT): tensor-core kernel with 128-row x 256-column tiles;
+ *   > 16 rows and the same K rule, N % 224 == 0 (NONE): tensor-core kernel
+ *     with 128-row x 224-column tiles and two accumulators (the epilogue of
+ *     one tile overlaps the next tile's MMAs); else N % 256 == 0 (NONE) or
+ *     I % 128 == 0 (SWIGLU_REQUANT): 128-row x 256-column tiles;
  *   otherwise: a dp4a weight-streaming kernel (any segment length).
- * Shapes: K % 64 == 0; NONE needs N % 64 == 0; SWIGLU_REQUANT needs
- *   I % 32 == 0.  offsets[E] must equal S. */
+ * Shapes: K % 64 == 0; NONE needs N % 64 == 0 unless a tensor-core kernel
+ *   takes the call; SWIGLU_REQUANT needs I % 32 == 0.  offsets[E] must
+ *   equal S. */
 ds4g_status ds4g_grouped_gemm_fp4(const ds4g_fp4* a, const int32_t* offsets, int E,
                                   int max_rows_per_expert, const ds4g_fp4* w, int N, int epilogue,
                                   float* out, ds4g_fp4* out_q, float* h_debug, void* stream);

@@ -176,7 +176,9 @@ GEMV_CASES = [([3, 0, 1, 8, 5], 512, 7168), ([1, 1, 1, 1, 1, 1], 256, 2048), ([2
 # tensor-core kernel cases (MX needs K % 512, NV K % 256; others take the
 # GEMV kernel with long segments, which is covered as well)
 TC_CASES = [([300, 0, 1, 129, 77], 512, 512), ([256, 128], 256, 1024), ([9, 200, 0, 0, 1000], 256, 512),
-            ([130], 512, 7168), ([17, 140], 256, 768), ([40, 12], 256, 384)]
+            ([130], 512, 7168), ([17, 140], 256, 768), ([40, 12], 256, 384),
+            # N a multiple of 224: 224-column tiles, two accumulators
+            ([300, 0, 1, 129, 77], 448, 512), ([130, 20], 224, 2048), ([17, 600], 672, 1024)]
 
 
 @pytest.mark.parametrize("fmt", [MX, NV])
@@ -185,8 +187,6 @@ def test_grouped_gemm_plain(fmt, case):
     seg, N, K = case
     offsets, a, w, gw = _grouped_problem(seg, N, K, fmt)
     max_rows = max(seg)
-    if max_rows > 8 and N % 256:
-        pytest.skip("tensor-core path needs N % 256 == 0")
     out = ds4g.ds4g_grouped_gemm_fp4(to_dev(a), torch.from_numpy(offsets).to(dev()), len(seg), max_rows,
                                      to_dev(w, g_per_expert=gw), N)
     ds4g.ds4g_check_device()
@@ -250,6 +250,7 @@ def test_swiglu_requant(fmt):
 
 @pytest.mark.parametrize("fmt", [MX, NV])
 @pytest.mark.parametrize("T,k,E,N,K", [(300, 6, 16, 512, 1024),    # tensor-core kernel
+                                       (300, 6, 16, 448, 1024),    # tensor-core kernel, 224-column tiles
                                        (3, 6, 64, 256, 1024),      # decode tensor-core kernel
                                        (4, 2, 8, 128, 256)])       # dp4a kernel (MX) / decode tc (NV)
 def test_fc2_combine_fused(fmt, T, k, E, N, K):
