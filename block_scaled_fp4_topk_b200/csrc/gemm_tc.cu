@@ -42,7 +42,6 @@ constexpr int BM = 128;            // tile rows (tokens)
 constexpr int BKB = 128;           // bytes of K per stage per row (256 FP4)
 constexpr int BK = 256;            // K elements per stage
 constexpr int STAGES = 4;
-constexpr int SF_STAGES = 2;       // scale stages, each covering two K stages (512 K)
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = 32 * (4 + kEpiWarps);
 constexpr int A_BYTES = BM * BKB;  // 16 KB
@@ -55,22 +54,37 @@ constexpr unsigned long long kWaitNs = 4000000000ull;
 // multiple of 224, e.g. FC2 with N = 7168) with two, so that the epilogue of
 // one tile overlaps the MMAs of the next: 2 x 224 accumulator columns plus
 // the scale columns fit the 512 TMEM columns, 2 x 256 do not.
-template <int FMT, int TBN>
+template <int FMT, int TBN, int NISS>
 struct Cfg {
     static_assert(TBN == 256 || TBN == 224, "tile width");
+    static_assert(NISS == 1 || (NISS == 2 && TBN == 224), "two issuers need two accumulators");
     static constexpr int NACC = (TBN == 256) ? 1 : 2;               // accumulator buffers
     static constexpr int HALF = TBN / 2;                             // weight rows per TMA box
     static constexpr int B_BYTES = TBN * BKB;
-    static constexpr int COL_SFA = NACC * TBN;                       // TMEM columns of the scales
-    static constexpr int COL_SFB = COL_SFA + 16;
     static constexpr int WPS = (FMT == DS4G_MXFP4) ? 2 : 4;         // 4-scale words per row per K stage
+    // TMEM scale columns per issuer: A (4 per word) then W (8 per word)
+    static constexpr int SF_COLS = 12 * WPS;
+    // scale stages, each covering two K stages (512 K): two per issuer
+    static constexpr int SF_STAGES = 2 * NISS;
+    static constexpr int COL_SFA = NACC * TBN;
+    static_assert(COL_SFA + NISS * SF_COLS <= 512, "TMEM columns");
     static constexpr int SF_ROW = 2 * WPS * 4;                       // scale bytes per row per scale stage
     static constexpr int SFA_BYTES = BM * SF_ROW;                    // one scale stage of A
     static constexpr int SFB_BYTES = 256 * SF_ROW;                   // one scale stage of W (two 128-row groups)
-    static_assert(COL_SFB + 8 * WPS <= kTmemCols, "TMEM columns");
     static constexpr int DATA_BYTES = STAGES * (A_BYTES + B_BYTES);
     static constexpr int SF_BYTES = SF_STAGES * (SFA_BYTES + SFB_BYTES);
-    static constexpr size_t SMEM = 1024 + (size_t)DATA_BYTES + SF_BYTES + 256 + (kMaxE + 1) * 4;
+    // 224-column tiles with one MMA issuer stage their fp32 epilogue through
+    // shared memory, 16 rows x 32 columns per warp (rows padded to 33
+    // floats), so that each store / reduction instruction covers 4 rows x 128
+    // contiguous bytes.  With two issuers the mainloop is already bound by
+    // shared-memory bandwidth and the staging traffic slows it more than the
+    // wider reductions gain (measured: FC2 0.389 -> 0.448 ms at T = 2048), so
+    // that configuration stores straight from registers.
+    static constexpr bool STAGED = (TBN == 224 && NISS == 1);
+    static constexpr int STAGE_OFF = DATA_BYTES + SF_BYTES + 256 + ((kMaxE + 1) * 4 + 15) / 16 * 16;
+    static constexpr int STAGE_BYTES = STAGED ? kEpiWarps * 16 * 33 * 4 : 0;
+    static constexpr size_t SMEM = 1024 + (size_t)STAGE_OFF + STAGE_BYTES;
+    static_assert(SMEM <= 232448, "shared memory per CTA");
 };
 
 // ---- PTX wrappers ----------------------------------------------------------
@@ -308,12 +322,13 @@ __device__ __forceinline__ void w_rows(const Tile& tl, int N, int I, int64_t& y0
     }
 }
 
-template <int FMT, int EPI, int TBN>
+template <int FMT, int EPI, int TBN, int NISS>
 __global__ void __launch_bounds__(kThreads, 1)
 k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
           const __grid_constant__ CUtensorMap map_sfa, const __grid_constant__ CUtensorMap map_sfb, const GemmArgs p)
 {
-    using C = Cfg<FMT, TBN>;
+    using C = Cfg<FMT, TBN, NISS>;
+    constexpr int SF_STAGES = C::SF_STAGES;
     static_assert(EPI != DS4G_EPI_SWIGLU_REQUANT || TBN == 256, "SwiGLU tiles pair 128 gate and 128 up rows");
     constexpr int NACC = C::NACC;
     constexpr int B_BYTES = C::B_BYTES;
@@ -414,32 +429,50 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
 
     if (warp == 0) {
         // ================= TMA producer =================
+        // This CTA's tiles in groups of NISS consecutive ones; the stages of a
+        // group are interleaved (K stage by K stage, member by member) so that
+        // each MMA issuer finds its next stage while the other works.
         if (lane == 0) {
             uint32_t it = 0, sit = 0;
             bool ok = true;
-            for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-                const Tile tl = tile_of(t, prefix, p.offsets, E, n_tiles);
-                int64_t y0, y1;
-                w_rows<EPI, TBN>(tl, p.N, I, y0, y1);
-                for (int ks = 0; ks < nks; ++ks, ++it) {
-                    if ((ks & 1) == 0) {
-                        const int r = sit % SF_STAGES;
-                        if (!mbar_wait(smem_u32(&sf_empty[r]), ((sit / SF_STAGES) & 1) ^ 1, abort_flag)) { ok = false; break; }
-                        const uint32_t fb = smem_u32(&sf_full[r]);
-                        mbar_arrive_tx(fb, C::SFA_BYTES + TBN * C::SF_ROW);
-                        const int x = (ks >> 1) * C::SF_ROW;
-                        tma_load_2d(smem_u32(sSFA + r * C::SFA_BYTES), &map_sfa, fb, x, (int)tl.m0);
-                        tma_load_2d(smem_u32(sSFB + r * C::SFB_BYTES), &map_sfb, fb, x, (int)y0);
-                        tma_load_2d(smem_u32(sSFB + r * C::SFB_BYTES + C::HALF * C::SF_ROW), &map_sfb, fb, x, (int)y1);
-                        ++sit;
+            for (int64_t j0 = 0; ok; j0 += NISS) {
+                const int64_t t0 = blockIdx.x + j0 * gridDim.x;
+                if (t0 >= ntiles) break;
+                const int gsz = (NISS == 2 && t0 + gridDim.x < ntiles) ? 2 : 1;
+                Tile tls[NISS];
+                int64_t y0s[NISS], y1s[NISS];
+#pragma unroll
+                for (int u = 0; u < NISS; ++u) {
+                    if (u < gsz) {
+                        tls[u] = tile_of(t0 + u * (int64_t)gridDim.x, prefix, p.offsets, E, n_tiles);
+                        w_rows<EPI, TBN>(tls[u], p.N, I, y0s[u], y1s[u]);
                     }
-                    const int s = it % STAGES;
-                    if (!mbar_wait(smem_u32(&empty[s]), ((it / STAGES) & 1) ^ 1, abort_flag)) { ok = false; break; }
-                    const uint32_t fb = smem_u32(&full[s]);
-                    mbar_arrive_tx(fb, A_BYTES + B_BYTES);
-                    tma_load_2d(smem_u32(sA + s * A_BYTES), &map_a, fb, ks * BKB, (int)tl.m0);
-                    tma_load_2d(smem_u32(sB + s * B_BYTES), &map_b, fb, ks * BKB, (int)y0);
-                    tma_load_2d(smem_u32(sB + s * B_BYTES + B_BYTES / 2), &map_b, fb, ks * BKB, (int)y1);
+                }
+                for (int ks = 0; ks < nks && ok; ++ks) {
+#pragma unroll
+                    for (int u = 0; u < NISS; ++u) {
+                        if (u >= gsz || !ok) continue;
+                        const Tile& tl = tls[u];
+                        if ((ks & 1) == 0) {
+                            const int r = sit % SF_STAGES;
+                            if (!mbar_wait(smem_u32(&sf_empty[r]), ((sit / SF_STAGES) & 1) ^ 1, abort_flag)) { ok = false; break; }
+                            const uint32_t fb = smem_u32(&sf_full[r]);
+                            mbar_arrive_tx(fb, C::SFA_BYTES + TBN * C::SF_ROW);
+                            const int x = (ks >> 1) * C::SF_ROW;
+                            tma_load_2d(smem_u32(sSFA + r * C::SFA_BYTES), &map_sfa, fb, x, (int)tl.m0);
+                            tma_load_2d(smem_u32(sSFB + r * C::SFB_BYTES), &map_sfb, fb, x, (int)y0s[u]);
+                            tma_load_2d(smem_u32(sSFB + r * C::SFB_BYTES + C::HALF * C::SF_ROW), &map_sfb, fb, x, (int)y1s[u]);
+                            ++sit;
+                        }
+                        const int s = it % STAGES;
+                        if (!mbar_wait(smem_u32(&empty[s]), ((it / STAGES) & 1) ^ 1, abort_flag)) { ok = false; break; }
+                        const uint32_t fb = smem_u32(&full[s]);
+                        mbar_arrive_tx(fb, A_BYTES + B_BYTES);
+                        tma_load_2d(smem_u32(sA + s * A_BYTES), &map_a, fb, ks * BKB, (int)tl.m0);
+                        tma_load_2d(smem_u32(sB + s * B_BYTES), &map_b, fb, ks * BKB, (int)y0s[u]);
+                        tma_load_2d(smem_u32(sB + s * B_BYTES + B_BYTES / 2), &map_b, fb, ks * BKB, (int)y1s[u]);
+                        ++it;
+                    }
                 }
             }
             if (!ok) {
@@ -452,57 +485,72 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
             }
         }
         __syncwarp();
-    } else if (warp == 1) {
-        // ================= MMA issuer =================
+    } else if (warp == 1 || (NISS == 2 && warp == 3)) {
+        // ================= MMA issuer(s) =================
+        // Issuer pi takes member pi of each tile group, accumulating into
+        // accumulator pi (two issuers) with its own scale columns.  An issuing
+        // thread that waits on a barrier first drains its own tensor-core
+        // work; with two issuers the other one's MMAs fill that gap.
         if (lane == 0) {
+            const int pi = (warp == 1) ? 0 : 1;
             const uint32_t ibase = idesc_base<FMT, TBN>();
-            uint32_t it = 0, sit = 0, tcount = 0;
+            const uint32_t col_sfa = tmem + C::COL_SFA + pi * C::SF_COLS;
+            const uint32_t col_sfb = col_sfa + 4 * C::WPS;
+            uint32_t it_base = 0, sit_base = 0;
             bool ok = true;
-            for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++tcount) {
-                const int buf = (int)(tcount % NACC);
-                if (!mbar_wait(smem_u32(&tmem_empty[buf]), ((tcount / NACC) & 1) ^ 1, abort_flag)) { ok = false; break; }
-                const uint32_t acc = tmem + kColAcc + buf * TBN;
-                tc_fence_after();
-                for (int ks = 0; ks < nks; ++ks, ++it) {
-                    const int r = sit % SF_STAGES;
-                    if ((ks & 1) == 0) {
-                        if (!mbar_wait(smem_u32(&sf_ready[r]), (sit / SF_STAGES) & 1, abort_flag)) { ok = false; break; }
-                    }
-                    const int s = it % STAGES;
-                    if (!mbar_wait(smem_u32(&full[s]), (it / STAGES) & 1, abort_flag)) { ok = false; break; }
+            for (int64_t j0 = 0; ok; j0 += NISS) {
+                const int64_t t0 = blockIdx.x + j0 * gridDim.x;
+                if (t0 >= ntiles) break;
+                const int gsz = (NISS == 2 && t0 + gridDim.x < ntiles) ? 2 : 1;
+                if (pi < gsz) {
+                    const int64_t jt = j0 + pi;                        // this CTA's local tile index
+                    const int buf = (NISS == 2) ? pi : (int)(jt % NACC);
+                    const uint32_t use = (NISS == 2) ? (uint32_t)(j0 / 2) : (uint32_t)(jt / NACC);
+                    if (!mbar_wait(smem_u32(&tmem_empty[buf]), (use & 1) ^ 1, abort_flag)) { ok = false; break; }
+                    const uint32_t acc = tmem + kColAcc + buf * TBN;
                     tc_fence_after();
-                    // this K stage's scale words -> TMEM
-                    const int w0 = (ks & 1) * C::WPS;
-                    const uint32_t sfa_s = smem_u32(sSFA + r * C::SFA_BYTES);
-                    const uint32_t sfb_s = smem_u32(sSFB + r * C::SFB_BYTES);
-#pragma unroll
-                    for (int c = 0; c < C::WPS; ++c) {
-                        utccp(tmem + C::COL_SFA + 4 * c, desc_sf(sfa_s + (w0 + c) * 512));
-                        utccp(tmem + C::COL_SFB + 8 * c, desc_sf(sfb_s + ((w0 + c) * 2 + 0) * 512));
-                        utccp(tmem + C::COL_SFB + 8 * c + 4, desc_sf(sfb_s + ((w0 + c) * 2 + 1) * 512));
-                    }
-                    const int64_t krem = K - (int64_t)ks * BK;
-                    const int nmma = krem >= BK ? 4 : (int)(krem / 64);
-                    const uint32_t a_s = smem_u32(sA + s * A_BYTES);
-                    const uint32_t b_s = smem_u32(sB + s * B_BYTES);
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        if (j < nmma) {
-                            const int c = (FMT == DS4G_MXFP4) ? (j >> 1) : j;
-                            const uint32_t sfid = (FMT == DS4G_MXFP4) ? (uint32_t)((j & 1) * 2) : 0u;
-                            const uint32_t idesc = ibase | (sfid << 4) | (sfid << 29);
-                            mma<FMT>(acc, desc_sw128(a_s + 32 * j), desc_sw128(b_s + 32 * j), idesc,
-                                     (ks > 0 || j > 0) ? 1u : 0u, tmem + C::COL_SFA + 4 * c, tmem + C::COL_SFB + 8 * c);
+                    for (int ks = 0; ks < nks; ++ks) {
+                        const uint32_t it = it_base + (uint32_t)(ks * gsz + pi);
+                        const uint32_t sit = sit_base + (uint32_t)((ks >> 1) * gsz + pi);
+                        const int r = sit % SF_STAGES;
+                        if ((ks & 1) == 0) {
+                            if (!mbar_wait(smem_u32(&sf_ready[r]), (sit / SF_STAGES) & 1, abort_flag)) { ok = false; break; }
                         }
+                        const int s = it % STAGES;
+                        if (!mbar_wait(smem_u32(&full[s]), (it / STAGES) & 1, abort_flag)) { ok = false; break; }
+                        tc_fence_after();
+                        // this K stage's scale words -> TMEM
+                        const int w0 = (ks & 1) * C::WPS;
+                        const uint32_t sfa_s = smem_u32(sSFA + r * C::SFA_BYTES);
+                        const uint32_t sfb_s = smem_u32(sSFB + r * C::SFB_BYTES);
+#pragma unroll
+                        for (int c = 0; c < C::WPS; ++c) {
+                            utccp(col_sfa + 4 * c, desc_sf(sfa_s + (w0 + c) * 512));
+                            utccp(col_sfb + 8 * c, desc_sf(sfb_s + ((w0 + c) * 2 + 0) * 512));
+                            utccp(col_sfb + 8 * c + 4, desc_sf(sfb_s + ((w0 + c) * 2 + 1) * 512));
+                        }
+                        const int64_t krem = K - (int64_t)ks * BK;
+                        const int nmma = krem >= BK ? 4 : (int)(krem / 64);
+                        const uint32_t a_s = smem_u32(sA + s * A_BYTES);
+                        const uint32_t b_s = smem_u32(sB + s * B_BYTES);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            if (j < nmma) {
+                                const int c = (FMT == DS4G_MXFP4) ? (j >> 1) : j;
+                                const uint32_t sfid = (FMT == DS4G_MXFP4) ? (uint32_t)((j & 1) * 2) : 0u;
+                                const uint32_t idesc = ibase | (sfid << 4) | (sfid << 29);
+                                mma<FMT>(acc, desc_sw128(a_s + 32 * j), desc_sw128(b_s + 32 * j), idesc,
+                                         (ks > 0 || j > 0) ? 1u : 0u, col_sfa + 4 * c, col_sfb + 8 * c);
+                            }
+                        }
+                        tc_commit(smem_u32(&empty[s]));
+                        if ((ks & 1) == 1 || ks == nks - 1) tc_commit(smem_u32(&sf_empty[r]));
                     }
-                    tc_commit(smem_u32(&empty[s]));
-                    if ((ks & 1) == 1 || ks == nks - 1) {
-                        tc_commit(smem_u32(&sf_empty[r]));
-                        ++sit;
-                    }
+                    if (!ok) break;
+                    tc_commit(smem_u32(&tmem_full[buf]));
                 }
-                if (!ok) break;
-                tc_commit(smem_u32(&tmem_full[buf]));
+                it_base += (uint32_t)(nks * gsz);
+                sit_base += (uint32_t)(npairs * gsz);
             }
         }
         __syncwarp();
@@ -548,8 +596,47 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
                     dst_row = p.out + (int64_t)(s / p.topk) * p.N;
                     wr = p.route_w[s] * gscale;
                 }
-                // this warp's half of the columns: 32-column pieces (and a
-                // 16-column one when the half is 112 wide)
+                if (C::STAGED) {
+                    // 32-column pieces of this warp's half (the last one 16 wide),
+                    // each as two 16-row blocks through the warp's staging area
+                    float* stg = reinterpret_cast<float*>(smem + C::STAGE_OFF) + (warp - 4) * (16 * 33);
+                    const unsigned long long my_dst =
+                        valid ? reinterpret_cast<unsigned long long>(dst_row + (int64_t)tl.nt * TBN) : 0ull;
+#pragma unroll 1
+                    for (int c8 = 0; c8 < (C::HALF + 31) / 32; ++c8) {
+                        const int col = half * C::HALF + 32 * c8;
+                        const int ncol = min(32, C::HALF - 32 * c8);
+                        float v[32];
+                        if (ncol == 32) tmem_ld32(tbase + col, v);
+                        else tmem_ld16(tbase + col, v);
+#pragma unroll 1
+                        for (int hh = 0; hh < 2; ++hh) {
+                            if ((lane >> 4) == hh) {
+                                float* srow = stg + (lane & 15) * 33;
+#pragma unroll
+                                for (int i = 0; i < 32; ++i)
+                                    if (i < ncol) srow[i] = v[i] * wr;
+                            }
+                            __syncwarp();
+#pragma unroll
+                            for (int i4 = 0; i4 < 4; ++i4) {
+                                const int rl = 4 * i4 + (lane >> 3);       // staged row
+                                const unsigned long long d = __shfl_sync(0xffffffffu, my_dst, 16 * hh + rl);
+                                const int cc = (lane & 7) * 4;
+                                if (d != 0ull && cc < ncol) {
+                                    const float* sr = stg + rl * 33 + cc;
+                                    float* g = reinterpret_cast<float*>(d) + col + cc;
+                                    if (EPI == kEpiCombine)
+                                        red_add_v4(g, sr[0], sr[1], sr[2], sr[3]);
+                                    else
+                                        *reinterpret_cast<float4*>(g) = make_float4(sr[0], sr[1], sr[2], sr[3]);
+                                }
+                            }
+                            __syncwarp();
+                        }
+                    }
+                } else {
+                // this warp's half of the columns, 32-column pieces
 #pragma unroll 1
                 for (int c8 = 0; c8 < C::HALF / 32; ++c8) {
                     const int col = half * C::HALF + 32 * c8;
@@ -567,7 +654,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
                         }
                     }
                 }
-                if (C::HALF % 32 != 0) {
+                if (C::HALF % 32 != 0) {                    // the last 16 columns of a 112-wide half
                     const int col = half * C::HALF + 32 * (C::HALF / 32);
                     float v[16];
                     tmem_ld16(tbase + col, v);
@@ -582,6 +669,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
                                     make_float4(v[4 * i] * wr, v[4 * i + 1] * wr, v[4 * i + 2] * wr, v[4 * i + 3] * wr);
                         }
                     }
+                }
                 }
             } else {
 #pragma unroll 1
@@ -694,10 +782,10 @@ static bool make_map(CUtensorMap* m, const uint8_t* base, int64_t rows, int64_t 
     return r == CUDA_SUCCESS;
 }
 
-template <int FMT, int EPI, int TBN>
+template <int FMT, int EPI, int TBN, int NISS>
 static cudaError_t run_tc(const GemmArgs& a, cudaStream_t st)
 {
-    using C = tc::Cfg<FMT, TBN>;
+    using C = tc::Cfg<FMT, TBN, NISS>;
     const int blk = (FMT == DS4G_MXFP4) ? 32 : 16;
     CUtensorMap ma, mb, msa, msb;
     if (!make_map(&ma, a.a_data, a.S, a.K / 2, 128, 128, true) ||
@@ -705,7 +793,7 @@ static cudaError_t run_tc(const GemmArgs& a, cudaStream_t st)
         !make_map(&msa, a.a_scales, a.S, a.K / blk, C::SF_ROW, 128, false) ||
         !make_map(&msb, a.w_scales, (int64_t)a.E * a.N, a.K / blk, C::SF_ROW, C::HALF, false))
         return cudaErrorInvalidValue;
-    auto kern = tc::k_gemm_tc<FMT, EPI, TBN>;
+    auto kern = tc::k_gemm_tc<FMT, EPI, TBN, NISS>;
     const size_t shm = C::SMEM;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)shm);
     if (e != cudaSuccess) return e;
@@ -716,11 +804,13 @@ static cudaError_t run_tc(const GemmArgs& a, cudaStream_t st)
 }
 
 // plain and combine epilogues: 224-column tiles with two accumulators when N
-// allows, else 256-column tiles
+// allows (and, for MXFP4, whose scale columns fit beside them, two MMA
+// issuers), else 256-column tiles
 template <int FMT, int EPI>
 static cudaError_t run_tc_plain(const GemmArgs& a, cudaStream_t st)
 {
-    return (a.N % 224 == 0) ? run_tc<FMT, EPI, 224>(a, st) : run_tc<FMT, EPI, 256>(a, st);
+    constexpr int kIss224 = (FMT == DS4G_MXFP4) ? 2 : 1;
+    return (a.N % 224 == 0) ? run_tc<FMT, EPI, 224, kIss224>(a, st) : run_tc<FMT, EPI, 256, 1>(a, st);
 }
 
 bool gemm_tc_supports(int fmt, int64_t K)
@@ -737,10 +827,10 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st)
     if (a.fmt == DS4G_MXFP4)
         return a.epilogue == DS4G_EPI_NONE ? run_tc_plain<DS4G_MXFP4, DS4G_EPI_NONE>(a, st)
              : a.epilogue == kEpiCombine   ? run_tc_plain<DS4G_MXFP4, kEpiCombine>(a, st)
-                                           : run_tc<DS4G_MXFP4, DS4G_EPI_SWIGLU_REQUANT, 256>(a, st);
+                                           : run_tc<DS4G_MXFP4, DS4G_EPI_SWIGLU_REQUANT, 256, 1>(a, st);
     return a.epilogue == DS4G_EPI_NONE ? run_tc_plain<DS4G_NVFP4, DS4G_EPI_NONE>(a, st)
          : a.epilogue == kEpiCombine   ? run_tc_plain<DS4G_NVFP4, kEpiCombine>(a, st)
-                                       : run_tc<DS4G_NVFP4, DS4G_EPI_SWIGLU_REQUANT, 256>(a, st);
+                                       : run_tc<DS4G_NVFP4, DS4G_EPI_SWIGLU_REQUANT, 256, 1>(a, st);
 }
 
 }  // namespace ds4g
