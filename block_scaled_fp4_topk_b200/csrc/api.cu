@@ -117,6 +117,47 @@ ds4g_status ds4g_moe_permute(const int32_t* idx, int T, int k, int E, const ds4g
                                       S(stream)));
 }
 
+size_t ds4g_dispatch_workspace_bytes(int T, int k, int E, int fmt, int has_g_in)
+{
+    if (T < 0 || k < 1 || E < 1) return 0;
+    return dispatch_workspace_bytes(T, k, E, fmt, has_g_in);
+}
+
+ds4g_status ds4g_moe_dispatch(const float* logits, const void* x, int dtype, int T, int E, int k, int fmt,
+                              const float* g_in, int32_t* idx, float* w, ds4g_fp4* x_q, int32_t* offsets,
+                              int32_t* row_to_slot, int32_t* slot_to_row, ds4g_fp4* a_perm, void* workspace,
+                              size_t ws_bytes, void* stream)
+{
+    if (fmt != DS4G_MXFP4 && fmt != DS4G_NVFP4) return DS4G_ERR_INVALID_ARG;
+    if (dtype != DS4G_BF16 && dtype != DS4G_F32) return DS4G_ERR_INVALID_ARG;
+    if (T < 0 || E < 1 || E > 1024 || k < 1 || k > E || k > 32) return DS4G_ERR_INVALID_ARG;
+    if (!x_q || !a_perm || !offsets) return DS4G_ERR_INVALID_ARG;
+    const int64_t S_ = (int64_t)T * k;
+    if (S_ > 0x7FFFFFFF) return DS4G_ERR_SHAPE;
+    const int64_t K = x_q->K;
+    if (K <= 0 || K % 64 != 0) return DS4G_ERR_SHAPE;
+    if (T > 0 && (!logits || !x || !aligned16(x) || !idx || !w || !row_to_slot || !slot_to_row))
+        return DS4G_ERR_INVALID_ARG;
+    ds4g_status st = check_fp4(x_q, T, K, fmt, true);
+    if (st != DS4G_OK) return st;
+    st = check_fp4(a_perm, S_, K, fmt, true);
+    if (st != DS4G_OK) return st;
+    const size_t need = ds4g_dispatch_workspace_bytes(T, k, E, fmt, g_in != nullptr);
+    if (S_ > 0 && (!workspace || ws_bytes < need || !aligned16(workspace))) return DS4G_ERR_WORKSPACE;
+    if (S_ == 0) {
+        // nothing routed: what the separate calls do on an empty batch
+        // (offsets all zero; the permuted tensor takes x_q's tensor scale)
+        if (cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (E + 1), S(stream)) != cudaSuccess) return DS4G_ERR_CUDA;
+        if (fmt == DS4G_NVFP4 &&
+            cudaMemcpyAsync(a_perm->g, x_q->g, sizeof(float), cudaMemcpyDeviceToDevice, S(stream)) != cudaSuccess)
+            return DS4G_ERR_CUDA;
+        return DS4G_OK;
+    }
+    return cuda_status(launch_dispatch(logits, x, dtype, T, E, k, K, fmt, g_in, idx, w, x_q->data, x_q->scales,
+                                       x_q->g, offsets, row_to_slot, slot_to_row, a_perm->data, a_perm->scales,
+                                       a_perm->g, workspace, S(stream)));
+}
+
 static ds4g_status grouped_gemm(const ds4g_fp4* a, const int32_t* offsets, int E, int max_rows_per_expert,
                                 const ds4g_fp4* w, int N, int epilogue, float* out, ds4g_fp4* out_q, float* h_debug,
                                 const int32_t* row_to_slot, const float* route_w, int k, int T, void* stream)

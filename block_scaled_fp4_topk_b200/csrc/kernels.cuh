@@ -14,6 +14,11 @@ cudaError_t launch_route_topk(const float* logits, int T, int E, int k, int32_t*
                               cudaStream_t st);
 
 size_t permute_workspace_bytes(int T, int k, int E);
+size_t dispatch_workspace_bytes(int T, int k, int E, int fmt, int has_g_in);
+cudaError_t launch_dispatch(const float* logits, const void* x, int dtype, int Tn, int E, int k, int64_t d, int fmt,
+                            const float* g_in, int32_t* idx, float* w, uint8_t* xd, uint8_t* xs, float* xg,
+                            int32_t* offsets, int32_t* r2s, int32_t* s2r, uint8_t* ad, uint8_t* as, float* ag,
+                            void* ws, cudaStream_t st);
 cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, const uint8_t* xd, const uint8_t* xs,
                            const float* xg, int64_t K, int fmt, int32_t* offsets, int32_t* row_to_slot,
                            int32_t* slot_to_row, uint8_t* ad, uint8_t* as, float* ag, void* ws,

@@ -11,14 +11,12 @@
 
 namespace ds4g {
 
+// one token's routing by one warp: lane j < k receives the j-th pick (expert
+// and softmax weight over the k picks)
 template <int VPL>  // logits per lane (E <= 32 * VPL)
-__global__ void k_route_topk(const float* __restrict__ logits, int T, int E, int k,
-                             int32_t* __restrict__ idx, float* __restrict__ w)
+__device__ __forceinline__ void route_token(const float* __restrict__ l, int E, int k, int lane, int& out_e,
+                                            float& out_w)
 {
-    const int lane = threadIdx.x & 31;
-    const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-    if (t >= T) return;
-    const float* l = logits + (int64_t)t * E;
     float v[VPL];
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
@@ -51,9 +49,23 @@ __global__ void k_route_topk(const float* __restrict__ logits, int T, int E, int
         den += p;
         if (lane == j) { my_e = be; my_v = p; }
     }
+    out_e = my_e;
+    out_w = __fdiv_rn(my_v, den);
+}
+
+template <int VPL>
+__global__ void k_route_topk(const float* __restrict__ logits, int T, int E, int k,
+                             int32_t* __restrict__ idx, float* __restrict__ w)
+{
+    const int lane = threadIdx.x & 31;
+    const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (t >= T) return;
+    int e;
+    float wt;
+    route_token<VPL>(logits + (int64_t)t * E, E, k, lane, e, wt);
     if (lane < k) {
-        idx[(int64_t)t * k + lane] = my_e;
-        w[(int64_t)t * k + lane] = __fdiv_rn(my_v, den);
+        idx[(int64_t)t * k + lane] = e;
+        w[(int64_t)t * k + lane] = wt;
     }
 }
 

@@ -5,6 +5,7 @@
 #include "quantize.cu"
 #include "route.cu"
 #include "permute.cu"
+#include "dispatch.cu"
 #include "gemv.cu"
 #include "gemm_tc.cu"
 #include "gemv_tc.cu"

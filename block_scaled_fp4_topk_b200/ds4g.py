@@ -50,6 +50,9 @@ _SIGS = {
     "ds4g_route_topk": ([_vp, _i32, _i32, _i32, _vp, _vp, _vp], _i32),
     "ds4g_permute_workspace_bytes": ([_i32, _i32, _i32], _sz),
     "ds4g_moe_permute": ([_vp, _i32, _i32, _i32, _P, _vp, _vp, _vp, _P, _vp, _sz, _vp], _i32),
+    "ds4g_dispatch_workspace_bytes": ([_i32, _i32, _i32, _i32, _i32], _sz),
+    "ds4g_moe_dispatch": ([_vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _P, _vp, _vp, _vp, _P, _vp, _sz,
+                           _vp], _i32),
     "ds4g_grouped_gemm_fp4": ([_P, _vp, _i32, _i32, _P, _i32, _i32, _vp, _P, _vp, _vp], _i32),
     "ds4g_swiglu_requant": ([_vp, _i64, _i32, _i32, _P, _vp, _vp], _i32),
     "ds4g_grouped_gemm_fp4_combine": ([_P, _vp, _i32, _i32, _P, _i32, _vp, _vp, _i32, _i32, _vp, _vp], _i32),
@@ -164,6 +167,45 @@ def ds4g_moe_permute(idx, E, x_q, offsets=None, row_to_slot=None, slot_to_row=No
                                                      row_to_slot.data_ptr(), slot_to_row.data_ptr(), ctypes.byref(ac),
                                                      workspace.data_ptr(), workspace.numel(), _stream()))
     return offsets, row_to_slot[:S], slot_to_row[:S], a_perm
+
+
+def dispatch_workspace(T, k, E, fmt, has_g_in=False, device="cuda"):
+    n = _lib.ds4g_dispatch_workspace_bytes(T, k, E, fmt, 1 if has_g_in else 0)
+    return torch.empty(max(n, 16), dtype=torch.uint8, device=device)
+
+
+def ds4g_moe_dispatch(logits, x, k, fmt, g_in=None, idx=None, w=None, x_q=None, offsets=None, row_to_slot=None,
+                      slot_to_row=None, a_perm=None, workspace=None):
+    """route + quantise + permute in one call; returns
+    (idx, w, x_q, offsets, row_to_slot[:S], slot_to_row[:S], a_perm)"""
+    T, E = logits.shape
+    d = x.shape[1]
+    S = T * k
+    dev = x.device
+    if idx is None:
+        idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    if w is None:
+        w = torch.empty((T, k), dtype=torch.float32, device=dev)
+    if x_q is None:
+        x_q = Fp4Tensor.empty(T, d, fmt, dev)
+    if offsets is None:
+        offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    if row_to_slot is None:
+        row_to_slot = torch.empty(max(S, 1), dtype=torch.int32, device=dev)
+    if slot_to_row is None:
+        slot_to_row = torch.empty(max(S, 1), dtype=torch.int32, device=dev)
+    if a_perm is None:
+        a_perm = Fp4Tensor.empty(S, d, fmt, dev)
+    if workspace is None:
+        workspace = dispatch_workspace(T, k, E, fmt, g_in is not None, dev)
+    dtype = BF16 if x.dtype == torch.bfloat16 else F32
+    xc, ac = x_q.c(), a_perm.c()
+    _check("ds4g_moe_dispatch",
+           _lib.ds4g_moe_dispatch(logits.data_ptr(), x.data_ptr(), dtype, T, E, k, fmt, _ptr(g_in), idx.data_ptr(),
+                                  w.data_ptr(), ctypes.byref(xc), offsets.data_ptr(), row_to_slot.data_ptr(),
+                                  slot_to_row.data_ptr(), ctypes.byref(ac), workspace.data_ptr(), workspace.numel(),
+                                  _stream()))
+    return idx, w, x_q, offsets, row_to_slot[:S], slot_to_row[:S], a_perm
 
 
 def ds4g_moe_permute_static(idx, E, x_q, offsets=None, row_to_slot=None, slot_to_row=None, a_perm=None):

@@ -13,7 +13,7 @@ from .ds4g import EPI_NONE, EPI_SWIGLU_REQUANT, NVFP4, Fp4Tensor
 
 
 class MoeLayer:
-    def __init__(self, w1, w2, E, k, d, I, fmt, g_h=None, fused=True, fused_combine=True):
+    def __init__(self, w1, w2, E, k, d, I, fmt, g_h=None, fused=True, fused_combine=True, fused_dispatch=True):
         """w1: Fp4Tensor [E*2I][d] (gate rows then up rows per expert),
         w2: Fp4Tensor [E*d][I]; NVFP4 weights carry one tensor scale per
         expert (w.g has E floats); g_h: the static NVFP4 tensor scale of h."""
@@ -21,6 +21,7 @@ class MoeLayer:
         self.E, self.k, self.d, self.I, self.fmt = E, k, d, I, fmt
         self.fused = fused
         self.fused_combine = fused_combine
+        self.fused_dispatch = fused_dispatch
         self.g_h = None
         if fmt == NVFP4:
             dev = w1.data.device
@@ -43,6 +44,7 @@ class MoeLayer:
                 hq=Fp4Tensor.empty(S, self.I, self.fmt, device),
                 out=torch.empty((T, self.d), dtype=torch.float32, device=device),
                 pws=ds4g.permute_workspace(T, self.k, self.E, device),
+                dws=ds4g.dispatch_workspace(T, self.k, self.E, self.fmt, False, device),
                 qws=torch.empty(16, dtype=torch.uint8, device=device),
             )
             if self.fmt == NVFP4:
@@ -63,7 +65,14 @@ class MoeLayer:
         return self.fc2(b, T)
 
     def dispatch(self, x, logits, b):
-        """routing, activation quantisation and the expert-contiguous permutation"""
+        """routing, activation quantisation and the expert-contiguous
+        permutation (one library call; self.fused_dispatch=False issues the
+        three separate calls)"""
+        if self.fused_dispatch:
+            ds4g.ds4g_moe_dispatch(logits, x, self.k, self.fmt, idx=b["idx"], w=b["w"], x_q=b["xq"],
+                                   offsets=b["offsets"], row_to_slot=b["r2s"], slot_to_row=b["s2r"], a_perm=b["a"],
+                                   workspace=b["dws"])
+            return
         ds4g.ds4g_route_topk(logits, self.k, idx=b["idx"], w=b["w"])
         ds4g.ds4g_quantize_mx(x, self.fmt, out=b["xq"], workspace=b["qws"])
         ds4g.ds4g_moe_permute(b["idx"], self.E, b["xq"], offsets=b["offsets"], row_to_slot=b["r2s"],

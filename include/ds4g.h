@@ -6,11 +6,13 @@
  *   ds4g_route_topk       top-k routing of each token over E experts
  *   ds4g_quantize_mx      activations -> MXFP4 / NVFP4 (on the fly)
  *   ds4g_moe_permute      expert-contiguous reordering of the quantised rows
+ *     (ds4g_moe_dispatch does these three in one call)
  *   ds4g_grouped_gemm_fp4 FC1 (gate+up), optionally with the SwiGLU +
  *                         requantisation epilogue fused
  *   ds4g_swiglu_requant   the same epilogue as a separate step
  *   ds4g_grouped_gemm_fp4 FC2
  *   ds4g_moe_combine      routing-weighted sum of each token's k expert rows
+ *     (ds4g_grouped_gemm_fp4_combine does FC2 and the combine in one call)
  *
  * Sources: "DGX Spark native FP4 matrix instructions: how DwarfStar uses
  * Blackwell" (sec. 1 FP4 formats and the block-scaled MMA, sec. 2 MoE
@@ -133,6 +135,27 @@ size_t ds4g_permute_workspace_bytes(int T, int k, int E);
 ds4g_status ds4g_moe_permute(const int32_t* idx, int T, int k, int E, const ds4g_fp4* x_q,
                              int32_t* offsets, int32_t* row_to_slot, int32_t* slot_to_row,
                              ds4g_fp4* a_perm, void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Dispatch: ds4g_route_topk, ds4g_quantize_mx and ds4g_moe_permute as one call
+ * (the routing, quantisation and permutation steps of the pages cited at each
+ * of those three).  Same arguments and the same results, bit for bit, as
+ *   ds4g_route_topk(logits, T, E, k, idx, w);
+ *   ds4g_quantize_mx(x, dtype, T, x_q->K, fmt, g_in, x_q, ...);
+ *   ds4g_moe_permute(idx, T, k, E, x_q, offsets, row_to_slot, slot_to_row, a_perm, ...);
+ * x: [T][x_q->K] bf16 or fp32 (16-byte aligned).  x_q: [T] rows, a_perm:
+ * [T*k] rows, both of format fmt (NVFP4: both need g; with g_in NULL the
+ * tensor scale is derived from amax |x| as ds4g_quantize_mx does).
+ * Up to 512 slots (T*k) one kernel does all three steps (decode batches);
+ * larger batches run the separate calls' kernels.  Limits as the separate
+ * calls: E <= 1024, 1 <= k <= min(E, 32), K % 64 == 0.
+ * Workspace: ds4g_dispatch_workspace_bytes(T, k, E, fmt, g_in != NULL), 16-byte
+ * aligned, owned by the caller. */
+size_t ds4g_dispatch_workspace_bytes(int T, int k, int E, int fmt, int has_g_in);
+ds4g_status ds4g_moe_dispatch(const float* logits, const void* x, int dtype, int T, int E, int k, int fmt,
+                              const float* g_in, int32_t* idx, float* w, ds4g_fp4* x_q, int32_t* offsets,
+                              int32_t* row_to_slot, int32_t* slot_to_row, ds4g_fp4* a_perm,
+                              void* workspace, size_t workspace_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
  * Grouped block-scaled FP4 GEMM ("DGX Spark native FP4 ..." sec. 1-2; the

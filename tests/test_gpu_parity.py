@@ -134,6 +134,56 @@ def test_permute_empty():
     assert np.array_equal(offs.cpu().numpy(), np.zeros(E + 1, np.int32))
 
 
+# ---- dispatch (route + quantise + permute in one call) --------------------------
+
+@pytest.mark.parametrize("T,k,E,fmt,f32,g_given", [
+    (1, 6, 256, MX, False, False), (8, 6, 256, NV, False, False), (85, 6, 256, MX, False, False),
+    (86, 6, 256, MX, False, False), (16, 2, 8, NV, True, True), (300, 6, 256, NV, False, False),
+    (37, 6, 1000, MX, True, False), (4, 8, 8, NV, False, True), (512, 1, 64, MX, False, False)])
+def test_dispatch_bitexact(T, k, E, fmt, f32, g_given):
+    """single-CTA path up to 512 slots (T*k), the three-kernel path above;
+    every output bit-exact against the oracle's routing, quantisation and
+    permutation of the same inputs"""
+    K = 512
+    lg = synth.logits(T, E, 3, 1.5)
+    if f32:
+        xr = _x_f32(T, K, 61, 2.0)
+        xd = torch.from_numpy(xr).to(dev())
+    else:
+        bits = synth.normal_bf16_bits((T, K), 0, 61, 2.0)
+        xd = bf16_dev(bits)
+        xr = synth.bf16_bits_to_f32(bits)
+    g = np.float32(0.0117) if g_given else None
+    idx, w, xq, offs, r2s, s2r, a = ds4g.ds4g_moe_dispatch(
+        torch.from_numpy(lg).to(dev()), xd, k, fmt, g_in=torch.tensor([g], device=dev()) if g_given else None)
+    ds4g.ds4g_check_device()
+    ridx, rw = oracle.route_topk(lg, k)
+    assert np.array_equal(idx.cpu().numpy(), ridx)
+    assert np.allclose(w.cpu().numpy(), rw, rtol=0, atol=2e-6)
+    rq = oracle.quantize(xr, fmt, g=float(g) if g_given else None)
+    gq = from_dev(xq)
+    assert np.array_equal(gq.data, rq.data) and np.array_equal(gq.scales, rq.scales)
+    if fmt == NV:
+        assert np.float32(gq.g) == np.float32(rq.g)
+    roffs, rr2s, rs2r = oracle.moe_permute(ridx, E)
+    assert np.array_equal(offs.cpu().numpy(), roffs)
+    assert np.array_equal(r2s.cpu().numpy(), rr2s) and np.array_equal(s2r.cpu().numpy(), rs2r)
+    ra = oracle.gather_rows(rq, rr2s, k)
+    ga = from_dev(a)
+    assert np.array_equal(ga.data, ra.data) and np.array_equal(ga.scales, ra.scales)
+    if fmt == NV:
+        assert np.float32(ga.g) == np.float32(rq.g)
+
+
+def test_dispatch_empty():
+    E = 8
+    lg = torch.empty((0, E), dtype=torch.float32, device=dev())
+    x = torch.empty((0, 256), dtype=torch.bfloat16, device=dev())
+    _, _, _, offs, _, _, _ = ds4g.ds4g_moe_dispatch(lg, x, 2, MX)
+    ds4g.ds4g_check_device()
+    assert np.array_equal(offs.cpu().numpy(), np.zeros(E + 1, np.int32))
+
+
 # ---- grouped GEMM ------------------------------------------------------------------
 
 def _grouped_problem(seg, N, K, fmt, stream=11):
@@ -297,13 +347,15 @@ def test_combine():
 
 # ---- full layer --------------------------------------------------------------------
 
-@pytest.mark.parametrize("fused,fused_combine", [(True, True), (False, False), (True, False)])
-def test_layer_tiny(fused, fused_combine):
+@pytest.mark.parametrize("fused,fused_combine,fused_dispatch", [(True, True, True), (False, False, False),
+                                                               (True, False, True)])
+def test_layer_tiny(fused, fused_combine, fused_dispatch):
     from synth import workloads
     from block_scaled_fp4_topk_b200.layer import MoeLayer
     wl = workloads.WORKLOADS["tiny"]
     w1, w2 = MoeLayer.synthetic_weights(wl.E, wl.d, wl.I, wl.fmt, device=dev())
-    layer = MoeLayer(w1, w2, wl.E, wl.k, wl.d, wl.I, wl.fmt, fused=fused, fused_combine=fused_combine)
+    layer = MoeLayer(w1, w2, wl.E, wl.k, wl.d, wl.I, wl.fmt, fused=fused, fused_combine=fused_combine,
+                     fused_dispatch=fused_dispatch)
     xb = workloads.host_x_bits(wl)
     lg = workloads.host_logits(wl)
     out = layer.forward(bf16_dev(xb), torch.from_numpy(lg).to(dev())).cpu().numpy()
