@@ -56,8 +56,8 @@ constexpr unsigned long long kWaitNs = 4000000000ull;
 // the scale columns fit the 512 TMEM columns, 2 x 256 do not.
 template <int FMT, int TBN, int NISS>
 struct Cfg {
-    static_assert(TBN == 256 || TBN == 224, "tile width");
-    static_assert(NISS == 1 || (NISS == 2 && TBN == 224), "two issuers need two accumulators");
+    static_assert(TBN == 256 || TBN == 224 || TBN == 192, "tile width");
+    static_assert(NISS == 1 || (NISS == 2 && TBN < 256), "two issuers need two accumulators");
     static constexpr int NACC = (TBN == 256) ? 1 : 2;               // accumulator buffers
     static constexpr int HALF = TBN / 2;                             // weight rows per TMA box
     static constexpr int B_BYTES = TBN * BKB;
@@ -314,8 +314,8 @@ __device__ __forceinline__ void w_rows(const Tile& tl, int N, int I, int64_t& y0
 {
     const int64_t wbase = (int64_t)tl.e * N;
     if (EPI == DS4G_EPI_SWIGLU_REQUANT) {
-        y0 = wbase + (int64_t)tl.nt * 128;          // gate rows
-        y1 = wbase + I + (int64_t)tl.nt * 128;      // up rows
+        y0 = wbase + (int64_t)tl.nt * (TBN / 2);          // gate rows
+        y1 = wbase + I + (int64_t)tl.nt * (TBN / 2);      // up rows
     } else {
         y0 = wbase + (int64_t)tl.nt * TBN;
         y1 = y0 + TBN / 2;
@@ -329,7 +329,8 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
 {
     using C = Cfg<FMT, TBN, NISS>;
     constexpr int SF_STAGES = C::SF_STAGES;
-    static_assert(EPI != DS4G_EPI_SWIGLU_REQUANT || TBN == 256, "SwiGLU tiles pair 128 gate and 128 up rows");
+    static_assert(EPI != DS4G_EPI_SWIGLU_REQUANT || TBN == 256 || TBN == 192,
+                  "SwiGLU tiles pair TBN/2 gate and TBN/2 up rows, a multiple of 32 each");
     constexpr int NACC = C::NACC;
     constexpr int B_BYTES = C::B_BYTES;
     extern __shared__ uint8_t smem_raw[];
@@ -357,7 +358,9 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
     const int nks = (int)ceil_div(K, BK);
     const int npairs = (nks + 1) / 2;
     const int I = p.N / 2;
-    const int n_tiles = (EPI == DS4G_EPI_SWIGLU_REQUANT) ? (I / 128) : (p.N / TBN);
+    // SwiGLU: the last tile may be ragged (I % (TBN/2) != 0); its columns past
+    // I are computed from other rows and never stored
+    const int n_tiles = (EPI == DS4G_EPI_SWIGLU_REQUANT) ? (int)ceil_div(I, TBN / 2) : (p.N / TBN);
 
     // ---- prologue
     if (threadIdx.x == 0) {
@@ -673,12 +676,13 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
                 }
             } else {
 #pragma unroll 1
-                for (int j = 0; j < 2; ++j) {
-                    const int gcol = half * 64 + 32 * j;            // gate column within the tile
+                for (int j = half; j < C::HALF / 32; j += 2) {       // 32-column blocks of h
+                    const int gcol = 32 * j;                         // gate column within the tile
+                    const int64_t col0 = (int64_t)tl.nt * C::HALF + gcol;
+                    if (col0 >= I) break;                            // ragged last tile
                     float gv[32], uv[32];
                     tmem_ld32(tbase + gcol, gv);
-                    tmem_ld32(tbase + 128 + gcol, uv);
-                    const int64_t col0 = (int64_t)tl.nt * 128 + gcol;
+                    tmem_ld32(tbase + C::HALF + gcol, uv);
                     float h[32];
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
@@ -827,10 +831,10 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st)
     if (a.fmt == DS4G_MXFP4)
         return a.epilogue == DS4G_EPI_NONE ? run_tc_plain<DS4G_MXFP4, DS4G_EPI_NONE>(a, st)
              : a.epilogue == kEpiCombine   ? run_tc_plain<DS4G_MXFP4, kEpiCombine>(a, st)
-                                           : run_tc<DS4G_MXFP4, DS4G_EPI_SWIGLU_REQUANT, 256, 1>(a, st);
+                                           : run_tc<DS4G_MXFP4, DS4G_EPI_SWIGLU_REQUANT, 192, 2>(a, st);
     return a.epilogue == DS4G_EPI_NONE ? run_tc_plain<DS4G_NVFP4, DS4G_EPI_NONE>(a, st)
          : a.epilogue == kEpiCombine   ? run_tc_plain<DS4G_NVFP4, kEpiCombine>(a, st)
-                                       : run_tc<DS4G_NVFP4, DS4G_EPI_SWIGLU_REQUANT, 256, 1>(a, st);
+                                       : run_tc<DS4G_NVFP4, DS4G_EPI_SWIGLU_REQUANT, 192, 2>(a, st);
 }
 
 }  // namespace ds4g

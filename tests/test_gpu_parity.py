@@ -260,7 +260,8 @@ def _h_bound(y1_ref, ab1, I):
 @pytest.mark.parametrize("fmt", [MX, NV])
 @pytest.mark.parametrize("case", [([3, 0, 1, 8, 5], 256, 7168), ([300, 0, 1, 129, 77], 256, 512),
                                   ([2, 1], 64, 256), ([131], 128, 2048), ([20, 0, 150], 128, 768),
-                                  ([200, 9], 384, 1024), ([100, 30], 96, 1024), ([5, 16, 2], 192, 1024)])
+                                  ([200, 9], 384, 1024), ([100, 30], 96, 1024), ([5, 16, 2], 192, 1024),
+                                  ([140, 60], 160, 512)])
 def test_fc1_fused_swiglu_requant(fmt, case):
     seg, I, K = case
     offsets, a, w, gw = _grouped_problem(seg, 2 * I, K, fmt, stream=21)
