@@ -360,7 +360,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
     const int I = p.N / 2;
     // SwiGLU: the last tile may be ragged (I % (TBN/2) != 0); its columns past
     // I are computed from other rows and never stored
-    const int n_tiles = (EPI == DS4G_EPI_SWIGLU_REQUANT) ? (int)ceil_div(I, TBN / 2) : (p.N / TBN);
+    const int n_tiles = (EPI == DS4G_EPI_SWIGLU_REQUANT) ? (int)ceil_div(I, TBN / 2) : (int)ceil_div(p.N, TBN);
 
     // ---- prologue
     if (threadIdx.x == 0) {
@@ -643,6 +643,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
 #pragma unroll 1
                 for (int c8 = 0; c8 < C::HALF / 32; ++c8) {
                     const int col = half * C::HALF + 32 * c8;
+                    if ((int64_t)tl.nt * TBN + col >= p.N) break;   // ragged last tile (N % 32 == 0)
                     float v[32];
                     tmem_ld32(tbase + col, v);
                     if (valid) {
@@ -807,14 +808,18 @@ static cudaError_t run_tc(const GemmArgs& a, cudaStream_t st)
     return cudaGetLastError();
 }
 
-// plain and combine epilogues: 224-column tiles with two accumulators when N
-// allows (and, for MXFP4, whose scale columns fit beside them, two MMA
-// issuers), else 256-column tiles
+// plain and combine epilogues, N % 224 == 0 (FC2, N = 7168): 224-column
+// tiles with two accumulators; MXFP4 with two MMA issuers, NVFP4 (whose scale
+// columns do not fit beside them twice) with one issuer and the staged
+// epilogue.  (NVFP4 192-column tiles with two issuers measured slower: FC2
+// at T = 16384 2.48 ms against 1.92 ms.)  Other N: 256-column tiles, one
+// accumulator.
 template <int FMT, int EPI>
 static cudaError_t run_tc_plain(const GemmArgs& a, cudaStream_t st)
 {
-    constexpr int kIss224 = (FMT == DS4G_MXFP4) ? 2 : 1;
-    return (a.N % 224 == 0) ? run_tc<FMT, EPI, 224, kIss224>(a, st) : run_tc<FMT, EPI, 256, 1>(a, st);
+    if (a.N % 224 != 0) return run_tc<FMT, EPI, 256, 1>(a, st);
+    if constexpr (FMT == DS4G_MXFP4) return run_tc<FMT, EPI, 224, 2>(a, st);
+    else return run_tc<FMT, EPI, 224, 1>(a, st);
 }
 
 bool gemm_tc_supports(int fmt, int64_t K)
