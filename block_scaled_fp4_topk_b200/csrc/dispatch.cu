@@ -13,8 +13,9 @@
 // every warp routes tokens, the CTA counts the picks per expert, one warp
 // scans and ranks them stably, and then each token row is quantised once and
 // its packed blocks are written both to x_q and to the token's k permuted
-// rows (no second pass that reads x_q back).  Larger batches run the three
-// kernels of the separate calls.
+// rows (no second pass that reads x_q back).  Larger batches run the
+// separate calls' routing and ranking kernels, then one quantise-and-scatter
+// pass.
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -160,6 +161,51 @@ k_dispatch_small(const float* __restrict__ logits, const T* __restrict__ x, int 
     }
 }
 
+// larger batches: the permutation is ranked first, then each token row is
+// quantised once and written to x_q and to its k permuted rows (the separate
+// calls quantise, then gather the rows back out of x_q)
+template <typename T, int FMT>
+__global__ void k_quant_scatter(const T* __restrict__ x, int Tn, int64_t d, int k, const float* __restrict__ g_ptr,
+                                const int32_t* __restrict__ slot_to_row, uint8_t* __restrict__ xd,
+                                uint8_t* __restrict__ xs, uint8_t* __restrict__ ad, uint8_t* __restrict__ as,
+                                float* __restrict__ ag)
+{
+    constexpr int BLK = (FMT == DS4G_MXFP4) ? 32 : 16;
+    const float g = (FMT == DS4G_NVFP4) ? *g_ptr : 1.0f;
+    if (FMT == DS4G_NVFP4 && blockIdx.x == 0 && threadIdx.x == 0) *ag = g;
+    const int64_t bpr = d / BLK;
+    const int64_t nb = (int64_t)Tn * bpr;
+    for (int64_t b = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; b < nb; b += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t t = b / bpr;
+        const int64_t c = b - t * bpr;
+        float v[BLK];
+        load_block<T>(x + t * d + c * BLK, v, BLK);
+        if (FMT == DS4G_MXFP4) {
+            uint4 pk;
+            uint8_t sc;
+            quant_mx_block(v, pk, sc);
+            reinterpret_cast<uint4*>(xd)[b] = pk;
+            xs[b] = sc;
+            for (int j = 0; j < k; ++j) {
+                const int64_t r = slot_to_row[t * k + j];
+                *reinterpret_cast<uint4*>(ad + r * (d / 2) + c * 16) = pk;
+                as[r * bpr + c] = sc;
+            }
+        } else {
+            uint2 pk;
+            uint8_t sc;
+            quant_nv_block(v, g, pk, sc);
+            reinterpret_cast<uint2*>(xd)[b] = pk;
+            xs[b] = sc;
+            for (int j = 0; j < k; ++j) {
+                const int64_t r = slot_to_row[t * k + j];
+                *reinterpret_cast<uint2*>(ad + r * (d / 2) + c * 8) = pk;
+                as[r * bpr + c] = sc;
+            }
+        }
+    }
+}
+
 size_t dispatch_workspace_bytes(int T, int k, int E, int fmt, int has_g_in)
 {
     // the multi-kernel path: the permutation's counts, then the quantiser's
@@ -207,13 +253,49 @@ cudaError_t launch_dispatch(const float* logits, const void* x, int dtype, int T
                    : launch_small<float, DS4G_NVFP4>(logits, (const float*)x, Tn, E, k, d, g_in, idx, w, xd, xs, xg,
                                                      offsets, r2s, s2r, ad, as, ag, st);
     }
+    // route; NVFP4 tensor scale (amax, g) unless given; counts, scan, ranks;
+    // then one pass that quantises and scatters
     cudaError_t e = launch_route_topk(logits, Tn, E, k, idx, w, st);
     if (e != cudaSuccess) return e;
     const size_t pw = (permute_workspace_bytes(Tn, k, E) + 15) / 16 * 16;
-    e = launch_quantize(x, dtype, Tn, d, fmt, g_in, xd, xs, fmt == DS4G_NVFP4 ? xg : nullptr,
-                        static_cast<uint8_t*>(ws) + pw, st);
-    if (e != cudaSuccess) return e;
-    return launch_permute(idx, Tn, k, E, xd, xs, xg, d, fmt, offsets, r2s, s2r, ad, as, ag, ws, st);
+    const float* g = nullptr;
+    if (fmt == DS4G_NVFP4) {
+        if (g_in) {
+            if (g_in != xg) e = cudaMemcpyAsync(xg, g_in, sizeof(float), cudaMemcpyDeviceToDevice, st);
+        } else {
+            unsigned int* amax = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(ws) + pw);
+            e = cudaMemsetAsync(amax, 0, sizeof(unsigned int), st);
+            if (e != cudaSuccess) return e;
+            const int64_t n = (int64_t)Tn * d;
+            const int64_t ga0 = ceil_div(n / 8, 256);
+            const int ga = (int)(ga0 < (int64_t)kNumSMs * 16 ? ga0 : (int64_t)kNumSMs * 16);
+            if (dtype == DS4G_BF16) k_amax<uint16_t><<<ga, 256, 0, st>>>((const uint16_t*)x, n, amax);
+            else k_amax<float><<<ga, 256, 0, st>>>((const float*)x, n, amax);
+            k_g_from_amax<<<1, 1, 0, st>>>(amax, xg);
+            e = cudaGetLastError();
+        }
+        if (e != cudaSuccess) return e;
+        g = xg;
+    }
+    int32_t* pws = reinterpret_cast<int32_t*>(ws);
+    const int B = (int)ceil_div(S, kChunk);
+    const size_t shm = (size_t)E * sizeof(int32_t);
+    k_perm_hist<<<B, 256, shm, st>>>(idx, S, E, B, pws);
+    k_perm_scan<<<1, 1024, 0, st>>>(pws, E * B, E, B, S, offsets);
+    k_perm_rank<<<B, 32, shm, st>>>(idx, S, E, B, pws, r2s, s2r);
+    const int64_t nb = (int64_t)Tn * (d / (fmt == DS4G_MXFP4 ? 32 : 16));
+    const int64_t gq0 = ceil_div(nb, 256);
+    const int gq = (int)(gq0 < (int64_t)kNumSMs * 16 ? gq0 : (int64_t)kNumSMs * 16);
+#define DS4G_QS(TT, F) k_quant_scatter<TT, F><<<gq, 256, 0, st>>>((const TT*)x, Tn, d, k, g, s2r, xd, xs, ad, as, ag)
+    if (fmt == DS4G_MXFP4) {
+        if (dtype == DS4G_BF16) DS4G_QS(uint16_t, DS4G_MXFP4);
+        else DS4G_QS(float, DS4G_MXFP4);
+    } else {
+        if (dtype == DS4G_BF16) DS4G_QS(uint16_t, DS4G_NVFP4);
+        else DS4G_QS(float, DS4G_NVFP4);
+    }
+#undef DS4G_QS
+    return cudaGetLastError();
 }
 
 }  // namespace ds4g

@@ -17,7 +17,7 @@
 
 namespace ds4g {
 
-constexpr int kChunk = 1024;
+constexpr int kChunk = 256;       // slots per rank warp (more warps in flight than 1024-slot chunks)
 
 size_t permute_workspace_bytes(int T, int k, int E)
 {
@@ -40,30 +40,53 @@ __global__ void k_perm_hist(const int32_t* __restrict__ idx, int64_t S, int E, i
 }
 
 // exclusive scan of n = E*B ints in place (one block of 1024 threads); also
-// offsets[e] = scanned[e*B], offsets[E] = S
-__global__ void k_perm_scan(int32_t* __restrict__ ws, int n, int E, int B, int64_t S, int32_t* __restrict__ offsets)
+// offsets[e] = scanned[e*B], offsets[E] = S.  Tiles of 4096 ints: each thread
+// takes 4 adjacent ones (a warp reads 512 contiguous bytes), scans them, then
+// warp and block scans of the thread totals and a carry across tiles.
+__global__ void __launch_bounds__(1024) k_perm_scan(int32_t* __restrict__ ws, int n, int E, int B, int64_t S,
+                                                    int32_t* __restrict__ offsets)
 {
-    __shared__ int32_t part[1024];
-    const int tid = threadIdx.x;
-    const int per = (n + blockDim.x - 1) / blockDim.x;
-    const int b0 = tid * per, b1 = min(b0 + per, n);
-    int32_t sum = 0;
-    for (int i = b0; i < b1; ++i) sum += ws[i];
-    part[tid] = sum;
+    __shared__ int32_t wsum[32];
+    __shared__ int32_t carry_s;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (tid == 0) carry_s = 0;
     __syncthreads();
-    for (int o = 1; o < (int)blockDim.x; o <<= 1) {   // Hillis-Steele inclusive scan
-        int32_t v = (tid >= o) ? part[tid - o] : 0;
+    for (int base = 0; base < n; base += 4 * 1024) {
+        const int i0 = base + 4 * tid;
+        int32_t v[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) v[j] = (i0 + j < n) ? ws[i0 + j] : 0;
+        const int32_t tsum = v[0] + v[1] + v[2] + v[3];
+        int32_t incl = tsum;                               // inclusive scan of thread totals in the warp
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (lane == 31) wsum[warp] = incl;
         __syncthreads();
-        part[tid] += v;
+        if (warp == 0) {
+            const int32_t x = wsum[lane];
+            int32_t wi = x;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int32_t y = __shfl_up_sync(0xffffffffu, wi, o);
+                if (lane >= o) wi += y;
+            }
+            wsum[lane] = wi - x;                           // exclusive base of each warp
+        }
+        __syncthreads();
+        const int32_t carry = carry_s;
+        int32_t run = carry + wsum[warp] + incl - tsum;    // exclusive base of this thread
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            if (i0 + j < n) ws[i0 + j] = run;
+            run += v[j];
+        }
+        __syncthreads();                                   // every thread has read carry_s and wsum
+        if (tid == 1023) carry_s = run;                    // the tile's total, carried on
         __syncthreads();
     }
-    int32_t run = part[tid] - sum;                      // exclusive base of this thread
-    for (int i = b0; i < b1; ++i) {
-        int32_t c = ws[i];
-        ws[i] = run;
-        run += c;
-    }
-    __syncthreads();
     for (int e = tid; e < E; e += blockDim.x) offsets[e] = ws[(int64_t)e * B];
     if (tid == 0) offsets[E] = (int32_t)S;
 }

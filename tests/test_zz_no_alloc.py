@@ -42,7 +42,7 @@ def test_permute_static_rejects_too_large():
     from block_scaled_fp4_topk_b200 import ds4g
     dev = torch.device("cuda:0")
     E, k = 4096, 6
-    T = 20000                                           # E * ceil(T*k/1024) * 4 B > 256 KiB
+    T = 20000                                           # E * ceil(T*k/256) * 4 B > 256 KiB
     assert ds4g._lib.ds4g_permute_workspace_bytes(T, k, E) > ds4g._lib.ds4g_permute_static_max_bytes()
     idx = torch.zeros((T, k), dtype=torch.int32, device=dev)
     xq = ds4g.Fp4Tensor.empty(T, 64, 0, dev)
