@@ -219,6 +219,17 @@ __device__ __forceinline__ void tc_commit(uint32_t mbar)
                  : "memory");
 }
 
+// 16 TMEM lanes x 16 columns: thread t gets lanes t/4 and t/4 + 8, columns
+// 2(t%4), 2(t%4)+1 (r0, r1 / r2, r3) and 8 + 2(t%4), +1 (r4, r5 / r6, r7)
+__device__ __forceinline__ void tmem_ld_16x256b_x2(uint32_t taddr, uint32_t* r)
+{
+    asm volatile("tcgen05.ld.sync.aligned.16x256b.x2.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr)
+                 : "memory");
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v)
 {
     uint32_t r[16];
@@ -639,41 +650,54 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
                         }
                     }
                 } else {
-                // this warp's half of the columns, 32-column pieces
+                    // 16-lane x 16-column TMEM loads: four threads hold 32
+                    // contiguous bytes of one row, so a store / reduction
+                    // instruction writes 8 rows x 32 bytes (full sectors)
+                    const int sub = lane & 3, rsub = lane >> 2;
 #pragma unroll 1
-                for (int c8 = 0; c8 < C::HALF / 32; ++c8) {
-                    const int col = half * C::HALF + 32 * c8;
-                    if ((int64_t)tl.nt * TBN + col >= p.N) break;   // ragged last tile (N % 32 == 0)
-                    float v[32];
-                    tmem_ld32(tbase + col, v);
-                    if (valid) {
-                        float* dst = dst_row + (int64_t)tl.nt * TBN + col;
+                    for (int hh = 0; hh < 2; ++hh) {
+                        float* dk[2];
+                        float wk[2];
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            if (EPI == kEpiCombine)
-                                red_add_v4(dst + 4 * i, v[4 * i] * wr, v[4 * i + 1] * wr, v[4 * i + 2] * wr, v[4 * i + 3] * wr);
-                            else
-                                reinterpret_cast<float4*>(dst)[i] =
-                                    make_float4(v[4 * i] * wr, v[4 * i + 1] * wr, v[4 * i + 2] * wr, v[4 * i + 3] * wr);
+                        for (int k = 0; k < 2; ++k) {
+                            const int64_t rk = tl.m0 + 32 * q + 16 * hh + rsub + 8 * k;
+                            dk[k] = nullptr;
+                            wk[k] = gscale;
+                            if (rk < tl.end) {
+                                if (EPI == kEpiCombine) {
+                                    const int32_t s = p.r2s[rk];
+                                    dk[k] = p.out + (int64_t)(s / p.topk) * p.N + (int64_t)tl.nt * TBN;
+                                    wk[k] = p.route_w[s] * gscale;
+                                } else {
+                                    dk[k] = p.out + rk * p.N + (int64_t)tl.nt * TBN;
+                                }
+                            }
+                        }
+                        const uint32_t tb = tmem + kColAcc + buf * TBN + ((uint32_t)(32 * q + 16 * hh) << 16);
+#pragma unroll 1
+                        for (int g = 0; g < C::HALF / 16; ++g) {
+                            const int col = half * C::HALF + 16 * g;
+                            if ((int64_t)tl.nt * TBN + col >= p.N) break;      // ragged last tile
+                            uint32_t r[8];
+                            tmem_ld_16x256b_x2(tb + col, r);
+#pragma unroll
+                            for (int k = 0; k < 2; ++k) {
+                                if (dk[k] == nullptr) continue;
+                                float* g0 = dk[k] + col + 2 * sub;
+                                const float a0 = __uint_as_float(r[2 * k]) * wk[k];
+                                const float a1 = __uint_as_float(r[2 * k + 1]) * wk[k];
+                                const float b0 = __uint_as_float(r[4 + 2 * k]) * wk[k];
+                                const float b1 = __uint_as_float(r[4 + 2 * k + 1]) * wk[k];
+                                if (EPI == kEpiCombine) {
+                                    red_add_v2(g0, a0, a1);
+                                    red_add_v2(g0 + 8, b0, b1);
+                                } else {
+                                    *reinterpret_cast<float2*>(g0) = make_float2(a0, a1);
+                                    *reinterpret_cast<float2*>(g0 + 8) = make_float2(b0, b1);
+                                }
+                            }
                         }
                     }
-                }
-                if (C::HALF % 32 != 0) {                    // the last 16 columns of a 112-wide half
-                    const int col = half * C::HALF + 32 * (C::HALF / 32);
-                    float v[16];
-                    tmem_ld16(tbase + col, v);
-                    if (valid) {
-                        float* dst = dst_row + (int64_t)tl.nt * TBN + col;
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            if (EPI == kEpiCombine)
-                                red_add_v4(dst + 4 * i, v[4 * i] * wr, v[4 * i + 1] * wr, v[4 * i + 2] * wr, v[4 * i + 3] * wr);
-                            else
-                                reinterpret_cast<float4*>(dst)[i] =
-                                    make_float4(v[4 * i] * wr, v[4 * i + 1] * wr, v[4 * i + 2] * wr, v[4 * i + 3] * wr);
-                        }
-                    }
-                }
                 }
             } else {
 #pragma unroll 1
