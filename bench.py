@@ -23,6 +23,10 @@ import time
 import numpy as np
 
 L2_BYTES = 126 * 1000 * 1000
+# DRAM bytes (read + write) of one FC1 launch, from a one-pass ncu capture of
+# the full-size workload (profiles/dram_traffic_k_gemm_tc_prefill_T2048_mxfp4.md);
+# workloads without a capture of the current kernel report null
+FC1_TRAFFIC = {"prefill": (2334835968, "profiles/dram_traffic_k_gemm_tc_prefill_T2048_mxfp4.md")}
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
@@ -344,9 +348,14 @@ def run_ours(args, rank, world, local_rank):
         roof = {"bound": "tensor", "achieved": alg["fc1_flops"] / fc1_s / 1e12, "peak": fp4_peak, "unit": "TFLOP/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["traffic"] = None
-    roof["kernel"] = "grouped FP4 GEMM FC1 + fused SwiGLU/requant (tcgen05)" if wl.T > 8 else "grouped FP4 GEMV FC1"
+    roof["kernel"] = ("FC1 + fused SwiGLU/requant, decode tensor-core kernel (weights as MMA M, <= 16 tokens as N)"
+                      if alg["max_rows"] <= 16 else
+                      "FC1 + fused SwiGLU/requant, tcgen05 grouped GEMM (128 x 192 tiles, two MMA issuers)")
     roof["peak_source"] = ("measured (MEASURED_PEAKS.json" + ("; FP4 = bf16 burst x 4 nominal ratio" if
                            roof["bound"] == "tensor" else "") + ")") if peaks else "fallback"
+    if args.workload in FC1_TRAFFIC:
+        roof["traffic"] = FC1_TRAFFIC[args.workload][0]
+        roof["traffic_source"] = FC1_TRAFFIC[args.workload][1]
     roof["fc1_ms"] = fc1_ms
     roof["fc1_tflops"] = alg["fc1_flops"] / fc1_s / 1e12
     roof["fc1_gbs"] = alg["fc1_bytes"] / fc1_s / 1e9
