@@ -35,7 +35,12 @@ def test_host_only_helpers():
     assert L.ds4g_status_str(0) == b"ok"
     assert b"64" in L.ds4g_status_str(2)
     assert L.ds4g_quantize_workspace_bytes(1, 0) >= 4 and L.ds4g_quantize_workspace_bytes(0, 0) == 0
-    assert L.ds4g_permute_workspace_bytes(2048, 6, 256) == 256 * 12 * 4
+    # per-expert counts of each 256-slot chunk: E * ceil(T*k / 256) int32
+    assert L.ds4g_permute_workspace_bytes(2048, 6, 256) == 256 * 48 * 4
+    # dispatch: the permutation's counts (16-byte rounded), plus the NVFP4 amax word without g_in
+    assert L.ds4g_dispatch_workspace_bytes(2048, 6, 256, 0, 0) == 256 * 48 * 4
+    assert L.ds4g_dispatch_workspace_bytes(2048, 6, 256, 1, 0) == 256 * 48 * 4 + 16
+    assert L.ds4g_dispatch_workspace_bytes(2048, 6, 256, 1, 1) == 256 * 48 * 4
     assert L.ds4g_permute_static_max_bytes() == 256 * 1024
 
 
