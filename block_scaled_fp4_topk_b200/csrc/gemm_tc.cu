@@ -30,6 +30,7 @@
 // the device error word and the CTA winds down.
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <stdlib.h>
 
 #include "common.cuh"
 #include "kernels.cuh"
@@ -54,13 +55,21 @@ constexpr unsigned long long kWaitNs = 4000000000ull;
 // multiple of 224, e.g. FC2 with N = 7168) with two, so that the epilogue of
 // one tile overlaps the MMAs of the next: 2 x 224 accumulator columns plus
 // the scale columns fit the 512 TMEM columns, 2 x 256 do not.
-template <int FMT, int TBN, int NISS>
+// CTAS: 1 = one CTA per tile (M = 128); 2 = a CTA pair per tile
+// (tcgen05 cta_group::2, M = 256): each CTA of the pair loads its own 128
+// activation rows and half of the TBN weight rows, the pair's MMA reads both
+// halves, and each CTA's tensor memory receives its own 128 rows x TBN
+// columns.  Per unit of MMA work a CTA then moves half the weight bytes
+// through its shared memory.
+template <int FMT, int TBN, int NISS, int CTAS = 1>
 struct Cfg {
     static_assert(TBN == 256 || TBN == 224 || TBN == 192, "tile width");
     static_assert(NISS == 1 || (NISS == 2 && TBN < 256), "two issuers need two accumulators");
+    static_assert(CTAS == 1 || CTAS == 2, "one CTA or a CTA pair per tile");
     static constexpr int NACC = (TBN == 256) ? 1 : 2;               // accumulator buffers
     static constexpr int HALF = TBN / 2;                             // weight rows per TMA box
-    static constexpr int B_BYTES = TBN * BKB;
+    static constexpr int BMT = BM * CTAS;                            // activation rows per tile
+    static constexpr int B_BYTES = (CTAS == 1 ? TBN : HALF) * BKB;   // weight bytes per stage in this CTA
     static constexpr int WPS = (FMT == DS4G_MXFP4) ? 2 : 4;         // 4-scale words per row per K stage
     // TMEM scale columns per issuer: A (4 per word) then W (8 per word)
     static constexpr int SF_COLS = 12 * WPS;
@@ -71,7 +80,6 @@ struct Cfg {
     static constexpr int SF_ROW = 2 * WPS * 4;                       // scale bytes per row per scale stage
     static constexpr int SFA_BYTES = BM * SF_ROW;                    // one scale stage of A
     static constexpr int SFB_BYTES = 256 * SF_ROW;                   // one scale stage of W (two 128-row groups)
-    static constexpr int DATA_BYTES = STAGES * (A_BYTES + B_BYTES);
     static constexpr int SF_BYTES = SF_STAGES * (SFA_BYTES + SFB_BYTES);
     // 224-column tiles with one MMA issuer stage their fp32 epilogue through
     // shared memory, 16 rows x 32 columns per warp (rows padded to 33
@@ -80,11 +88,20 @@ struct Cfg {
     // shared-memory bandwidth and the staging traffic slows it more than the
     // wider reductions gain (measured: FC2 0.389 -> 0.448 ms at T = 2048), so
     // that configuration stores straight from registers.
-    static constexpr bool STAGED = (TBN == 224 && NISS == 1);
-    static constexpr int STAGE_OFF = DATA_BYTES + SF_BYTES + 256 + ((kMaxE + 1) * 4 + 15) / 16 * 16;
+    static constexpr bool STAGED = (TBN == 224 && NISS == 1 && CTAS == 1);
+    static constexpr int BAR_BYTES = (CTAS == 1) ? 256 : 512;        // barriers + TMEM slot + flags
+    static constexpr int PREFIX_BYTES = ((kMaxE + 1) * 4 + 15) / 16 * 16;
     static constexpr int STAGE_BYTES = STAGED ? kEpiWarps * 16 * 33 * 4 : 0;
+    // data ring: 4 stages with one CTA per tile; a pair's stages are smaller,
+    // so as many as fit (at most 8)
+    static constexpr int PAIR_STAGES =
+        (232448 - 1024 - SF_BYTES - BAR_BYTES - PREFIX_BYTES - STAGE_BYTES) / (A_BYTES + B_BYTES);
+    static constexpr int NST = (CTAS == 1) ? STAGES : (PAIR_STAGES > 8 ? 8 : PAIR_STAGES);
+    static constexpr int DATA_BYTES = NST * (A_BYTES + B_BYTES);
+    static constexpr int STAGE_OFF = DATA_BYTES + SF_BYTES + BAR_BYTES + PREFIX_BYTES;
     static constexpr size_t SMEM = 1024 + (size_t)STAGE_OFF + STAGE_BYTES;
     static_assert(SMEM <= 232448, "shared memory per CTA");
+    static_assert((2 * NST + 3 * SF_STAGES + 4) * 8 + 16 <= BAR_BYTES, "barrier block");
 };
 
 // ---- PTX wrappers ----------------------------------------------------------
@@ -157,6 +174,55 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
         : "memory");
 }
 
+// ---- CTA-pair (cluster of two) wrappers
+__device__ __forceinline__ uint32_t cluster_ctarank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t cluster_id_x()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t nclusters_x()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+    return r;
+}
+// all threads of both CTAs of the cluster
+__device__ __forceinline__ void cluster_sync_all()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// shared::cluster address of the object at shared::cta address `a` in CTA `rank`
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t a, uint32_t rank)
+{
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
+    return r;
+}
+// arrive on an mbarrier of either CTA of the cluster.  Default (CTA-scope)
+// release: a cluster-scope release made the leader see each arrival about
+// 2,000 cycles late (measured), stalling the MMA issuer at every scale stage.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr)
+{
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+// tile load into this CTA's shared memory whose completion is counted on an
+// mbarrier of the pair's leader CTA
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, uint32_t mbar_cluster, int x,
+                                                 int y)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
+        ::"r"(dst), "l"((uint64_t)map), "r"(mbar_cluster), "r"(x), "r"(y)
+        : "memory");
+}
+
 // shared-memory matrix descriptor (tcgen05): K-major, 128-byte swizzle,
 // 8-row core groups 1024 bytes apart
 __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr)
@@ -181,42 +247,70 @@ __device__ __forceinline__ uint64_t desc_sf(uint32_t saddr)
 }
 
 // instruction descriptor: E2M1 x E2M1, fp32 accumulate, K-major A and B,
-// N = TBN, M = 128; scale format UE8M0 (MX) or UE4M3 (NV)
-template <int FMT, int TBN>
+// N = TBN, M = 128 (one CTA) or 256 (a CTA pair); scale format UE8M0 (MX) or
+// UE4M3 (NV)
+template <int FMT, int TBN, int CTAS = 1>
 __device__ __forceinline__ uint32_t idesc_base()
 {
     return (1u << 7) | (1u << 10) | ((uint32_t)(TBN >> 3) << 17) | ((FMT == DS4G_MXFP4 ? 1u : 0u) << 23) |
-           ((uint32_t)(BM >> 4) << 24);
+           ((uint32_t)((BM * CTAS) >> 4) << 24);
 }
 
-template <int FMT>
+template <int FMT, int CTAS = 1>
 __device__ __forceinline__ void mma(uint32_t d_tmem, uint64_t ad, uint64_t bd, uint32_t idesc, uint32_t acc,
                                     uint32_t sfa, uint32_t sfb)
 {
-    if (FMT == DS4G_MXFP4) {
+    if (FMT == DS4G_MXFP4 && CTAS == 1) {
         asm volatile(
             "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
             "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
             ::"r"(d_tmem), "l"(ad), "l"(bd), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb)
             : "memory");
-    } else {
+    } else if (FMT == DS4G_MXFP4) {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+            ::"r"(d_tmem), "l"(ad), "l"(bd), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb)
+            : "memory");
+    } else if (CTAS == 1) {
         asm volatile(
             "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
             "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
             ::"r"(d_tmem), "l"(ad), "l"(bd), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb)
             : "memory");
+    } else {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+            ::"r"(d_tmem), "l"(ad), "l"(bd), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb)
+            : "memory");
     }
 }
 
+// shared -> tensor memory copy of one 32 x 16-byte scale chunk into all four
+// lane quarters; with a CTA pair each CTA copies its own chunk into its own
+// tensor memory
+template <int CTAS = 1>
 __device__ __forceinline__ void utccp(uint32_t taddr, uint64_t sdesc)
 {
-    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+    if (CTAS == 1)
+        asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+    else
+        asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
+// arrive on `mbar` once the thread's earlier tensor-core operations are done;
+// with a CTA pair on the mbarrier at the same offset in both CTAs
+template <int CTAS = 1>
 __device__ __forceinline__ void tc_commit(uint32_t mbar)
 {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(mbar)
-                 : "memory");
+    if (CTAS == 1)
+        asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(mbar)
+                     : "memory");
+    else
+        asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+                     ::"r"(mbar), "h"((uint16_t)3)
+                     : "memory");
 }
 
 // 16 TMEM lanes x 16 columns: thread t gets lanes t/4 and t/4 + 8, columns
@@ -300,6 +394,7 @@ struct Tile {
     int64_t end;  // end of the expert's segment
 };
 
+template <int BMT = BM>
 __device__ __forceinline__ Tile tile_of(int64_t t, const int32_t* prefix, const int32_t* offsets, int E,
                                         int n_tiles)
 {
@@ -312,10 +407,10 @@ __device__ __forceinline__ Tile tile_of(int64_t t, const int32_t* prefix, const 
     r.e = lo;
     const int64_t beg = offsets[lo];
     r.end = offsets[lo + 1];
-    const int64_t mt_cnt = ceil_div(r.end - beg, BM);
+    const int64_t mt_cnt = ceil_div(r.end - beg, BMT);
     const int64_t local = t - prefix[lo];
     r.nt = (int)(local / mt_cnt);
-    r.m0 = beg + (local % mt_cnt) * BM;
+    r.m0 = beg + (local % mt_cnt) * BMT;
     return r;
 }
 
@@ -333,12 +428,14 @@ __device__ __forceinline__ void w_rows(const Tile& tl, int N, int I, int64_t& y0
     }
 }
 
-template <int FMT, int EPI, int TBN, int NISS>
+template <int FMT, int EPI, int TBN, int NISS, int CTAS>
 __global__ void __launch_bounds__(kThreads, 1)
 k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
           const __grid_constant__ CUtensorMap map_sfa, const __grid_constant__ CUtensorMap map_sfb, const GemmArgs p)
 {
-    using C = Cfg<FMT, TBN, NISS>;
+    using C = Cfg<FMT, TBN, NISS, CTAS>;
+    constexpr bool PAIR = (CTAS == 2);
+    constexpr int STAGES = C::NST;
     constexpr int SF_STAGES = C::SF_STAGES;
     static_assert(EPI != DS4G_EPI_SWIGLU_REQUANT || TBN == 256 || TBN == 192,
                   "SwiGLU tiles pair TBN/2 gate and TBN/2 up rows, a multiple of 32 each");
@@ -361,7 +458,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tmem_empty + 2);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int32_t* total_tiles = reinterpret_cast<int32_t*>(tmem_slot + 2);
-    int32_t* prefix = reinterpret_cast<int32_t*>(smem + C::DATA_BYTES + C::SF_BYTES + 256);
+    int32_t* prefix = reinterpret_cast<int32_t*>(smem + C::DATA_BYTES + C::SF_BYTES + C::BAR_BYTES);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int E = p.E;
@@ -372,6 +469,11 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
     // SwiGLU: the last tile may be ragged (I % (TBN/2) != 0); its columns past
     // I are computed from other rows and never stored
     const int n_tiles = (EPI == DS4G_EPI_SWIGLU_REQUANT) ? (int)ceil_div(I, TBN / 2) : (int)ceil_div(p.N, TBN);
+    // A CTA pair walks the tiles of its cluster; rank 0 (the leader) issues
+    // the pair's MMAs, rank 1 only loads its halves and drains its rows.
+    const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+    const int64_t tile0 = PAIR ? (int64_t)cluster_id_x() : (int64_t)blockIdx.x;
+    const int64_t tstride = PAIR ? (int64_t)nclusters_x() : (int64_t)gridDim.x;
 
     // ---- prologue
     if (threadIdx.x == 0) {
@@ -381,12 +483,13 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
         }
         for (int r = 0; r < SF_STAGES; ++r) {
             mbar_init(smem_u32(&sf_full[r]), 1);
-            mbar_init(smem_u32(&sf_ready[r]), 1);
+            mbar_init(smem_u32(&sf_ready[r]), PAIR ? 2 : 1);     // pair: both CTAs' transposers
             mbar_init(smem_u32(&sf_empty[r]), 1);
         }
         for (int b2 = 0; b2 < NACC; ++b2) {
             mbar_init(smem_u32(&tmem_full[b2]), 1);
-            mbar_init(smem_u32(&tmem_empty[b2]), 32 * kEpiWarps);
+            // pair: one arrival per epilogue warp of either CTA
+            mbar_init(smem_u32(&tmem_empty[b2]), PAIR ? 2 * kEpiWarps : 32 * kEpiWarps);
         }
         *abort_flag = 0;
         fence_barrier_init();
@@ -397,7 +500,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
         int32_t sum = 0;
         for (int i = 0; i < per; ++i) {
             const int e = lane * per + i;
-            if (e < E) sum += (int32_t)(ceil_div((int64_t)p.offsets[e + 1] - p.offsets[e], BM) * n_tiles);
+            if (e < E) sum += (int32_t)(ceil_div((int64_t)p.offsets[e + 1] - p.offsets[e], C::BMT) * n_tiles);
         }
         int32_t incl = sum;
 #pragma unroll
@@ -410,7 +513,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
             const int e = lane * per + i;
             if (e < E) {
                 prefix[e] = run;
-                run += (int32_t)(ceil_div((int64_t)p.offsets[e + 1] - p.offsets[e], BM) * n_tiles);
+                run += (int32_t)(ceil_div((int64_t)p.offsets[e + 1] - p.offsets[e], C::BMT) * n_tiles);
             }
         }
         if (lane == 31) {
@@ -430,13 +533,22 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
         }
     }
     if (warp == 3) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                     "r"(kTmemCols)
-                     : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        if (PAIR) {
+            // both CTAs' warp 3 allocate together: the same columns in each
+            asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                         "r"(kTmemCols)
+                         : "memory");
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+        } else {
+            asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                         "r"(kTmemCols)
+                         : "memory");
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        }
     }
     tc_fence_before();
-    __syncthreads();
+    // a pair: the peer's barriers must be initialised before anything arrives on them
+    if (PAIR) cluster_sync_all(); else __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const int64_t ntiles = *total_tiles;
@@ -446,19 +558,23 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
         // This CTA's tiles in groups of NISS consecutive ones; the stages of a
         // group are interleaved (K stage by K stage, member by member) so that
         // each MMA issuer finds its next stage while the other works.
+        // A pair: each CTA loads its own 128 activation rows and its half of
+        // the weight rows, counted on the leader's `full` barrier (the leader
+        // expects both CTAs' bytes); the scales of its own activation rows and
+        // of all TBN weight rows go to its own shared memory.
         if (lane == 0) {
             uint32_t it = 0, sit = 0;
             bool ok = true;
             for (int64_t j0 = 0; ok; j0 += NISS) {
-                const int64_t t0 = blockIdx.x + j0 * gridDim.x;
+                const int64_t t0 = tile0 + j0 * tstride;
                 if (t0 >= ntiles) break;
-                const int gsz = (NISS == 2 && t0 + gridDim.x < ntiles) ? 2 : 1;
+                const int gsz = (NISS == 2 && t0 + tstride < ntiles) ? 2 : 1;
                 Tile tls[NISS];
                 int64_t y0s[NISS], y1s[NISS];
 #pragma unroll
                 for (int u = 0; u < NISS; ++u) {
                     if (u < gsz) {
-                        tls[u] = tile_of(t0 + u * (int64_t)gridDim.x, prefix, p.offsets, E, n_tiles);
+                        tls[u] = tile_of<C::BMT>(t0 + u * tstride, prefix, p.offsets, E, n_tiles);
                         w_rows<EPI, TBN>(tls[u], p.N, I, y0s[u], y1s[u]);
                     }
                 }
@@ -467,60 +583,90 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
                     for (int u = 0; u < NISS; ++u) {
                         if (u >= gsz || !ok) continue;
                         const Tile& tl = tls[u];
+                        const int64_t arow = tl.m0 + (int64_t)BM * rank;   // this CTA's first activation row
                         if ((ks & 1) == 0) {
                             const int r = sit % SF_STAGES;
                             if (!mbar_wait(smem_u32(&sf_empty[r]), ((sit / SF_STAGES) & 1) ^ 1, abort_flag)) { ok = false; break; }
                             const uint32_t fb = smem_u32(&sf_full[r]);
                             mbar_arrive_tx(fb, C::SFA_BYTES + TBN * C::SF_ROW);
                             const int x = (ks >> 1) * C::SF_ROW;
-                            tma_load_2d(smem_u32(sSFA + r * C::SFA_BYTES), &map_sfa, fb, x, (int)tl.m0);
+                            tma_load_2d(smem_u32(sSFA + r * C::SFA_BYTES), &map_sfa, fb, x, (int)arow);
                             tma_load_2d(smem_u32(sSFB + r * C::SFB_BYTES), &map_sfb, fb, x, (int)y0s[u]);
                             tma_load_2d(smem_u32(sSFB + r * C::SFB_BYTES + C::HALF * C::SF_ROW), &map_sfb, fb, x, (int)y1s[u]);
                             ++sit;
                         }
                         const int s = it % STAGES;
                         if (!mbar_wait(smem_u32(&empty[s]), ((it / STAGES) & 1) ^ 1, abort_flag)) { ok = false; break; }
-                        const uint32_t fb = smem_u32(&full[s]);
-                        mbar_arrive_tx(fb, A_BYTES + B_BYTES);
-                        tma_load_2d(smem_u32(sA + s * A_BYTES), &map_a, fb, ks * BKB, (int)tl.m0);
-                        tma_load_2d(smem_u32(sB + s * B_BYTES), &map_b, fb, ks * BKB, (int)y0s[u]);
-                        tma_load_2d(smem_u32(sB + s * B_BYTES + B_BYTES / 2), &map_b, fb, ks * BKB, (int)y1s[u]);
+                        if (PAIR) {
+                            // the second CTA's activation rows may lie wholly
+                            // past the expert's segment: then they are not
+                            // loaded (the MMA computes rows that are never stored)
+                            const bool peer_live = tl.m0 + BM < tl.end;
+                            const uint32_t fb = mapa_shared(smem_u32(&full[s]), 0);
+                            if (rank == 0)
+                                mbar_arrive_tx(smem_u32(&full[s]), (peer_live ? 2 * A_BYTES : A_BYTES) + 2 * B_BYTES);
+                            if (rank == 0 || peer_live)
+                                tma_load_2d_pair(smem_u32(sA + s * A_BYTES), &map_a, fb, ks * BKB, (int)arow);
+                            tma_load_2d_pair(smem_u32(sB + s * B_BYTES), &map_b, fb, ks * BKB,
+                                             (int)(rank == 0 ? y0s[u] : y1s[u]));
+                        } else {
+                            const uint32_t fb = smem_u32(&full[s]);
+                            mbar_arrive_tx(fb, A_BYTES + B_BYTES);
+                            tma_load_2d(smem_u32(sA + s * A_BYTES), &map_a, fb, ks * BKB, (int)tl.m0);
+                            tma_load_2d(smem_u32(sB + s * B_BYTES), &map_b, fb, ks * BKB, (int)y0s[u]);
+                            tma_load_2d(smem_u32(sB + s * B_BYTES + B_BYTES / 2), &map_b, fb, ks * BKB, (int)y1s[u]);
+                        }
                         ++it;
                     }
                 }
             }
             if (!ok) {
                 // let the copies already issued land before the CTA goes away
+                // (a pair's data copies count on the leader's barriers, which
+                // only the leader can wait on)
                 volatile int never = 0;
-                for (uint32_t j = (it > STAGES ? it - STAGES : 0); j < it; ++j)
-                    mbar_wait(smem_u32(&full[j % STAGES]), (j / STAGES) & 1, &never);
+                if (!PAIR || rank == 0)
+                    for (uint32_t j = (it > STAGES ? it - STAGES : 0); j < it; ++j)
+                        mbar_wait(smem_u32(&full[j % STAGES]), (j / STAGES) & 1, &never);
                 for (uint32_t j = (sit > SF_STAGES ? sit - SF_STAGES : 0); j < sit; ++j)
                     mbar_wait(smem_u32(&sf_full[j % SF_STAGES]), (j / SF_STAGES) & 1, &never);
+            } else if (PAIR) {
+                // the leader's last commits arrive on this CTA's barriers:
+                // wait for them so that none lands after the CTA has exited
+                for (uint32_t j = (it > STAGES ? it - STAGES : 0); j < it; ++j)
+                    if (!mbar_wait(smem_u32(&empty[j % STAGES]), (j / STAGES) & 1, abort_flag)) break;
+                for (uint32_t j = (sit > SF_STAGES ? sit - SF_STAGES : 0); j < sit; ++j)
+                    if (!mbar_wait(smem_u32(&sf_empty[j % SF_STAGES]), (j / SF_STAGES) & 1, abort_flag)) break;
             }
         }
         __syncwarp();
-    } else if (warp == 1 || (NISS == 2 && warp == 3)) {
+    } else if ((warp == 1 || (NISS == 2 && warp == 3)) && rank == 0) {
         // ================= MMA issuer(s) =================
         // Issuer pi takes member pi of each tile group, accumulating into
         // accumulator pi (two issuers) with its own scale columns.  An issuing
         // thread that waits on a barrier first drains its own tensor-core
         // work; with two issuers the other one's MMAs fill that gap.
+        // A pair: only the leader issues; its scale copies, MMAs and commits
+        // act on both CTAs (each CTA's own shared and tensor memory at the
+        // same addresses, the commits arrive on both CTAs' barriers).
         if (lane == 0) {
             const int pi = (warp == 1) ? 0 : 1;
-            const uint32_t ibase = idesc_base<FMT, TBN>();
+            const uint32_t ibase = idesc_base<FMT, TBN, CTAS>();
             const uint32_t col_sfa = tmem + C::COL_SFA + pi * C::SF_COLS;
             const uint32_t col_sfb = col_sfa + 4 * C::WPS;
             uint32_t it_base = 0, sit_base = 0;
+            uint32_t uses[2] = {0, 0};
             bool ok = true;
             for (int64_t j0 = 0; ok; j0 += NISS) {
-                const int64_t t0 = blockIdx.x + j0 * gridDim.x;
+                const int64_t t0 = tile0 + j0 * tstride;
                 if (t0 >= ntiles) break;
-                const int gsz = (NISS == 2 && t0 + gridDim.x < ntiles) ? 2 : 1;
+                const int gsz = (NISS == 2 && t0 + tstride < ntiles) ? 2 : 1;
                 if (pi < gsz) {
                     const int64_t jt = j0 + pi;                        // this CTA's local tile index
                     const int buf = (NISS == 2) ? pi : (int)(jt % NACC);
                     const uint32_t use = (NISS == 2) ? (uint32_t)(j0 / 2) : (uint32_t)(jt / NACC);
                     if (!mbar_wait(smem_u32(&tmem_empty[buf]), (use & 1) ^ 1, abort_flag)) { ok = false; break; }
+                    uses[buf] = use + 1;
                     const uint32_t acc = tmem + kColAcc + buf * TBN;
                     tc_fence_after();
                     for (int ks = 0; ks < nks; ++ks) {
@@ -539,9 +685,9 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
                         const uint32_t sfb_s = smem_u32(sSFB + r * C::SFB_BYTES);
 #pragma unroll
                         for (int c = 0; c < C::WPS; ++c) {
-                            utccp(col_sfa + 4 * c, desc_sf(sfa_s + (w0 + c) * 512));
-                            utccp(col_sfb + 8 * c, desc_sf(sfb_s + ((w0 + c) * 2 + 0) * 512));
-                            utccp(col_sfb + 8 * c + 4, desc_sf(sfb_s + ((w0 + c) * 2 + 1) * 512));
+                            utccp<CTAS>(col_sfa + 4 * c, desc_sf(sfa_s + (w0 + c) * 512));
+                            utccp<CTAS>(col_sfb + 8 * c, desc_sf(sfb_s + ((w0 + c) * 2 + 0) * 512));
+                            utccp<CTAS>(col_sfb + 8 * c + 4, desc_sf(sfb_s + ((w0 + c) * 2 + 1) * 512));
                         }
                         const int64_t krem = K - (int64_t)ks * BK;
                         const int nmma = krem >= BK ? 4 : (int)(krem / 64);
@@ -553,25 +699,33 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
                                 const int c = (FMT == DS4G_MXFP4) ? (j >> 1) : j;
                                 const uint32_t sfid = (FMT == DS4G_MXFP4) ? (uint32_t)((j & 1) * 2) : 0u;
                                 const uint32_t idesc = ibase | (sfid << 4) | (sfid << 29);
-                                mma<FMT>(acc, desc_sw128(a_s + 32 * j), desc_sw128(b_s + 32 * j), idesc,
-                                         (ks > 0 || j > 0) ? 1u : 0u, col_sfa + 4 * c, col_sfb + 8 * c);
+                                mma<FMT, CTAS>(acc, desc_sw128(a_s + 32 * j), desc_sw128(b_s + 32 * j), idesc,
+                                               (ks > 0 || j > 0) ? 1u : 0u, col_sfa + 4 * c, col_sfb + 8 * c);
                             }
                         }
-                        tc_commit(smem_u32(&empty[s]));
-                        if ((ks & 1) == 1 || ks == nks - 1) tc_commit(smem_u32(&sf_empty[r]));
+                        tc_commit<CTAS>(smem_u32(&empty[s]));
+                        if ((ks & 1) == 1 || ks == nks - 1) tc_commit<CTAS>(smem_u32(&sf_empty[r]));
                     }
                     if (!ok) break;
-                    tc_commit(smem_u32(&tmem_full[buf]));
+                    tc_commit<CTAS>(smem_u32(&tmem_full[buf]));
                 }
                 it_base += (uint32_t)(nks * gsz);
                 sit_base += (uint32_t)(npairs * gsz);
+            }
+            if (PAIR && ok) {
+                // both CTAs' epilogues have released the last accumulators
+                // (their arrivals on this CTA's barriers have landed)
+                for (int b2 = 0; b2 < NACC; ++b2)
+                    if ((NISS == 1 || b2 == pi) && uses[b2] > 0)
+                        if (!mbar_wait(smem_u32(&tmem_empty[b2]), (uses[b2] & 1) ^ 1, abort_flag)) break;
             }
         }
         __syncwarp();
     } else if (warp == 2) {
         // ================= scale transposer =================
+        // (a pair: each CTA transposes its own scales and tells the leader)
         uint32_t sit = 0;
-        for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x) {
+        for (int64_t t = tile0; t < ntiles; t += tstride) {
             bool ok = true;
             for (int pr = 0; pr < npairs; ++pr, ++sit) {
                 const int r = sit % SF_STAGES;
@@ -582,7 +736,10 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
                 sf_transpose<2 * C::WPS, 2>(sSFB + r * C::SFB_BYTES, lane);
                 fence_proxy_async();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(smem_u32(&sf_ready[r]));
+                if (lane == 0) {
+                    if (PAIR) mbar_arrive_cluster(mapa_shared(smem_u32(&sf_ready[r]), 0));
+                    else mbar_arrive(smem_u32(&sf_ready[r]));
+                }
             }
             if (!ok) break;
         }
@@ -592,11 +749,15 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
         const int half = (warp - 4) >> 2;       // which half of the tile's columns
         uint32_t tcount = 0;
         const float gh = (FMT == DS4G_NVFP4 && EPI == DS4G_EPI_SWIGLU_REQUANT) ? *p.oq_g : 1.0f;
-        for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, ++tcount) {
+        for (int64_t t = tile0; t < ntiles; t += tstride, ++tcount) {
             const int buf = (int)(tcount % NACC);
-            if (!mbar_wait(smem_u32(&tmem_full[buf]), (tcount / NACC) & 1, abort_flag)) break;
+            const bool got = mbar_wait(smem_u32(&tmem_full[buf]), (tcount / NACC) & 1, abort_flag);
+            // a pair's teardown is a warp-aligned cluster barrier: the whole
+            // warp leaves the loop together
+            if (PAIR ? !__all_sync(0xffffffffu, got) : !got) break;
             tc_fence_after();
-            const Tile tl = tile_of(t, prefix, p.offsets, E, n_tiles);
+            Tile tl = tile_of<C::BMT>(t, prefix, p.offsets, E, n_tiles);
+            tl.m0 += (int64_t)BM * rank;           // a pair: this CTA's 128 rows of the tile
             const float gscale = (FMT == DS4G_NVFP4) ? __fmul_rn(p.a_g[0], p.w_g[tl.e]) : 1.0f;
             const int64_t row = tl.m0 + 32 * q + lane;
             const bool valid = row < tl.end;
@@ -762,16 +923,25 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
                 }
             }
             tc_fence_before();
-            mbar_arrive(smem_u32(&tmem_empty[buf]));
+            if (PAIR) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tmem_empty[buf]), 0));
+            } else {
+                mbar_arrive(smem_u32(&tmem_empty[buf]));
+            }
         }
     }
 
-    // ---- teardown
+    // ---- teardown (a pair: neither CTA leaves while the other may still
+    // touch its shared or tensor memory)
     tc_fence_before();
-    __syncthreads();
+    if (PAIR) cluster_sync_all(); else __syncthreads();
     tc_fence_after();
     if (warp == 3) {
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+        if (PAIR)
+            asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+        else
+            asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
     }
 }
 
@@ -811,10 +981,10 @@ static bool make_map(CUtensorMap* m, const uint8_t* base, int64_t rows, int64_t 
     return r == CUDA_SUCCESS;
 }
 
-template <int FMT, int EPI, int TBN, int NISS>
+template <int FMT, int EPI, int TBN, int NISS, int CTAS = 1>
 static cudaError_t run_tc(const GemmArgs& a, cudaStream_t st)
 {
-    using C = tc::Cfg<FMT, TBN, NISS>;
+    using C = tc::Cfg<FMT, TBN, NISS, CTAS>;
     const int blk = (FMT == DS4G_MXFP4) ? 32 : 16;
     CUtensorMap ma, mb, msa, msb;
     if (!make_map(&ma, a.a_data, a.S, a.K / 2, 128, 128, true) ||
@@ -822,13 +992,38 @@ static cudaError_t run_tc(const GemmArgs& a, cudaStream_t st)
         !make_map(&msa, a.a_scales, a.S, a.K / blk, C::SF_ROW, 128, false) ||
         !make_map(&msb, a.w_scales, (int64_t)a.E * a.N, a.K / blk, C::SF_ROW, C::HALF, false))
         return cudaErrorInvalidValue;
-    auto kern = tc::k_gemm_tc<FMT, EPI, TBN, NISS>;
+    auto kern = tc::k_gemm_tc<FMT, EPI, TBN, NISS, CTAS>;
     const size_t shm = C::SMEM;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)shm);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = kNumSMs;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    kern<<<sms, tc::kThreads, shm, st>>>(ma, mb, msa, msb, a);
+    if (CTAS == 1) {
+        kern<<<sms, tc::kThreads, shm, st>>>(ma, mb, msa, msb, a);
+        return cudaGetLastError();
+    }
+    // CTA pairs: clusters of two, as many as can be resident at once (the
+    // grid is persistent, so a cluster that had to wait for another to finish
+    // would double the time)
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3((unsigned)(sms & ~1));
+    cfg.blockDim = dim3(tc::kThreads);
+    cfg.dynamicSmemBytes = shm;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int nclusters = 0;
+    e = cudaOccupancyMaxActiveClusters(&nclusters, kern, &cfg);
+    if (e != cudaSuccess) return e;
+    if (nclusters < 1) return cudaErrorInvalidConfiguration;
+    cfg.gridDim = dim3((unsigned)(2 * (nclusters < sms / 2 ? nclusters : sms / 2)));
+    e = cudaLaunchKernelEx(&cfg, kern, ma, mb, msa, msb, a);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
@@ -839,11 +1034,20 @@ static cudaError_t run_tc(const GemmArgs& a, cudaStream_t st)
 // at T = 16384 2.48 ms against 1.92 ms.)  Other N: 256-column tiles, one
 // accumulator.
 template <int FMT, int EPI>
-static cudaError_t run_tc_plain(const GemmArgs& a, cudaStream_t st)
+static cudaError_t run_tc_plain(const GemmArgs& a, cudaStream_t st, bool pair)
 {
-    if (a.N % 224 != 0) return run_tc<FMT, EPI, 256, 1>(a, st);
-    if constexpr (FMT == DS4G_MXFP4) return run_tc<FMT, EPI, 224, 2>(a, st);
-    else return run_tc<FMT, EPI, 224, 1>(a, st);
+    if (a.N % 224 != 0) return pair ? run_tc<FMT, EPI, 256, 1, 2>(a, st) : run_tc<FMT, EPI, 256, 1>(a, st);
+    if constexpr (FMT == DS4G_MXFP4)
+        return pair ? run_tc<FMT, EPI, 224, 2, 2>(a, st) : run_tc<FMT, EPI, 224, 2>(a, st);
+    else
+        return pair ? run_tc<FMT, EPI, 224, 1, 2>(a, st) : run_tc<FMT, EPI, 224, 1>(a, st);
+}
+
+template <int FMT>
+static cudaError_t run_tc_swiglu(const GemmArgs& a, cudaStream_t st, bool pair)
+{
+    return pair ? run_tc<FMT, DS4G_EPI_SWIGLU_REQUANT, 192, 2, 2>(a, st)
+                : run_tc<FMT, DS4G_EPI_SWIGLU_REQUANT, 192, 2>(a, st);
 }
 
 bool gemm_tc_supports(int fmt, int64_t K)
@@ -853,17 +1057,33 @@ bool gemm_tc_supports(int fmt, int64_t K)
     return fmt == DS4G_MXFP4 ? (K % 512 == 0) : (K % 256 == 0);
 }
 
+// One CTA per 128-row tile (default), or CTA pairs per 256-row tile (tcgen05
+// cta_group::2) when DS4G_TC_PAIR=1 is set in the environment.  Pairs halve
+// the MMA instructions and the weight bytes per SM of a tile, but each SM
+// still runs all of its scale-factor copies, and the tensor pipe executes
+// copies and MMAs one after another (about 60 cycles per copy, N/2 per MMA):
+// per SM a K stage costs the same in both modes, and 256-row tiles waste
+// more rows on short expert segments.  Measured on the prefill layers, FC1
+// T = 2048 MXFP4 0.516 ms (one CTA) vs 0.698 ms (pairs), T = 16384 NVFP4
+// 2.44 vs 2.64 ms; FC2 + combine 0.377 vs 0.520 ms and 1.94 vs 2.14 ms.
+static bool use_pairs(const GemmArgs&)
+{
+    const char* env = getenv("DS4G_TC_PAIR");
+    return env && env[0] == '1';
+}
+
 cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st)
 {
     if (a.S == 0) return cudaSuccess;
     if (a.E > tc::kMaxE || !gemm_tc_supports(a.fmt, a.K)) return cudaErrorInvalidValue;
+    const bool pair = use_pairs(a);
     if (a.fmt == DS4G_MXFP4)
-        return a.epilogue == DS4G_EPI_NONE ? run_tc_plain<DS4G_MXFP4, DS4G_EPI_NONE>(a, st)
-             : a.epilogue == kEpiCombine   ? run_tc_plain<DS4G_MXFP4, kEpiCombine>(a, st)
-                                           : run_tc<DS4G_MXFP4, DS4G_EPI_SWIGLU_REQUANT, 192, 2>(a, st);
-    return a.epilogue == DS4G_EPI_NONE ? run_tc_plain<DS4G_NVFP4, DS4G_EPI_NONE>(a, st)
-         : a.epilogue == kEpiCombine   ? run_tc_plain<DS4G_NVFP4, kEpiCombine>(a, st)
-                                       : run_tc<DS4G_NVFP4, DS4G_EPI_SWIGLU_REQUANT, 192, 2>(a, st);
+        return a.epilogue == DS4G_EPI_NONE ? run_tc_plain<DS4G_MXFP4, DS4G_EPI_NONE>(a, st, pair)
+             : a.epilogue == kEpiCombine   ? run_tc_plain<DS4G_MXFP4, kEpiCombine>(a, st, pair)
+                                           : run_tc_swiglu<DS4G_MXFP4>(a, st, pair);
+    return a.epilogue == DS4G_EPI_NONE ? run_tc_plain<DS4G_NVFP4, DS4G_EPI_NONE>(a, st, pair)
+         : a.epilogue == kEpiCombine   ? run_tc_plain<DS4G_NVFP4, kEpiCombine>(a, st, pair)
+                                       : run_tc_swiglu<DS4G_NVFP4>(a, st, pair);
 }
 
 }  // namespace ds4g

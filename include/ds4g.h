@@ -180,9 +180,15 @@ ds4g_status ds4g_moe_dispatch(const float* logits, const void* x, int dtype, int
  *     weights as the MMA's M side (decode);
  *   > 16 rows and the same K rule, N % 224 == 0 (NONE): tensor-core kernel
  *     with 128-row x 224-column tiles and two accumulators (the epilogue of
- *     one tile overlaps the next tile's MMAs); else N % 256 == 0 (NONE) or
- *     I % 128 == 0 (SWIGLU_REQUANT): 128-row x 256-column tiles;
+ *     one tile overlaps the next tile's MMAs); else N % 256 == 0 (NONE):
+ *     128-row x 256-column tiles; SWIGLU_REQUANT with I % 32 == 0: 128-row
+ *     tiles of 96 gate + 96 up columns (the last one ragged), two
+ *     accumulators;
  *   otherwise: a dp4a weight-streaming kernel (any segment length).
+ *   With DS4G_TC_PAIR=1 in the environment the > 16-row tensor-core kernel
+ *   runs on CTA pairs (tcgen05 cta_group::2, 256-row tiles, each CTA loading
+ *   its own 128 rows and half of the weight rows); same results within the
+ *   GEMM bound, slower on the layer shapes measured, so off by default.
  * Shapes: K % 64 == 0; NONE needs N % 64 == 0 unless a tensor-core kernel
  *   takes the call; SWIGLU_REQUANT needs I % 32 == 0.  offsets[E] must
  *   equal S. */

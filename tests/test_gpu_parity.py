@@ -231,9 +231,22 @@ TC_CASES = [([300, 0, 1, 129, 77], 512, 512), ([256, 128], 256, 1024), ([9, 200,
             ([300, 0, 1, 129, 77], 448, 512), ([130, 20], 224, 2048), ([17, 600], 672, 1024)]
 
 
+# the prefill tensor-core kernel runs with one CTA per 128-row tile
+# (DS4G_TC_PAIR=0) or with CTA pairs per 256-row tile (DS4G_TC_PAIR=1,
+# tcgen05 cta_group::2); both are checked on every tensor-core case
+PAIR_MODES = ["0", "1"]
+
+
+@pytest.fixture
+def tc_mode(request, monkeypatch):
+    monkeypatch.setenv("DS4G_TC_PAIR", request.param)
+    return request.param
+
+
 @pytest.mark.parametrize("fmt", [MX, NV])
-@pytest.mark.parametrize("case", GEMV_CASES + TC_CASES)
-def test_grouped_gemm_plain(fmt, case):
+@pytest.mark.parametrize("case,tc_mode", [(c, "0") for c in GEMV_CASES] +
+                         [(c, m) for c in TC_CASES for m in PAIR_MODES], indirect=["tc_mode"])
+def test_grouped_gemm_plain(fmt, case, tc_mode):
     seg, N, K = case
     offsets, a, w, gw = _grouped_problem(seg, N, K, fmt)
     max_rows = max(seg)
@@ -261,8 +274,9 @@ def _h_bound(y1_ref, ab1, I):
 @pytest.mark.parametrize("case", [([3, 0, 1, 8, 5], 256, 7168), ([300, 0, 1, 129, 77], 256, 512),
                                   ([2, 1], 64, 256), ([131], 128, 2048), ([20, 0, 150], 128, 768),
                                   ([200, 9], 384, 1024), ([100, 30], 96, 1024), ([5, 16, 2], 192, 1024),
-                                  ([140, 60], 160, 512)])
-def test_fc1_fused_swiglu_requant(fmt, case):
+                                  ([140, 60], 160, 512), ([700, 3, 260], 2048, 1024)])
+@pytest.mark.parametrize("tc_mode", PAIR_MODES, indirect=True)
+def test_fc1_fused_swiglu_requant(fmt, case, tc_mode):
     seg, I, K = case
     offsets, a, w, gw = _grouped_problem(seg, 2 * I, K, fmt, stream=21)
     S = int(offsets[-1])
@@ -304,7 +318,8 @@ def test_swiglu_requant(fmt):
                                        (300, 6, 16, 448, 1024),    # tensor-core kernel, 224-column tiles
                                        (3, 6, 64, 256, 1024),      # decode tensor-core kernel
                                        (4, 2, 8, 128, 256)])       # dp4a kernel (MX) / decode tc (NV)
-def test_fc2_combine_fused(fmt, T, k, E, N, K):
+@pytest.mark.parametrize("tc_mode", PAIR_MODES, indirect=True)
+def test_fc2_combine_fused(fmt, T, k, E, N, K, tc_mode):
     lg = synth.logits(T, E, 0, 1.5)
     idx, w = oracle.route_topk(lg, k)
     offsets, r2s, s2r = oracle.moe_permute(idx, E)
