@@ -178,7 +178,7 @@ static ds4g_status grouped_gemm(const ds4g_fp4* a, const int32_t* offsets, int E
     const bool swiglu = epilogue == DS4G_EPI_SWIGLU_REQUANT;
     const bool tc_shape = gemm_tc_supports(fmt, K) &&
                           (!swiglu ? (N % 256 == 0 || N % 224 == 0) : (N % 2 == 0 && (N / 2) % 32 == 0));
-    const bool dtc = max_rows_per_expert <= 16 && gemv_tc_supports(fmt, K, N, epilogue);
+    const bool dtc = max_rows_per_expert <= 16 && gemv_tc_supports(fmt, K, N, epilogue, E);
     const bool gemv = !dtc && (max_rows_per_expert <= 8 || !tc_shape);
     const int64_t Sr = a->rows;
     if (!swiglu) {

@@ -95,10 +95,11 @@ struct Cfg {
     // data ring: 4 stages with one CTA per tile; a pair's stages are smaller,
     // so as many as fit (at most 8)
     static constexpr int PAIR_STAGES =
-        (232448 - 1024 - SF_BYTES - BAR_BYTES - PREFIX_BYTES - STAGE_BYTES) / (A_BYTES + B_BYTES);
+        (232448 - 1024 - SF_BYTES - BAR_BYTES - 2 * PREFIX_BYTES - STAGE_BYTES) / (A_BYTES + B_BYTES);
     static constexpr int NST = (CTAS == 1) ? STAGES : (PAIR_STAGES > 8 ? 8 : PAIR_STAGES);
     static constexpr int DATA_BYTES = NST * (A_BYTES + B_BYTES);
-    static constexpr int STAGE_OFF = DATA_BYTES + SF_BYTES + BAR_BYTES + PREFIX_BYTES;
+    // tile prefix, then the expert offsets staged once ([E + 1] int32 each)
+    static constexpr int STAGE_OFF = DATA_BYTES + SF_BYTES + BAR_BYTES + 2 * PREFIX_BYTES;
     static constexpr size_t SMEM = 1024 + (size_t)STAGE_OFF + STAGE_BYTES;
     static_assert(SMEM <= 232448, "shared memory per CTA");
     static_assert((2 * NST + 3 * SF_STAGES + 4) * 8 + 16 <= BAR_BYTES, "barrier block");
@@ -459,6 +460,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int32_t* total_tiles = reinterpret_cast<int32_t*>(tmem_slot + 2);
     int32_t* prefix = reinterpret_cast<int32_t*>(smem + C::DATA_BYTES + C::SF_BYTES + C::BAR_BYTES);
+    int32_t* soff = prefix + C::PREFIX_BYTES / 4;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int E = p.E;
@@ -494,43 +496,14 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
         *abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == 0) {
-        // tiles per expert, exclusive scan by one warp
-        const int per = (E + 31) / 32;
-        int32_t sum = 0;
-        for (int i = 0; i < per; ++i) {
-            const int e = lane * per + i;
-            if (e < E) sum += (int32_t)(ceil_div((int64_t)p.offsets[e + 1] - p.offsets[e], C::BMT) * n_tiles);
-        }
-        int32_t incl = sum;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            int32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += y;
-        }
-        int32_t run = incl - sum;
-        for (int i = 0; i < per; ++i) {
-            const int e = lane * per + i;
-            if (e < E) {
-                prefix[e] = run;
-                run += (int32_t)(ceil_div((int64_t)p.offsets[e + 1] - p.offsets[e], C::BMT) * n_tiles);
-            }
-        }
-        if (lane == 31) {
-            prefix[E] = incl;
-            int32_t tot = incl;
-            if ((int64_t)p.offsets[E] > p.S) {   // inconsistent offsets: do nothing
-                raise_error(kErrBadOffsets);
-                tot = 0;
-            }
-            *total_tiles = tot;
-        }
-        if (lane == 0) {
-            asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&map_a) : "memory");
-            asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&map_b) : "memory");
-            asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&map_sfa) : "memory");
-            asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&map_sfb) : "memory");
-        }
+    // the expert offsets -> shared memory in one parallel pass (a loop of
+    // dependent global loads here cost about 2 us per launch)
+    for (int e = threadIdx.x; e <= E; e += kThreads) soff[e] = p.offsets[e];
+    if (warp == 0 && lane == 0) {
+        asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&map_a) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&map_b) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&map_sfa) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&map_sfb) : "memory");
     }
     if (warp == 3) {
         if (PAIR) {
@@ -544,6 +517,39 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
                          "r"(kTmemCols)
                          : "memory");
             asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        }
+    }
+    __syncthreads();
+    if (warp == 0) {
+        // tiles per expert, exclusive scan by one warp
+        const int per = (E + 31) / 32;
+        int32_t sum = 0;
+        for (int i = 0; i < per; ++i) {
+            const int e = lane * per + i;
+            if (e < E) sum += (int32_t)(ceil_div((int64_t)soff[e + 1] - soff[e], C::BMT) * n_tiles);
+        }
+        int32_t incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            int32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        int32_t run = incl - sum;
+        for (int i = 0; i < per; ++i) {
+            const int e = lane * per + i;
+            if (e < E) {
+                prefix[e] = run;
+                run += (int32_t)(ceil_div((int64_t)soff[e + 1] - soff[e], C::BMT) * n_tiles);
+            }
+        }
+        if (lane == 31) {
+            prefix[E] = incl;
+            int32_t tot = incl;
+            if ((int64_t)soff[E] > p.S) {   // inconsistent offsets: do nothing
+                raise_error(kErrBadOffsets);
+                tot = 0;
+            }
+            *total_tiles = tot;
         }
     }
     tc_fence_before();
@@ -574,7 +580,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
 #pragma unroll
                 for (int u = 0; u < NISS; ++u) {
                     if (u < gsz) {
-                        tls[u] = tile_of<C::BMT>(t0 + u * tstride, prefix, p.offsets, E, n_tiles);
+                        tls[u] = tile_of<C::BMT>(t0 + u * tstride, prefix, soff, E, n_tiles);
                         w_rows<EPI, TBN>(tls[u], p.N, I, y0s[u], y1s[u]);
                     }
                 }
@@ -756,7 +762,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
             // warp leaves the loop together
             if (PAIR ? !__all_sync(0xffffffffu, got) : !got) break;
             tc_fence_after();
-            Tile tl = tile_of<C::BMT>(t, prefix, p.offsets, E, n_tiles);
+            Tile tl = tile_of<C::BMT>(t, prefix, soff, E, n_tiles);
             tl.m0 += (int64_t)BM * rank;           // a pair: this CTA's 128 rows of the tile
             const float gscale = (FMT == DS4G_NVFP4) ? __fmul_rn(p.a_g[0], p.w_g[tl.e]) : 1.0f;
             const int64_t row = tl.m0 + 32 * q + lane;

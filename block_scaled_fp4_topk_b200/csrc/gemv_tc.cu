@@ -48,7 +48,7 @@ constexpr int X_BYTES = BNT * BKB;   // 2 KB
 constexpr int kTmemCols = 128;
 constexpr int kColAcc = 0;         // [issuer][buffer] 16-column accumulators: 64 columns
 constexpr int kColSF = 64;         // [issuer] 16 weight-scale then 16 activation-scale columns
-constexpr int kMaxE = 1024;
+constexpr int kMaxE = 512;        // experts whose offsets and item counts fit in shared memory
 
 template <int FMT>
 struct Cfg {
@@ -63,7 +63,9 @@ struct Cfg {
     static constexpr int SFXC_BYTES = 2 * WPS * 512;            // activations, chunk order
     static constexpr int DATA_BYTES = STAGES * (W_BYTES + X_BYTES);
     static constexpr int SF_BYTES = SF_STAGES * (SFW_BYTES + SFXR_BYTES + SFXC_BYTES);
-    static constexpr size_t SMEM = 1024 + (size_t)DATA_BYTES + SF_BYTES + 512 + 64 * 16 * 4 + (kMaxE + 1) * 4;
+    static constexpr int EARR_BYTES = ((kMaxE + 1) * 4 + 15) / 16 * 16;   // one [E + 1] int32 array
+    // data, scales, barriers, the SwiGLU exchange, item prefix and offsets
+    static constexpr size_t SMEM = 1024 + (size_t)DATA_BYTES + SF_BYTES + 512 + 64 * 16 * 4 + 2 * EARR_BYTES;
     static_assert((2 * STAGES + 3 * SF_STAGES + 4) * 8 + 16 <= 512, "barrier block");
     static_assert(SMEM <= 232448, "shared memory per CTA");
 };
@@ -148,6 +150,7 @@ k_gemv_tc(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUt
     int32_t* total_items = reinterpret_cast<int32_t*>(tmem_slot + 2);
     float* xch = reinterpret_cast<float*>(smem + C::DATA_BYTES + C::SF_BYTES + 512);   // [64][16] up rows
     int32_t* prefix = reinterpret_cast<int32_t*>(xch + 64 * 16);
+    int32_t* soff = prefix + C::EARR_BYTES / 4;      // the expert offsets, staged once
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int E = p.E;
@@ -174,12 +177,29 @@ k_gemv_tc(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUt
         *abort_flag = 0;
         fence_barrier_init();
     }
+    // the expert offsets -> shared memory in one parallel pass (a loop of
+    // dependent global loads here cost about 2 us per launch)
+    for (int e = threadIdx.x; e <= E; e += kThreads) soff[e] = p.offsets[e];
+    if (warp == 0 && lane == 0) {
+        asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&map_w) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&map_x) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&map_sfw) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&map_sfx) : "memory");
+    }
+    if (warp == 3) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    __syncthreads();
     if (warp == 0) {
+        // items per expert, exclusive scan by one warp
         const int per = (E + 31) / 32;
         int32_t sum = 0;
         for (int i = 0; i < per; ++i) {
             const int e = lane * per + i;
-            if (e < E) sum += (int32_t)(ceil_div((int64_t)p.offsets[e + 1] - p.offsets[e], BNT) * wtiles);
+            if (e < E) sum += (int32_t)(ceil_div((int64_t)soff[e + 1] - soff[e], BNT) * wtiles);
         }
         int32_t incl = sum;
 #pragma unroll
@@ -192,30 +212,18 @@ k_gemv_tc(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUt
             const int e = lane * per + i;
             if (e < E) {
                 prefix[e] = run;
-                run += (int32_t)(ceil_div((int64_t)p.offsets[e + 1] - p.offsets[e], BNT) * wtiles);
+                run += (int32_t)(ceil_div((int64_t)soff[e + 1] - soff[e], BNT) * wtiles);
             }
         }
         if (lane == 31) {
             prefix[E] = incl;
             int32_t tot = incl;
-            if ((int64_t)p.offsets[E] > p.S) {
+            if ((int64_t)soff[E] > p.S) {
                 raise_error(kErrBadOffsets);
                 tot = 0;
             }
             *total_items = tot;
         }
-        if (lane == 0) {
-            asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&map_w) : "memory");
-            asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&map_x) : "memory");
-            asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&map_sfw) : "memory");
-            asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&map_sfx) : "memory");
-        }
-    }
-    if (warp == 3) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                     "r"(kTmemCols)
-                     : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     tc_fence_before();
     __syncthreads();
@@ -238,7 +246,7 @@ k_gemv_tc(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUt
             uint32_t tcount = 0, it_next = 0, sit_next = 0;
             bool ok = true;
             for (int64_t t = blockIdx.x; t < nitems && ok; t += gridDim.x, ++tcount) {
-                const Item itm = item_of(t, prefix, p.offsets, E, wtiles);
+                const Item itm = item_of(t, prefix, soff, E, wtiles);
                 int64_t y0, y1;
                 w_rows<EPI>(itm, p.N, I, y0, y1);
                 const uint32_t it0 = tcount * (uint32_t)nks, sit0 = tcount * (uint32_t)npairs;
@@ -372,7 +380,7 @@ k_gemv_tc(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUt
             const int buf = tcount & 1;
             if (!mbar_wait(smem_u32(&tmem_full[buf]), (tcount >> 1) & 1, abort_flag)) break;
             tc_fence_after();
-            const Item itm = item_of(t, prefix, p.offsets, E, wtiles);
+            const Item itm = item_of(t, prefix, soff, E, wtiles);
             const float gscale = (FMT == DS4G_NVFP4) ? __fmul_rn(p.a_g[0], p.w_g[itm.e]) : 1.0f;
             // issuer i holds the sum over the scale stages of parity i
             const uint32_t sit0 = tcount * (uint32_t)npairs;
@@ -478,16 +486,16 @@ static cudaError_t run_dtc(const GemmArgs& a, cudaStream_t st)
     return cudaGetLastError();
 }
 
-bool gemv_tc_supports(int fmt, int64_t K, int N, int epilogue)
+bool gemv_tc_supports(int fmt, int64_t K, int N, int epilogue, int E)
 {
-    if (!gemm_tc_supports(fmt, K)) return false;
+    if (E < 1 || E > dtc::kMaxE || !gemm_tc_supports(fmt, K)) return false;
     return epilogue != DS4G_EPI_SWIGLU_REQUANT ? (N % 128 == 0) : (N % 2 == 0 && (N / 2) % 64 == 0);
 }
 
 cudaError_t launch_gemv_tc(const GemmArgs& a, cudaStream_t st)
 {
     if (a.S == 0) return cudaSuccess;
-    if (a.E > dtc::kMaxE || !gemv_tc_supports(a.fmt, a.K, a.N, a.epilogue)) return cudaErrorInvalidValue;
+    if (!gemv_tc_supports(a.fmt, a.K, a.N, a.epilogue, a.E)) return cudaErrorInvalidValue;
     if (a.fmt == DS4G_MXFP4)
         return a.epilogue == DS4G_EPI_NONE ? run_dtc<DS4G_MXFP4, DS4G_EPI_NONE>(a, st)
              : a.epilogue == kEpiCombine   ? run_dtc<DS4G_MXFP4, kEpiCombine>(a, st)

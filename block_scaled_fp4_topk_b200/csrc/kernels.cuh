@@ -52,7 +52,7 @@ struct GemmArgs {
 cudaError_t launch_gemv(const GemmArgs& a, cudaStream_t st);
 bool gemm_tc_supports(int fmt, int64_t K);
 cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st);
-bool gemv_tc_supports(int fmt, int64_t K, int N, int epilogue);
+bool gemv_tc_supports(int fmt, int64_t K, int N, int epilogue, int E);
 cudaError_t launch_gemv_tc(const GemmArgs& a, cudaStream_t st);
 
 cudaError_t launch_swiglu_requant(const float* y1, int64_t rows, int I, int fmt, uint8_t* hd, uint8_t* hs,
