@@ -325,6 +325,27 @@ __device__ __forceinline__ void tmem_ld_16x256b_x2(uint32_t taddr, uint32_t* r)
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// G consecutive 16-column chunks of the same 16x256b.x2 shape, one wait for
+// all of them; the empty asm statements after the wait make every later use
+// of the registers depend on it
+template <int G>
+__device__ __forceinline__ void tmem_ld_16x256b_x2_batch(uint32_t taddr, uint32_t (&r)[G][8])
+{
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+        asm volatile("tcgen05.ld.sync.aligned.16x256b.x2.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                     : "=r"(r[g][0]), "=r"(r[g][1]), "=r"(r[g][2]), "=r"(r[g][3]), "=r"(r[g][4]), "=r"(r[g][5]),
+                       "=r"(r[g][6]), "=r"(r[g][7])
+                     : "r"(taddr + 16u * g)
+                     : "memory");
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+        asm volatile(""
+                     : "+r"(r[g][0]), "+r"(r[g][1]), "+r"(r[g][2]), "+r"(r[g][3]), "+r"(r[g][4]), "+r"(r[g][5]),
+                       "+r"(r[g][6]), "+r"(r[g][7]));
+}
+
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v)
 {
     uint32_t r[16];
@@ -757,27 +778,56 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
         const float gh = (FMT == DS4G_NVFP4 && EPI == DS4G_EPI_SWIGLU_REQUANT) ? *p.oq_g : 1.0f;
         for (int64_t t = tile0; t < ntiles; t += tstride, ++tcount) {
             const int buf = (int)(tcount % NACC);
+            // the tile, its scale and (register-direct plain / combine
+            // epilogue) the output rows of this thread's four tile rows are
+            // looked up before waiting for the accumulator, so that their
+            // global loads overlap the tile's mainloop
+            Tile tl = tile_of<C::BMT>(t, prefix, soff, E, n_tiles);
+            tl.m0 += (int64_t)BM * rank;           // a pair: this CTA's 128 rows of the tile
+            const float gscale = (FMT == DS4G_NVFP4) ? __fmul_rn(p.a_g[0], p.w_g[tl.e]) : 1.0f;
+            constexpr bool kDirect = (EPI != DS4G_EPI_SWIGLU_REQUANT) && !C::STAGED;
+            float* dk[2][2];
+            float wk[2][2];
+            if (kDirect) {
+                // rows 16 hh + rsub + 8 k of the warp's 32: four threads hold
+                // 32 contiguous bytes of one row in the 16-lane TMEM loads
+                const int rsub = lane >> 2;
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+                    for (int k = 0; k < 2; ++k) {
+                        const int64_t rk = tl.m0 + 32 * q + 16 * hh + rsub + 8 * k;
+                        dk[hh][k] = nullptr;
+                        wk[hh][k] = gscale;
+                        if (rk < tl.end) {
+                            if (EPI == kEpiCombine) {
+                                const int32_t s = p.r2s[rk];
+                                dk[hh][k] = p.out + (int64_t)(s / p.topk) * p.N + (int64_t)tl.nt * TBN;
+                                wk[hh][k] = p.route_w[s] * gscale;
+                            } else {
+                                dk[hh][k] = p.out + rk * p.N + (int64_t)tl.nt * TBN;
+                            }
+                        }
+                    }
+            }
             const bool got = mbar_wait(smem_u32(&tmem_full[buf]), (tcount / NACC) & 1, abort_flag);
             // a pair's teardown is a warp-aligned cluster barrier: the whole
             // warp leaves the loop together
             if (PAIR ? !__all_sync(0xffffffffu, got) : !got) break;
             tc_fence_after();
-            Tile tl = tile_of<C::BMT>(t, prefix, soff, E, n_tiles);
-            tl.m0 += (int64_t)BM * rank;           // a pair: this CTA's 128 rows of the tile
-            const float gscale = (FMT == DS4G_NVFP4) ? __fmul_rn(p.a_g[0], p.w_g[tl.e]) : 1.0f;
             const int64_t row = tl.m0 + 32 * q + lane;
             const bool valid = row < tl.end;
             const uint32_t tbase = tmem + kColAcc + buf * TBN + ((uint32_t)(32 * q) << 16);
             if (EPI != DS4G_EPI_SWIGLU_REQUANT) {
                 // plain: store the row; combine: add w * row into its token's output
-                float* dst_row = p.out + row * p.N;
-                float wr = gscale;
-                if (EPI == kEpiCombine && valid) {
-                    const int32_t s = p.r2s[row];
-                    dst_row = p.out + (int64_t)(s / p.topk) * p.N;
-                    wr = p.route_w[s] * gscale;
-                }
                 if (C::STAGED) {
+                    float* dst_row = p.out + row * p.N;
+                    float wr = gscale;
+                    if (EPI == kEpiCombine && valid) {
+                        const int32_t s = p.r2s[row];
+                        dst_row = p.out + (int64_t)(s / p.topk) * p.N;
+                        wr = p.route_w[s] * gscale;
+                    }
                     // 32-column pieces of this warp's half (the last one 16 wide),
                     // each as two 16-row blocks through the warp's staging area
                     float* stg = reinterpret_cast<float*>(smem + C::STAGE_OFF) + (warp - 4) * (16 * 33);
@@ -819,42 +869,29 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
                 } else {
                     // 16-lane x 16-column TMEM loads: four threads hold 32
                     // contiguous bytes of one row, so a store / reduction
-                    // instruction writes 8 rows x 32 bytes (full sectors)
-                    const int sub = lane & 3, rsub = lane >> 2;
-#pragma unroll 1
-                    for (int hh = 0; hh < 2; ++hh) {
-                        float* dk[2];
-                        float wk[2];
+                    // instruction writes 8 rows x 32 bytes (full sectors).
+                    // All of a row half's loads are issued before one wait.
+                    constexpr int G = C::HALF / 16;
+                    const int sub = lane & 3;
 #pragma unroll
-                        for (int k = 0; k < 2; ++k) {
-                            const int64_t rk = tl.m0 + 32 * q + 16 * hh + rsub + 8 * k;
-                            dk[k] = nullptr;
-                            wk[k] = gscale;
-                            if (rk < tl.end) {
-                                if (EPI == kEpiCombine) {
-                                    const int32_t s = p.r2s[rk];
-                                    dk[k] = p.out + (int64_t)(s / p.topk) * p.N + (int64_t)tl.nt * TBN;
-                                    wk[k] = p.route_w[s] * gscale;
-                                } else {
-                                    dk[k] = p.out + rk * p.N + (int64_t)tl.nt * TBN;
-                                }
-                            }
-                        }
-                        const uint32_t tb = tmem + kColAcc + buf * TBN + ((uint32_t)(32 * q + 16 * hh) << 16);
-#pragma unroll 1
-                        for (int g = 0; g < C::HALF / 16; ++g) {
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const uint32_t tb = tmem + kColAcc + buf * TBN + ((uint32_t)(32 * q + 16 * hh) << 16) +
+                                            half * C::HALF;
+                        uint32_t r[G][8];
+                        tmem_ld_16x256b_x2_batch<G>(tb, r);
+#pragma unroll
+                        for (int g = 0; g < G; ++g) {
                             const int col = half * C::HALF + 16 * g;
                             if ((int64_t)tl.nt * TBN + col >= p.N) break;      // ragged last tile
-                            uint32_t r[8];
-                            tmem_ld_16x256b_x2(tb + col, r);
 #pragma unroll
                             for (int k = 0; k < 2; ++k) {
-                                if (dk[k] == nullptr) continue;
-                                float* g0 = dk[k] + col + 2 * sub;
-                                const float a0 = __uint_as_float(r[2 * k]) * wk[k];
-                                const float a1 = __uint_as_float(r[2 * k + 1]) * wk[k];
-                                const float b0 = __uint_as_float(r[4 + 2 * k]) * wk[k];
-                                const float b1 = __uint_as_float(r[4 + 2 * k + 1]) * wk[k];
+                                if (dk[hh][k] == nullptr) continue;
+                                float* g0 = dk[hh][k] + col + 2 * sub;
+                                const float w = wk[hh][k];
+                                const float a0 = __uint_as_float(r[g][2 * k]) * w;
+                                const float a1 = __uint_as_float(r[g][2 * k + 1]) * w;
+                                const float b0 = __uint_as_float(r[g][4 + 2 * k]) * w;
+                                const float b1 = __uint_as_float(r[g][4 + 2 * k + 1]) * w;
                                 if (EPI == kEpiCombine) {
                                     red_add_v2(g0, a0, a1);
                                     red_add_v2(g0 + 8, b0, b1);
