@@ -50,11 +50,14 @@ constexpr int kColAcc = 0;         // [issuer][buffer] 16-column accumulators: 6
 constexpr int kColSF = 64;         // [issuer] 16 weight-scale then 16 activation-scale columns
 constexpr int kMaxE = 512;        // experts whose offsets and item counts fit in shared memory
 
-template <int FMT>
+// SPLIT: 1 = one CTA per item; 2 = a CTA pair shares each item, each CTA
+// taking half of its K range (few items: decode FC1 at T = 1)
+template <int FMT, int SPLIT = 1>
 struct Cfg {
     // ring depths: as many 18 KB data stages as shared memory holds next to
-    // the scale stages (each scale stage covers two data stages)
-    static constexpr int STAGES = 10;
+    // the scale stages (each scale stage covers two data stages); a split
+    // NVFP4 kernel gives one stage to the partial-sum exchange rows
+    static constexpr int STAGES = (SPLIT == 2 && FMT == DS4G_NVFP4) ? 9 : 10;
     static constexpr int SF_STAGES = (FMT == DS4G_MXFP4) ? 5 : 4;
     static constexpr int WPS = (FMT == DS4G_MXFP4) ? 2 : 4;    // 4-scale words per row per K stage
     static constexpr int SF_ROW = 2 * WPS * 4;                  // scale bytes per row per scale stage
@@ -64,9 +67,12 @@ struct Cfg {
     static constexpr int DATA_BYTES = STAGES * (W_BYTES + X_BYTES);
     static constexpr int SF_BYTES = SF_STAGES * (SFW_BYTES + SFXR_BYTES + SFXC_BYTES);
     static constexpr int EARR_BYTES = ((kMaxE + 1) * 4 + 15) / 16 * 16;   // one [E + 1] int32 array
-    // data, scales, barriers, the SwiGLU exchange, item prefix and offsets
-    static constexpr size_t SMEM = 1024 + (size_t)DATA_BYTES + SF_BYTES + 512 + 64 * 16 * 4 + 2 * EARR_BYTES;
-    static_assert((2 * STAGES + 3 * SF_STAGES + 4) * 8 + 16 <= 512, "barrier block");
+    static constexpr int XRED_BYTES = (SPLIT == 2) ? BMW * BNT * 4 : 0;   // the follower's partial sums
+    // data, scales, barriers, the SwiGLU exchange, item prefix and offsets,
+    // partial-sum rows
+    static constexpr size_t SMEM =
+        1024 + (size_t)DATA_BYTES + SF_BYTES + 512 + 64 * 16 * 4 + 2 * EARR_BYTES + XRED_BYTES;
+    static_assert((2 * STAGES + 3 * SF_STAGES + 6) * 8 + 16 <= 512, "barrier block");
     static_assert(SMEM <= 232448, "shared memory per CTA");
 };
 
@@ -121,12 +127,22 @@ __device__ __forceinline__ void sfx_transpose(const uint8_t* raw, uint8_t* chunk
     __syncwarp();
 }
 
-template <int FMT, int EPI>
+// the follower's partial sums into the leader's shared memory, counted on the
+// leader's mbarrier
+__device__ __forceinline__ void st_async_v4(uint32_t cluster_addr, float a, float b, float c, float d,
+                                            uint32_t mbar_cluster)
+{
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];"
+                 ::"r"(cluster_addr), "f"(a), "f"(b), "f"(c), "f"(d), "r"(mbar_cluster)
+                 : "memory");
+}
+
+template <int FMT, int EPI, int SPLIT>
 __global__ void __launch_bounds__(kThreads, 1)
 k_gemv_tc(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x,
           const __grid_constant__ CUtensorMap map_sfw, const __grid_constant__ CUtensorMap map_sfx, const GemmArgs p)
 {
-    using C = Cfg<FMT>;
+    using C = Cfg<FMT, SPLIT>;
     constexpr int STAGES = C::STAGES;
     constexpr int SF_STAGES = C::SF_STAGES;
     constexpr bool kSwiGLU = (EPI == DS4G_EPI_SWIGLU_REQUANT);
@@ -145,12 +161,15 @@ k_gemv_tc(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUt
     uint64_t* sf_empty = sf_ready + SF_STAGES;
     uint64_t* tmem_full = sf_empty + SF_STAGES;
     uint64_t* tmem_empty = tmem_full + 2;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tmem_empty + 2);
+    uint64_t* red_full = tmem_empty + 2;                      // split: the leader's exchange rows landed
+    uint64_t* red_empty = red_full + 1;                       // split: the follower may send the next item
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(red_empty + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int32_t* total_items = reinterpret_cast<int32_t*>(tmem_slot + 2);
     float* xch = reinterpret_cast<float*>(smem + C::DATA_BYTES + C::SF_BYTES + 512);   // [64][16] up rows
     int32_t* prefix = reinterpret_cast<int32_t*>(xch + 64 * 16);
     int32_t* soff = prefix + C::EARR_BYTES / 4;      // the expert offsets, staged once
+    float* xred = reinterpret_cast<float*>(soff + C::EARR_BYTES / 4);   // split: [128][16] partial sums
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int E = p.E;
@@ -158,6 +177,15 @@ k_gemv_tc(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUt
     const int nks = (int)ceil_div(K, BK);
     const int npairs = (nks + 1) / 2;
     const int I = p.N / 2;
+    // a split pair: rank r takes scale stages [jb, jb + np_loc) of every item
+    // (the leader the first half); both walk the items of their cluster
+    const uint32_t rank = (SPLIT == 2) ? cluster_ctarank() : 0u;
+    const int np_lo = (SPLIT == 2) ? (npairs + 1) / 2 : npairs;
+    const int jb = (rank == 1) ? np_lo : 0;
+    const int np_loc = (SPLIT == 2) ? (rank == 0 ? np_lo : npairs - np_lo) : npairs;
+    const int nks_loc = min(nks, 2 * (jb + np_loc)) - 2 * jb;
+    const int64_t t_first = (SPLIT == 2) ? (int64_t)cluster_id_x() : (int64_t)blockIdx.x;
+    const int64_t t_step = (SPLIT == 2) ? (int64_t)nclusters_x() : (int64_t)gridDim.x;
     const int wtiles = kSwiGLU ? (I / 64) : (p.N / BMW);
 
     if (threadIdx.x == 0) {
@@ -174,6 +202,8 @@ k_gemv_tc(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUt
             mbar_init(smem_u32(&tmem_full[b2]), 2);
             mbar_init(smem_u32(&tmem_empty[b2]), 128);
         }
+        mbar_init(smem_u32(red_full), 1);      // the leader's expect-tx arrival + the follower's bytes
+        mbar_init(smem_u32(red_empty), 4);     // one arrival per leader epilogue warp
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -226,7 +256,8 @@ k_gemv_tc(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUt
         }
     }
     tc_fence_before();
-    __syncthreads();
+    // a pair: the peer's barriers must be initialised before anything arrives on them
+    if (SPLIT == 2) cluster_sync_all(); else __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const int64_t nitems = *total_items;
@@ -245,13 +276,14 @@ k_gemv_tc(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUt
             const int pi = (warp == 0) ? 0 : 1;
             uint32_t tcount = 0, it_next = 0, sit_next = 0;
             bool ok = true;
-            for (int64_t t = blockIdx.x; t < nitems && ok; t += gridDim.x, ++tcount) {
+            for (int64_t t = t_first; t < nitems && ok; t += t_step, ++tcount) {
                 const Item itm = item_of(t, prefix, soff, E, wtiles);
                 int64_t y0, y1;
                 w_rows<EPI>(itm, p.N, I, y0, y1);
-                const uint32_t it0 = tcount * (uint32_t)nks, sit0 = tcount * (uint32_t)npairs;
-                for (int j = pi ^ (int)(sit0 & 1); j < npairs; j += 2) {
-                    const uint32_t sit = sit0 + j, ita = it0 + 2 * j;
+                const uint32_t it0 = tcount * (uint32_t)nks_loc, sit0 = tcount * (uint32_t)np_loc;
+                for (int jl = pi ^ (int)(sit0 & 1); jl < np_loc; jl += 2) {
+                    const int j = jb + jl;                        // scale stage within the item's K
+                    const uint32_t sit = sit0 + jl, ita = it0 + 2 * jl;
                     const int nd = min(2, nks - 2 * j);
                     const int r = sit % SF_STAGES;
                     if (!mbar_wait(smem_u32(&sf_empty[r]), ((sit / SF_STAGES) & 1) ^ 1, abort_flag)) { ok = false; break; }
@@ -283,7 +315,7 @@ k_gemv_tc(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUt
                 volatile int never = 0;
                 bool go = true;
                 for (uint32_t j = (it_next > STAGES + 2 ? it_next - STAGES - 2 : 0); j < it_next && go; ++j) {
-                    const uint32_t owner = ((j / nks) * npairs + (j % nks) / 2) & 1;
+                    const uint32_t owner = ((j / nks_loc) * np_loc + (j % nks_loc) / 2) & 1;
                     if ((int)owner == pi) go = mbar_wait(smem_u32(&full[j % STAGES]), (j / STAGES) & 1, &never);
                 }
                 for (uint32_t j = (sit_next > SF_STAGES + 1 ? sit_next - SF_STAGES - 1 : 0); j < sit_next && go; ++j)
@@ -302,15 +334,16 @@ k_gemv_tc(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUt
             const uint32_t col_sfw = tmem + kColSF + pi * 32, col_sfx = col_sfw + 16;
             uint32_t tcount = 0;
             bool ok = true;
-            for (int64_t t = blockIdx.x; t < nitems && ok; t += gridDim.x, ++tcount) {
+            for (int64_t t = t_first; t < nitems && ok; t += t_step, ++tcount) {
                 const int buf = tcount & 1;
                 if (!mbar_wait(smem_u32(&tmem_empty[buf]), ((tcount >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t acc = tmem + kColAcc + pi * 32 + buf * BNT;
-                const uint32_t it0 = tcount * (uint32_t)nks, sit0 = tcount * (uint32_t)npairs;
+                const uint32_t it0 = tcount * (uint32_t)nks_loc, sit0 = tcount * (uint32_t)np_loc;
                 bool first = true;
-                for (int j = pi ^ (int)(sit0 & 1); j < npairs; j += 2) {
-                    const uint32_t sit = sit0 + j, ita = it0 + 2 * j;
+                for (int jl = pi ^ (int)(sit0 & 1); jl < np_loc; jl += 2) {
+                    const int j = jb + jl;                        // scale stage within the item's K
+                    const uint32_t sit = sit0 + jl, ita = it0 + 2 * jl;
                     const int nd = min(2, nks - 2 * j);
                     const int r = sit % SF_STAGES;
                     if (!mbar_wait(smem_u32(&sf_ready[r]), (sit / SF_STAGES) & 1, abort_flag)) { ok = false; break; }
@@ -356,9 +389,9 @@ k_gemv_tc(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUt
     } else if (warp == 2) {
         // ================= scale transposer =================
         uint32_t sit = 0;
-        for (int64_t t = blockIdx.x; t < nitems; t += gridDim.x) {
+        for (int64_t t = t_first; t < nitems; t += t_step) {
             bool ok = true;
-            for (int pr = 0; pr < npairs; ++pr, ++sit) {
+            for (int pr = 0; pr < np_loc; ++pr, ++sit) {
                 const int r = sit % SF_STAGES;
                 bool w_ok = true;
                 if (lane == 0) w_ok = mbar_wait(smem_u32(&sf_full[r]), (sit / SF_STAGES) & 1, abort_flag);
@@ -376,17 +409,20 @@ k_gemv_tc(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUt
         const int q = warp & 3;                  // weight rows 32q .. 32q + 31 of the tile
         uint32_t tcount = 0;
         const float gh = (FMT == DS4G_NVFP4 && kSwiGLU) ? *p.oq_g : 1.0f;
-        for (int64_t t = blockIdx.x; t < nitems; t += gridDim.x, ++tcount) {
+        for (int64_t t = t_first; t < nitems; t += t_step, ++tcount) {
             const int buf = tcount & 1;
-            if (!mbar_wait(smem_u32(&tmem_full[buf]), (tcount >> 1) & 1, abort_flag)) break;
+            const bool got = mbar_wait(smem_u32(&tmem_full[buf]), (tcount >> 1) & 1, abort_flag);
+            // a pair's teardown is a warp-aligned cluster barrier: the whole
+            // warp leaves the loop together
+            if (SPLIT == 2 ? !__all_sync(0xffffffffu, got) : !got) break;
             tc_fence_after();
             const Item itm = item_of(t, prefix, soff, E, wtiles);
             const float gscale = (FMT == DS4G_NVFP4) ? __fmul_rn(p.a_g[0], p.w_g[itm.e]) : 1.0f;
             // issuer i holds the sum over the scale stages of parity i
-            const uint32_t sit0 = tcount * (uint32_t)npairs;
+            const uint32_t sit0 = tcount * (uint32_t)np_loc;
             const uint32_t lanes = (uint32_t)(32 * q) << 16;
             float v[16];
-            if (npairs >= 2) {
+            if (np_loc >= 2) {
                 float v1[16];
                 tmem_ld16(tmem + kColAcc + buf * BNT + lanes, v);
                 tmem_ld16(tmem + kColAcc + 32 + buf * BNT + lanes, v1);
@@ -397,6 +433,35 @@ k_gemv_tc(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUt
             }
             tc_fence_before();
             mbar_arrive(smem_u32(&tmem_empty[buf]));          // accumulator drained into registers
+            if (SPLIT == 2) {
+                // the follower sends its K half's sums for this item to the
+                // leader, which adds them and runs the epilogue
+                const int i = 32 * q + lane;                  // weight row of the tile
+                if (rank == 1) {
+                    const bool free_ = mbar_wait(smem_u32(red_empty), (tcount & 1) ^ 1, abort_flag);
+                    if (!__all_sync(0xffffffffu, free_)) break;
+                    const uint32_t dst = mapa_shared(smem_u32(xred + i * BNT), 0);
+                    const uint32_t mb = mapa_shared(smem_u32(red_full), 0);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+                        st_async_v4(dst + 16u * c, v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3], mb);
+                    continue;
+                }
+                if (threadIdx.x == 128) mbar_arrive_tx(smem_u32(red_full), BMW * BNT * 4);
+                const bool landed = mbar_wait(smem_u32(red_full), tcount & 1, abort_flag);
+                if (!__all_sync(0xffffffffu, landed)) break;
+                const float4* src = reinterpret_cast<const float4*>(xred + i * BNT);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const float4 u4 = src[c];
+                    v[4 * c] += u4.x;
+                    v[4 * c + 1] += u4.y;
+                    v[4 * c + 2] += u4.z;
+                    v[4 * c + 3] += u4.w;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(red_empty), 1));
+            }
             if (!kSwiGLU) {
                 const int64_t n = (int64_t)itm.wt * BMW + 32 * q + lane;
 #pragma unroll
@@ -455,7 +520,8 @@ k_gemv_tc(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUt
     }
 
     tc_fence_before();
-    __syncthreads();
+    // a pair: neither CTA leaves while the other may still reach its shared memory
+    if (SPLIT == 2) cluster_sync_all(); else __syncthreads();
     tc_fence_after();
     if (warp == 3) {
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
@@ -464,10 +530,10 @@ k_gemv_tc(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUt
 
 }  // namespace dtc
 
-template <int FMT, int EPI>
+template <int FMT, int EPI, int SPLIT = 1>
 static cudaError_t run_dtc(const GemmArgs& a, cudaStream_t st)
 {
-    using C = dtc::Cfg<FMT>;
+    using C = dtc::Cfg<FMT, SPLIT>;
     const int blk = (FMT == DS4G_MXFP4) ? 32 : 16;
     const uint32_t wbox = (EPI == DS4G_EPI_SWIGLU_REQUANT) ? 64 : 128;
     CUtensorMap mw, mx, msw, msx;
@@ -476,14 +542,53 @@ static cudaError_t run_dtc(const GemmArgs& a, cudaStream_t st)
         !make_map(&msw, a.w_scales, (int64_t)a.E * a.N, a.K / blk, C::SF_ROW, wbox, false) ||
         !make_map(&msx, a.a_scales, a.S, a.K / blk, C::SF_ROW, dtc::BNT, false))
         return cudaErrorInvalidValue;
-    auto kern = dtc::k_gemv_tc<FMT, EPI>;
+    auto kern = dtc::k_gemv_tc<FMT, EPI, SPLIT>;
     const size_t shm = C::SMEM;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)shm);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = kNumSMs;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    kern<<<sms, dtc::kThreads, shm, st>>>(mw, mx, msw, msx, a);
+    if (SPLIT == 1) {
+        kern<<<sms, dtc::kThreads, shm, st>>>(mw, mx, msw, msx, a);
+        return cudaGetLastError();
+    }
+    // CTA pairs: clusters of two, as many as can be resident at once
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3((unsigned)(sms & ~1));
+    cfg.blockDim = dim3(dtc::kThreads);
+    cfg.dynamicSmemBytes = shm;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int nclusters = 0;
+    e = cudaOccupancyMaxActiveClusters(&nclusters, kern, &cfg);
+    if (e != cudaSuccess) return e;
+    if (nclusters < 1) return cudaErrorInvalidConfiguration;
+    cfg.gridDim = dim3((unsigned)(2 * (nclusters < sms / 2 ? nclusters : sms / 2)));
+    e = cudaLaunchKernelEx(&cfg, kern, mw, mx, msw, msx, a);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
+}
+
+// FC1 with few items (at most about two per SM: decode T = 1) splits each
+// item's K range over a CTA pair, so that no SM streams two whole items while
+// others idle.  DS4G_DTC_SPLIT=0 / 1 in the environment forces it off / on.
+static bool use_split(const GemmArgs& a)
+{
+    const int64_t K = a.K;
+    const int npairs = (int)((ceil_div(K, 256) + 1) / 2);
+    if (a.epilogue != DS4G_EPI_SWIGLU_REQUANT || npairs < 2) return false;
+    const char* env = getenv("DS4G_DTC_SPLIT");
+    if (env && env[0] == '0') return false;
+    if (env && env[0] == '1') return true;
+    const int64_t wtiles = (a.N / 2) / 64;
+    const int64_t experts = a.E < a.S ? a.E : a.S;       // experts that can hold rows
+    return experts * wtiles <= 2 * kNumSMs;
 }
 
 bool gemv_tc_supports(int fmt, int64_t K, int N, int epilogue, int E)
@@ -496,12 +601,15 @@ cudaError_t launch_gemv_tc(const GemmArgs& a, cudaStream_t st)
 {
     if (a.S == 0) return cudaSuccess;
     if (!gemv_tc_supports(a.fmt, a.K, a.N, a.epilogue, a.E)) return cudaErrorInvalidValue;
+    const bool split = use_split(a);
     if (a.fmt == DS4G_MXFP4)
         return a.epilogue == DS4G_EPI_NONE ? run_dtc<DS4G_MXFP4, DS4G_EPI_NONE>(a, st)
              : a.epilogue == kEpiCombine   ? run_dtc<DS4G_MXFP4, kEpiCombine>(a, st)
+             : split                       ? run_dtc<DS4G_MXFP4, DS4G_EPI_SWIGLU_REQUANT, 2>(a, st)
                                            : run_dtc<DS4G_MXFP4, DS4G_EPI_SWIGLU_REQUANT>(a, st);
     return a.epilogue == DS4G_EPI_NONE ? run_dtc<DS4G_NVFP4, DS4G_EPI_NONE>(a, st)
          : a.epilogue == kEpiCombine   ? run_dtc<DS4G_NVFP4, kEpiCombine>(a, st)
+         : split                       ? run_dtc<DS4G_NVFP4, DS4G_EPI_SWIGLU_REQUANT, 2>(a, st)
                                        : run_dtc<DS4G_NVFP4, DS4G_EPI_SWIGLU_REQUANT>(a, st);
 }
 

@@ -177,7 +177,11 @@ ds4g_status ds4g_moe_dispatch(const float* logits, const void* x, int dtype, int
  *   routing); it selects the kernel:
  *   <= 16 rows, K a multiple of 512 (MXFP4) / 256 (NVFP4), N % 128 == 0
  *     (NONE) or I % 64 == 0 (SWIGLU_REQUANT): tensor-core kernel with the
- *     weights as the MMA's M side (decode);
+ *     weights as the MMA's M side (decode); with SWIGLU_REQUANT and at most
+ *     about two weight tiles per SM (min(E, rows) x I / 64 <= 296) each
+ *     tile's K range is split over a CTA pair whose follower sends its
+ *     partial sums to the leader (DS4G_DTC_SPLIT=0 / 1 in the environment
+ *     forces this off / on);
  *   > 16 rows and the same K rule, N % 224 == 0 (NONE): tensor-core kernel
  *     with 128-row x 224-column tiles and two accumulators (the epilogue of
  *     one tile overlaps the next tile's MMAs); else N % 256 == 0 (NONE):

@@ -243,6 +243,14 @@ def tc_mode(request, monkeypatch):
     return request.param
 
 
+# decode-sized FC1 (<= 16 rows per expert) runs either one CTA per item or
+# each item's K range split over a CTA pair (DS4G_DTC_SPLIT=0 / 1)
+@pytest.fixture
+def dtc_split(request, monkeypatch):
+    monkeypatch.setenv("DS4G_DTC_SPLIT", request.param)
+    return request.param
+
+
 @pytest.mark.parametrize("fmt", [MX, NV])
 @pytest.mark.parametrize("case,tc_mode", [(c, "0") for c in GEMV_CASES] +
                          [(c, m) for c in TC_CASES for m in PAIR_MODES], indirect=["tc_mode"])
@@ -276,7 +284,8 @@ def _h_bound(y1_ref, ab1, I):
                                   ([200, 9], 384, 1024), ([100, 30], 96, 1024), ([5, 16, 2], 192, 1024),
                                   ([140, 60], 160, 512), ([700, 3, 260], 2048, 1024)])
 @pytest.mark.parametrize("tc_mode", PAIR_MODES, indirect=True)
-def test_fc1_fused_swiglu_requant(fmt, case, tc_mode):
+@pytest.mark.parametrize("dtc_split", ["0", "1"], indirect=True)
+def test_fc1_fused_swiglu_requant(fmt, case, tc_mode, dtc_split):
     seg, I, K = case
     offsets, a, w, gw = _grouped_problem(seg, 2 * I, K, fmt, stream=21)
     S = int(offsets[-1])
