@@ -26,7 +26,7 @@ L2_BYTES = 126 * 1000 * 1000
 # DRAM bytes (read + write) of one FC1 launch, from a one-pass ncu capture of
 # the full-size workload (profiles/dram_traffic_k_gemm_tc_prefill_T2048_mxfp4.md);
 # workloads without a capture of the current kernel report null
-FC1_TRAFFIC = {"prefill": (2335091712, "profiles/dram_traffic_k_gemm_tc_prefill_T2048_mxfp4.md")}
+FC1_TRAFFIC = {"prefill": (2332562944, "profiles/dram_traffic_k_gemm_tc_prefill_T2048_mxfp4.md")}
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
