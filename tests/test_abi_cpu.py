@@ -52,3 +52,51 @@ def test_bad_arguments_rejected_before_any_launch():
     assert L.ds4g_moe_combine(None, None, None, 2, 2, 6, None, None) == 2   # d % 4 != 0
     out = ds4g._Fp4C(None, None, None, 4, 96, 0, 0)
     assert L.ds4g_quantize_mx(None, 0, 4, 96, 0, None, ctypes.byref(out), None, 0, None) == 2   # K % 64
+
+
+def _fp4(rows, K, fmt=0, buf=None):
+    """a ds4g_fp4 descriptor whose data / scale pointers are host addresses:
+    the calls below must reject their arguments before touching them"""
+    from block_scaled_fp4_topk_b200 import ds4g
+    p = buf.ctypes.data if buf is not None else None
+    return ds4g._Fp4C(p, p, p, rows, K, fmt, 0)
+
+
+def test_grouped_gemm_shapes_rejected_on_the_host():
+    import numpy as np
+    from block_scaled_fp4_topk_b200 import ds4g
+    L = ds4g._lib
+    buf = np.zeros(1 << 16, np.uint8)              # 64-byte aligned host buffer, never read
+    offs = np.zeros(5, np.int32)
+    op = offs.ctypes.data_as(ctypes.c_void_p)
+    out = buf.ctypes.data_as(ctypes.c_void_p)
+    a = _fp4(8, 96, buf=buf)
+    w = _fp4(4 * 128, 96, buf=buf)
+    # K % 64 != 0 (the FP4 path's K rule)
+    assert L.ds4g_grouped_gemm_fp4(ctypes.byref(a), op, 4, 8, ctypes.byref(w), 128, 0, out, None, None, None) == 2
+    a, w = _fp4(8, 128, buf=buf), _fp4(4 * 128, 128, buf=buf)
+    # no experts / missing operands
+    assert L.ds4g_grouped_gemm_fp4(ctypes.byref(a), op, 0, 8, ctypes.byref(w), 128, 0, out, None, None, None) == 1
+    assert L.ds4g_grouped_gemm_fp4(None, op, 4, 8, ctypes.byref(w), 128, 0, out, None, None, None) == 1
+    # an epilogue the call does not have
+    assert L.ds4g_grouped_gemm_fp4(ctypes.byref(a), op, 4, 8, ctypes.byref(w), 128, 7, out, None, None, None) == 1
+    # weights whose K differs from the activations'
+    wk = _fp4(4 * 128, 256, buf=buf)
+    assert L.ds4g_grouped_gemm_fp4(ctypes.byref(a), op, 4, 8, ctypes.byref(wk), 128, 0, out, None, None, None) == 2
+    # SwiGLU: N = 2I with I % 32 != 0
+    w80 = _fp4(4 * 80, 128, buf=buf)
+    hq = _fp4(8, 40, buf=buf)
+    assert L.ds4g_grouped_gemm_fp4(ctypes.byref(a), op, 4, 8, ctypes.byref(w80), 80, 1, None, ctypes.byref(hq),
+                                   None, None) == 2
+    # FC2 + combine: a must have T * k rows; k >= 1
+    r2s = offs.ctypes.data_as(ctypes.c_void_p)
+    assert L.ds4g_grouped_gemm_fp4_combine(ctypes.byref(a), op, 4, 8, ctypes.byref(w), 128, r2s, out, 3, 2, out,
+                                           None) == 2
+    assert L.ds4g_grouped_gemm_fp4_combine(ctypes.byref(a), op, 4, 8, ctypes.byref(w), 128, r2s, out, 8, 0, out,
+                                           None) == 1
+
+
+def test_empty_combine_is_a_no_op():
+    from block_scaled_fp4_topk_b200 import ds4g
+    # zero tokens: validated, nothing to launch
+    assert ds4g._lib.ds4g_moe_combine(None, None, None, 0, 6, 7168, None, None) == 0

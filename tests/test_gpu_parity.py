@@ -320,6 +320,28 @@ def test_swiglu_requant(fmt):
     check_requant(from_dev(hq), h_ref, dh, fmt, g=g_h, min_exact=0.9999)
 
 
+@pytest.mark.parametrize("fmt", [MX, NV])
+@pytest.mark.parametrize("max_rows", [0, 300])
+def test_grouped_gemm_no_rows(fmt, max_rows):
+    """no routed rows at all (every expert segment empty): each epilogue
+    returns without work, whichever kernel the row bound selects"""
+    E, N, K = 4, 448, 512
+    offsets = torch.zeros(E + 1, dtype=torch.int32, device=dev())
+    a = ds4g.Fp4Tensor.empty(0, K, fmt, dev())
+    w = ds4g.Fp4Tensor.empty(E * N, K, fmt, dev())
+    if fmt == NV:
+        w.g = torch.ones(E, dtype=torch.float32, device=dev())
+    out = ds4g.ds4g_grouped_gemm_fp4(a, offsets, E, max_rows, w, N)
+    assert out.shape == (0, N)
+    hq = ds4g.Fp4Tensor.empty(0, N // 2, fmt, dev())
+    ds4g.ds4g_grouped_gemm_fp4(a, offsets, E, max_rows, w, N, ds4g.EPI_SWIGLU_REQUANT, out_q=hq)
+    r2s = torch.empty(0, dtype=torch.int32, device=dev())
+    rw = torch.empty((0, 6), dtype=torch.float32, device=dev())
+    out2 = ds4g.ds4g_grouped_gemm_fp4_combine(a, offsets, E, max_rows, w, N, r2s, rw)
+    assert out2.shape == (0, N)
+    ds4g.ds4g_check_device()
+
+
 # ---- FC2 with the combine fused --------------------------------------------------------
 
 @pytest.mark.parametrize("fmt", [MX, NV])
