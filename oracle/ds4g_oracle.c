@@ -219,6 +219,13 @@ void orc_dequantize(const uint8_t* data, const uint8_t* scales, int fmt, double 
  * Selection: k rounds of "largest remaining logit, lower index on ties".
  * Weights: softmax over the selected logits, w_j = e^(l_j - l_max) / sum.
  * ------------------------------------------------------------------------- */
+/* Logits outside the finite numbers (the pages assume finite ones): a NaN
+ * ranks below every number, as -inf does, so each pick is a distinct expert
+ * in [0, E); a pick equal to the maximum has softmax factor exp(0) = 1, which
+ * is also the limit when the maximum is +inf or every pick is -inf. */
+static double route_key(float v) { return isnan(v) ? -INFINITY : (double)v; }
+static double route_factor(double v, double vmax) { return v == vmax ? 1.0 : exp(v - vmax); }
+
 void orc_route_topk(const float* logits, int T, int E, int k, int32_t* idx, double* w)
 {
     char* taken = (char*)malloc((size_t)E);
@@ -229,15 +236,15 @@ void orc_route_topk(const float* logits, int T, int E, int k, int32_t* idx, doub
             int best = -1;
             for (int e = 0; e < E; ++e) {
                 if (taken[e]) continue;
-                if (best < 0 || l[e] > l[best]) best = e;   /* strict: ties keep lower e */
+                if (best < 0 || route_key(l[e]) > route_key(l[best])) best = e;   /* strict: ties keep lower e */
             }
             taken[best] = 1;
             idx[t * k + j] = best;
         }
-        double lmax = l[idx[t * k]];
+        double lmax = route_key(l[idx[t * k]]);
         double den = 0.0;
-        for (int j = 0; j < k; ++j) den += exp((double)l[idx[t * k + j]] - lmax);
-        for (int j = 0; j < k; ++j) w[t * k + j] = exp((double)l[idx[t * k + j]] - lmax) / den;
+        for (int j = 0; j < k; ++j) den += route_factor(route_key(l[idx[t * k + j]]), lmax);
+        for (int j = 0; j < k; ++j) w[t * k + j] = route_factor(route_key(l[idx[t * k + j]]), lmax) / den;
     }
     free(taken);
 }

@@ -268,6 +268,37 @@ def test_topk_full_sort_and_softmax():
     assert np.all(np.diff(w2, axis=1) <= 0)
 
 
+def test_topk_non_finite_logits():
+    """A NaN logit ranks as -inf; a pick equal to the token's maximum has
+    softmax factor 1, the limit of the softmax when the maximum is +inf or
+    every pick is -inf.  Ranking is checked against a stable sort of that key,
+    the weights against the limits in closed form."""
+    E, k = 8, 3
+    lg = synth.logits(7, E, seed=1)
+    lg[0, :] = -np.inf                       # all -inf: experts 0..k-1, equal weights
+    lg[1, 4] = np.inf                        # one +inf takes all the weight
+    lg[2, [1, 6]] = np.inf                   # two +inf: half each, lower index first
+    lg[3, :] = np.nan
+    lg[3, 5] = 0.0                           # the one number first, then NaNs in index order
+    lg[4, [0, 2]] = np.nan                   # NaNs among numbers are never picked
+    lg[5, :] = np.nan                        # all NaN: as all -inf
+    lg[6, [3, 7]] = -np.inf                  # -inf among numbers
+    idx, w = oracle.route_topk(lg, k)
+    key = np.where(np.isnan(lg), -np.inf, lg.astype(np.float64))
+    for t in range(lg.shape[0]):
+        assert np.array_equal(idx[t], np.argsort(-key[t], kind="stable")[:k])
+    assert np.array_equal(idx[0], [0, 1, 2]) and np.array_equal(idx[5], [0, 1, 2])
+    assert np.allclose(w[0], 1.0 / k, rtol=1e-15) and np.allclose(w[5], 1.0 / k, rtol=1e-15)
+    assert idx[1, 0] == 4 and np.array_equal(w[1], [1.0, 0.0, 0.0])
+    assert np.array_equal(idx[2, :2], [1, 6]) and np.array_equal(w[2], [0.5, 0.5, 0.0])
+    assert idx[3, 0] == 5 and np.array_equal(idx[3, 1:], [0, 1]) and np.array_equal(w[3], [1.0, 0.0, 0.0])
+    for t in (4, 6):
+        sel = key[t, idx[t]]
+        assert np.all(np.isfinite(sel))
+        ref = np.exp(sel - sel.max())
+        assert np.allclose(w[t], ref / ref.sum(), rtol=1e-15, atol=0)
+
+
 def test_permute_invariants():
     T, k, E = 37, 3, 16
     lg = synth.logits(T, E, seed=0, bias_sigma=1.5)
