@@ -5,7 +5,9 @@
 //
 // One warp per token.  Each lane keeps E/32 logits in registers; k rounds of
 // a warp arg-max (largest value, lower index on ties) pick the experts in
-// descending order, then the weights are the softmax over the k picks.
+// descending order, then the weights are the softmax over the k picks.  A NaN
+// logit ranks as -inf and a pick equal to the maximum has softmax factor 1, so
+// any logits give k distinct experts in [0, E) (infinities take the limit).
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -21,7 +23,8 @@ __device__ __forceinline__ void route_token(const float* __restrict__ l, int E, 
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
         int e = i * 32 + lane;           // coalesced: lane-consecutive experts
-        v[i] = (e < E) ? l[e] : -INFINITY;
+        const float x = (e < E) ? l[e] : -INFINITY;
+        v[i] = isnan(x) ? -INFINITY : x; // a NaN ranks below every number: picks stay in [0, E)
     }
     unsigned taken = 0;                  // bit i: v[i] already selected
     float sel_v = 0.f, vmax = 0.f, den = 0.f;
@@ -45,7 +48,7 @@ __device__ __forceinline__ void route_token(const float* __restrict__ l, int E, 
         if ((be & 31) == lane) taken |= 1u << (be >> 5);
         if (j == 0) vmax = bv;
         sel_v = bv;
-        float p = expf(sel_v - vmax);
+        float p = (sel_v == vmax) ? 1.f : expf(sel_v - vmax);   // 1 also when the maximum is +-inf
         den += p;
         if (lane == j) { my_e = be; my_v = p; }
     }

@@ -37,7 +37,8 @@
  *   - Launch failures return DS4G_ERR_CUDA.  A device-side wait that gives up
  *     (a bounded spin in a persistent kernel) records an error word that
  *     ds4g_check_device() turns into DS4G_ERR_DEVICE.
- *   - Inputs must be finite (no NaN / Inf).
+ *   - Activations and weights must be finite (no NaN / Inf).  Router logits
+ *     may hold any value (see ds4g_route_topk).
  */
 #ifndef DS4G_H
 #define DS4G_H
@@ -116,7 +117,10 @@ ds4g_status ds4g_quantize_mx(const void* x, int dtype, int64_t rows, int64_t K, 
  * (fp32): the k largest logits, ties to the lower expert index, written in
  * descending order to idx [T][k] (int32); weights w [T][k] (fp32) are the
  * softmax over the k selected logits (they sum to 1).  1 <= k <= min(E, 32),
- * E <= 1024. */
+ * E <= 1024.  Non-finite logits: a NaN ranks below every number, as -inf
+ * does, and a pick equal to the token's maximum has softmax factor 1 (the
+ * limit when that maximum is +inf or every pick is -inf), so idx always
+ * holds k distinct experts in [0, E). */
 ds4g_status ds4g_route_topk(const float* logits, int T, int E, int k, int32_t* idx, float* w,
                             void* stream);
 
@@ -129,7 +133,9 @@ ds4g_status ds4g_route_topk(const float* logits, int T, int E, int k, int32_t* i
  *   slot_to_row [S] the inverse
  *   a_perm          row r = row t = row_to_slot[r] / k of x_q (data and
  *                   scales copied; for NVFP4 a_perm->g receives x_q->g)
- * S = T*k; a_perm->rows must be S, same K and fmt as x_q.
+ * S = T*k; a_perm->rows must be S, same K and fmt as x_q.  Every idx entry
+ * must lie in [0, E) (ds4g_route_topk's always do); the device does not
+ * check them, and an entry outside that range indexes out of bounds.
  * Workspace: ds4g_permute_workspace_bytes(T, k, E). */
 size_t ds4g_permute_workspace_bytes(int T, int k, int E);
 ds4g_status ds4g_moe_permute(const int32_t* idx, int T, int k, int E, const ds4g_fp4* x_q,

@@ -105,6 +105,46 @@ def test_route_topk(T, E, k, bias):
     assert np.allclose(w.cpu().numpy(), rw, rtol=0, atol=2e-6)
 
 
+def _non_finite_logits(T, E, seed):
+    lg = synth.logits(T, E, seed, 1.5)
+    lg[0, :] = -np.inf
+    lg[1, 17] = np.inf
+    lg[2, [3, E - 1]] = np.inf
+    lg[3, :] = np.nan
+    lg[3, E // 2] = 0.0
+    lg[4, ::3] = np.nan
+    lg[5, :] = np.nan
+    lg[6, 1::2] = -np.inf
+    return lg
+
+
+@pytest.mark.parametrize("T,E,k", [(8, 256, 6), (100, 256, 6), (9, 64, 8)])
+def test_route_topk_non_finite(T, E, k):
+    """NaN ranks as -inf, infinities take the softmax's limit: picks stay
+    distinct and in [0, E), identical to the oracle's"""
+    lg = _non_finite_logits(T, E, 5)
+    idx, w = ds4g.ds4g_route_topk(torch.from_numpy(lg).to(dev()), k)
+    ridx, rw = oracle.route_topk(lg, k)
+    assert np.array_equal(idx.cpu().numpy(), ridx)
+    assert np.allclose(w.cpu().numpy(), rw, rtol=0, atol=2e-6)
+
+
+@pytest.mark.parametrize("T,k,E", [(8, 6, 256), (200, 6, 256)])
+def test_dispatch_non_finite_logits(T, k, E):
+    """the fused dispatch (one-CTA path at 48 slots, three kernels at 1200)
+    routes non-finite logits like the oracle and permutes in bounds"""
+    lg = _non_finite_logits(T, E, 6)
+    bits = synth.normal_bf16_bits((T, 256), 0, 62, 1.0)
+    idx, w, xq, offs, r2s, s2r, a = ds4g.ds4g_moe_dispatch(torch.from_numpy(lg).to(dev()), bf16_dev(bits), k, MX)
+    ds4g.ds4g_check_device()
+    ridx, rw = oracle.route_topk(lg, k)
+    assert np.array_equal(idx.cpu().numpy(), ridx)
+    assert np.allclose(w.cpu().numpy(), rw, rtol=0, atol=2e-6)
+    roffs, rr2s, rs2r = oracle.moe_permute(ridx, E)
+    assert np.array_equal(offs.cpu().numpy(), roffs)
+    assert np.array_equal(r2s.cpu().numpy(), rr2s) and np.array_equal(s2r.cpu().numpy(), rs2r)
+
+
 # ---- permutation ---------------------------------------------------------------
 
 @pytest.mark.parametrize("T,k,E,fmt", [(16, 2, 8, MX), (1000, 6, 256, MX), (333, 6, 256, NV), (1, 6, 256, MX),
