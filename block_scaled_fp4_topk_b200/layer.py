@@ -56,13 +56,14 @@ class MoeLayer:
             self._bufs[key] = b
         return b
 
-    def forward(self, x, logits, h_debug=None):
-        """x: bf16 [T][d] (device), logits: fp32 [T][E] (device) -> fp32 [T][d]"""
+    def forward(self, x, logits, h_debug=None, out=None):
+        """x: bf16 [T][d] (device), logits: fp32 [T][E] (device) -> fp32 [T][d]
+        (written into `out` when given, else into the layer's own buffer)"""
         T = x.shape[0]
         b = self.buffers(T, x.device)
         self.dispatch(x, logits, b)
         self.fc1(b, T, h_debug)
-        return self.fc2(b, T)
+        return self.fc2(b, T, out)
 
     def dispatch(self, x, logits, b):
         """routing, activation quantisation and the expert-contiguous
@@ -87,15 +88,16 @@ class MoeLayer:
             ds4g.ds4g_grouped_gemm_fp4(b["a"], b["offsets"], self.E, T, self.w1, 2 * self.I, EPI_NONE, out=b["y1"])
             ds4g.ds4g_swiglu_requant(b["y1"], self.fmt, h_q=b["hq"], h_debug=h_debug)
 
-    def fc2(self, b, T):
+    def fc2(self, b, T, out=None):
         """grouped FC2 and the routing-weighted combine into out [T][d]"""
+        out = b["out"] if out is None else out
         if self.fused_combine:
             ds4g.ds4g_grouped_gemm_fp4_combine(b["hq"], b["offsets"], self.E, T, self.w2, self.d, b["r2s"],
-                                               b["w"], out=b["out"])
+                                               b["w"], out=out)
         else:
             ds4g.ds4g_grouped_gemm_fp4(b["hq"], b["offsets"], self.E, T, self.w2, self.d, EPI_NONE, out=b["y2"])
-            ds4g.ds4g_moe_combine(b["y2"], b["s2r"][:T * self.k], b["w"], out=b["out"])
-        return b["out"]
+            ds4g.ds4g_moe_combine(b["y2"], b["s2r"][:T * self.k], b["w"], out=out)
+        return out
 
     def _warm(self, x, logits):
         side = torch.cuda.Stream(device=x.device)
@@ -104,14 +106,15 @@ class MoeLayer:
             self.forward(x, logits)            # first call sets kernel attributes, buffers
         torch.cuda.current_stream(x.device).wait_stream(side)
 
-    def capture(self, x, logits):
+    def capture(self, x, logits, out=None):
         """Records forward(x, logits) on these (static) input buffers as a CUDA
         graph; returns (graph, out).  Replaying the graph re-runs the whole
-        layer on whatever x / logits hold at that time."""
+        layer on whatever x / logits hold at that time, writing `out` when
+        given (else the layer's own output buffer)."""
         self._warm(x, logits)
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph):
-            out = self.forward(x, logits)
+            out = self.forward(x, logits, out=out)
         return graph, out
 
     def capture_stages(self, x, logits):
