@@ -245,9 +245,10 @@ def run_ours(args, rank, world, local_rank):
     ds4g.ds4g_check_device()
     offsets = b["offsets"].cpu().numpy()
     alg = algorithmic(wl, offsets)
-    # route, quantise (NV: amax, g, quantise), permute (1 CTA kernel up to 512
-    # slots, else 4), FC1 + SwiGLU/requant, FC2 + combine
-    launches_per_step = 1 + (1 if wl.fmt == 0 else 3) + (1 if wl.S <= 512 else 4) + 1 + 1
+    # dispatch: one kernel up to 512 slots, else routing, counts, scan, ranks
+    # and quantise-and-scatter (NVFP4: amax and g before them); then FC1 +
+    # SwiGLU/requant and FC2 + combine
+    launches_per_step = (1 if wl.S <= 512 else (5 if wl.fmt == 0 else 7)) + 2
     # A step whose working set is under 3x L2 (decode) would find its weights
     # in L2 when the same layer ran just before.  Consecutive steps then run
     # R layers of the same shape with their own weights, as consecutive
@@ -291,19 +292,21 @@ def run_ours(args, rank, world, local_rank):
     ds4g.ds4g_check_device()
     ms_total = max_over_ranks(ms_total, world, dev)
 
-    # FC1 timed over the same number of whole steps, bracketed by events on
-    # the launching stream between the dispatch and FC2 graphs
-    # (events between all three stage graphs: dispatch, FC1, FC2 + combine)
-    st_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    # FC1, the dominant kernel, timed over the same number of whole steps:
+    # the layer replayed as its stage graphs (dispatch, FC1, FC2 + combine)
+    # with events on the launching stream between them
+    names = [n for n, _ in stages[0]]
+    ns = len(names)
+    st_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(ns + 1)] for _ in range(args.steps)]
     for i in range(args.steps):
         st_ev[i][0].record(st)
-        for g in range(3):
-            stages[i % R][g].replay()
+        for g in range(ns):
+            stages[i % R][g][1].replay()
             st_ev[i][g + 1].record(st)
     torch.cuda.synchronize()
     ds4g.ds4g_check_device()
-    stage_ms = [float(np.mean([ev[g].elapsed_time(ev[g + 1]) for ev in st_ev])) for g in range(3)]
-    fc1_ms = stage_ms[1]
+    stage_ms = {names[g]: float(np.mean([ev[g].elapsed_time(ev[g + 1]) for ev in st_ev])) for g in range(ns)}
+    fc1_ms = stage_ms["fc1_swiglu"]
 
     # end to end through the public API: every step copies its inputs from
     # pinned host memory to the device, runs the layer and copies its result
@@ -425,8 +428,7 @@ def run_ours(args, rank, world, local_rank):
                         "steps' compute (double-buffered device inputs/outputs)"},
         "gpu_launches": launches_per_step * args.steps,
         "step_mode": "CUDA graph of the layer's library calls",
-        "stage_ms": {"dispatch": stage_ms[0], "fc1_swiglu": stage_ms[1], "fc2_combine": stage_ms[2],
-                     "note": "each stage as its own graph, events between them"},
+        "stage_ms": dict(stage_ms, note="each stage as its own graph, events between them"),
         "clocks": clk.summary(),
     }
     return line

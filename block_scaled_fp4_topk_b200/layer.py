@@ -118,20 +118,21 @@ class MoeLayer:
         return graph, out
 
     def capture_stages(self, x, logits):
-        """The same layer as three graphs replayed in order: dispatch, FC1,
-        FC2 + combine (so that FC1 can be bracketed by events); returns
-        ([g_dispatch, g_fc1, g_fc2], out)."""
+        """The same layer as three graphs replayed in order, so that each
+        stage can be bracketed by events: dispatch, FC1, FC2 + combine;
+        returns ([(name, graph), ...], out)."""
         self._warm(x, logits)
         T = x.shape[0]
         b = self.buffers(T, x.device)
-        graphs = [torch.cuda.CUDAGraph() for _ in range(3)]
+        names = ["dispatch", "fc1_swiglu", "fc2_combine"]
+        graphs = [torch.cuda.CUDAGraph() for _ in names]
         with torch.cuda.graph(graphs[0]):
             self.dispatch(x, logits, b)
         with torch.cuda.graph(graphs[1]):
             self.fc1(b, T)
         with torch.cuda.graph(graphs[2]):
             out = self.fc2(b, T)
-        return graphs, out
+        return list(zip(names, graphs)), out
 
     # -- synthetic weights -----------------------------------------------------
     @staticmethod
