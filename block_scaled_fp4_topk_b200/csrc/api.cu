@@ -158,9 +158,12 @@ ds4g_status ds4g_moe_dispatch(const float* logits, const void* x, int dtype, int
                                        a_perm->g, workspace, S(stream)));
 }
 
+// chained: FC2 + combine adding into out (not zeroed) and launched to
+// overlap the previous kernel on the stream (decode kernel only)
 static ds4g_status grouped_gemm(const ds4g_fp4* a, const int32_t* offsets, int E, int max_rows_per_expert,
                                 const ds4g_fp4* w, int N, int epilogue, float* out, ds4g_fp4* out_q, float* h_debug,
-                                const int32_t* row_to_slot, const float* route_w, int k, int T, void* stream)
+                                const int32_t* row_to_slot, const float* route_w, int k, int T, void* stream,
+                                bool chained = false)
 {
     if (!a || !w || !offsets || E < 1 || N < 1 || max_rows_per_expert < 0) return DS4G_ERR_INVALID_ARG;
     const int fmt = a->fmt;
@@ -216,7 +219,8 @@ static ds4g_status grouped_gemm(const ds4g_fp4* a, const int32_t* offsets, int E
     g.r2s = row_to_slot;
     g.route_w = route_w;
     g.topk = k;
-    if (epilogue == kEpiCombine && T > 0) {
+    g.chained = chained ? 1 : 0;
+    if (epilogue == kEpiCombine && T > 0 && !chained) {
         cudaError_t e = cudaMemsetAsync(out, 0, sizeof(float) * (size_t)T * N, S(stream));
         if (e != cudaSuccess) return DS4G_ERR_CUDA;
     }
@@ -241,6 +245,25 @@ ds4g_status ds4g_grouped_gemm_fp4_combine(const ds4g_fp4* a, const int32_t* offs
     if (T > 0 && (!row_to_slot || !route_w || !out)) return DS4G_ERR_INVALID_ARG;
     return grouped_gemm(a, offsets, E, max_rows_per_expert, w, N, kEpiCombine, out, nullptr, nullptr, row_to_slot,
                         route_w, k, T, stream);
+}
+
+ds4g_status ds4g_grouped_gemm_fp4_combine_chained(const ds4g_fp4* a, const int32_t* offsets, int E,
+                                                  int max_rows_per_expert, const ds4g_fp4* w, int N,
+                                                  const int32_t* row_to_slot, const float* route_w, int T, int k,
+                                                  float* out, void* stream)
+{
+    if (T < 0 || k < 1) return DS4G_ERR_INVALID_ARG;
+    if (a && a->rows != (int64_t)T * k) return DS4G_ERR_SHAPE;
+    if (T > 0 && (!row_to_slot || !route_w || !out)) return DS4G_ERR_INVALID_ARG;
+    return grouped_gemm(a, offsets, E, max_rows_per_expert, w, N, kEpiCombine, out, nullptr, nullptr, row_to_slot,
+                        route_w, k, T, stream, true);
+}
+
+ds4g_status ds4g_zero_fill(void* p, size_t bytes, void* stream)
+{
+    if (bytes == 0) return DS4G_OK;
+    if (!p) return DS4G_ERR_INVALID_ARG;
+    return cudaMemsetAsync(p, 0, bytes, S(stream)) == cudaSuccess ? DS4G_OK : DS4G_ERR_CUDA;
 }
 
 ds4g_status ds4g_swiglu_requant(const float* y1, int64_t rows, int I, int fmt, ds4g_fp4* h_q, float* h_debug,

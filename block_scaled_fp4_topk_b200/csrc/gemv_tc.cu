@@ -171,6 +171,9 @@ k_gemv_tc(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUt
     int32_t* soff = prefix + C::EARR_BYTES / 4;      // the expert offsets, staged once
     float* xred = reinterpret_cast<float*>(soff + C::EARR_BYTES / 4);   // split: [128][16] partial sums
 
+    // a chained launch of the next kernel on the stream may start now: its
+    // CTAs take the SMs this grid's CTAs leave
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int E = p.E;
     const int64_t K = p.K;
@@ -276,6 +279,33 @@ k_gemv_tc(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUt
             const int pi = (warp == 0) ? 0 : 1;
             uint32_t tcount = 0, it_next = 0, sit_next = 0;
             bool ok = true;
+            // a chained launch may start while the previous kernel on the
+            // stream (the producer of the activations) still runs: the first
+            // SF_STAGES scale stages (whose ring slots are free at the start)
+            // load their weights at once and their activation rows only after
+            // griddepcontrol.wait; ndef counts this thread's deferred stages
+            // (scale stages pi, pi + 2, ...)
+            bool waited = (p.chained == 0);
+            uint32_t ndef = 0;
+            auto load_x = [&](uint32_t sit) {
+                const uint32_t n = sit / (uint32_t)np_loc, jl = sit % (uint32_t)np_loc;
+                const Item it = item_of(t_first + (int64_t)n * t_step, prefix, soff, E, wtiles);
+                const int j = jb + (int)jl;
+                const uint32_t ita = n * (uint32_t)nks_loc + 2 * jl;
+                const int nd = min(2, nks - 2 * j);
+                const int r = sit % SF_STAGES;
+                tma_load_2d(smem_u32(sSFXR + r * C::SFXR_BYTES), &map_sfx, smem_u32(&sf_full[r]), j * C::SF_ROW,
+                            (int)it.x0);
+                for (int d = 0; d < nd; ++d) {
+                    const int s = (ita + d) % STAGES;
+                    tma_load_2d(smem_u32(sX + s * X_BYTES), &map_x, smem_u32(&full[s]), (2 * j + d) * BKB, (int)it.x0);
+                }
+            };
+            auto release_deferred = [&]() {
+                asm volatile("griddepcontrol.wait;" ::: "memory");
+                for (uint32_t i = 0; i < ndef; ++i) load_x((uint32_t)pi + 2 * i);
+                waited = true;
+            };
             for (int64_t t = t_first; t < nitems && ok; t += t_step, ++tcount) {
                 const Item itm = item_of(t, prefix, soff, E, wtiles);
                 int64_t y0, y1;
@@ -286,6 +316,11 @@ k_gemv_tc(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUt
                     const uint32_t sit = sit0 + jl, ita = it0 + 2 * jl;
                     const int nd = min(2, nks - 2 * j);
                     const int r = sit % SF_STAGES;
+                    // deferred stages never wait for a slot; the first other
+                    // stage releases them before it waits (its slot frees
+                    // only once a deferred stage has been consumed)
+                    const bool defer = !waited && sit < (uint32_t)SF_STAGES;
+                    if (!waited && !defer) release_deferred();
                     if (!mbar_wait(smem_u32(&sf_empty[r]), ((sit / SF_STAGES) & 1) ^ 1, abort_flag)) { ok = false; break; }
                     for (int d = 0; d < nd && ok; ++d)
                         ok = mbar_wait(smem_u32(&empty[(ita + d) % STAGES]), (((ita + d) / STAGES) & 1) ^ 1, abort_flag);
@@ -295,7 +330,7 @@ k_gemv_tc(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUt
                     const int x = j * C::SF_ROW;
                     tma_load_2d(smem_u32(sSFW + r * C::SFW_BYTES), &map_sfw, sfb, x, (int)y0);
                     if (kSwiGLU) tma_load_2d(smem_u32(sSFW + r * C::SFW_BYTES + C::SFW_BYTES / 2), &map_sfw, sfb, x, (int)y1);
-                    tma_load_2d(smem_u32(sSFXR + r * C::SFXR_BYTES), &map_sfx, sfb, x, (int)itm.x0);
+                    if (!defer) tma_load_2d(smem_u32(sSFXR + r * C::SFXR_BYTES), &map_sfx, sfb, x, (int)itm.x0);
                     for (int d = 0; d < nd; ++d) {
                         const int s = (ita + d) % STAGES;
                         const int ks = 2 * j + d;
@@ -303,12 +338,15 @@ k_gemv_tc(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUt
                         mbar_arrive_tx(fb, W_BYTES + X_BYTES);
                         tma_load_2d(smem_u32(sW + s * W_BYTES), &map_w, fb, ks * BKB, (int)y0);
                         if (kSwiGLU) tma_load_2d(smem_u32(sW + s * W_BYTES + W_BYTES / 2), &map_w, fb, ks * BKB, (int)y1);
-                        tma_load_2d(smem_u32(sX + s * X_BYTES), &map_x, fb, ks * BKB, (int)itm.x0);
+                        if (!defer) tma_load_2d(smem_u32(sX + s * X_BYTES), &map_x, fb, ks * BKB, (int)itm.x0);
                     }
+                    if (defer) ++ndef;
                     it_next = ita + nd;
                     sit_next = sit + 1;
                 }
             }
+            // every armed stage gets its activation rows, also on an early exit
+            if (!waited) release_deferred();
             if (!ok) {
                 // let this thread's copies in flight land before the CTA goes
                 // away (stop at the first wait that gives up)
@@ -548,8 +586,25 @@ static cudaError_t run_dtc(const GemmArgs& a, cudaStream_t st)
     if (e != cudaSuccess) return e;
     int dev = 0, sms = kNumSMs;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (SPLIT == 1) {
+    if (SPLIT == 1 && !a.chained) {
         kern<<<sms, dtc::kThreads, shm, st>>>(mw, mx, msw, msx, a);
+        return cudaGetLastError();
+    }
+    if (SPLIT == 1) {
+        // chained: may start while the previous kernel on the stream runs
+        // (the kernel waits for it before loading activation rows)
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.gridDim = dim3((unsigned)sms);
+        cfg.blockDim = dim3(dtc::kThreads);
+        cfg.dynamicSmemBytes = shm;
+        cfg.stream = st;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, kern, mw, mx, msw, msx, a);
+        if (e != cudaSuccess) return e;
         return cudaGetLastError();
     }
     // CTA pairs: clusters of two, as many as can be resident at once

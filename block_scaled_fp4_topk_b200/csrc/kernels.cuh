@@ -47,6 +47,7 @@ struct GemmArgs {
     const int32_t* r2s;      // combine epilogue: row -> slot, routing weights, k
     const float* route_w;
     int topk;
+    int chained;             // decode kernel: launched to overlap the previous kernel on the stream
 };
 
 cudaError_t launch_gemv(const GemmArgs& a, cudaStream_t st);

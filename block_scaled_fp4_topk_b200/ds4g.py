@@ -57,6 +57,9 @@ _SIGS = {
     "ds4g_swiglu_requant": ([_vp, _i64, _i32, _i32, _P, _vp, _vp], _i32),
     "ds4g_grouped_gemm_fp4_combine": ([_P, _vp, _i32, _i32, _P, _i32, _vp, _vp, _i32, _i32, _vp, _vp], _i32),
     "ds4g_moe_combine": ([_vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp], _i32),
+    "ds4g_grouped_gemm_fp4_combine_chained": ([_P, _vp, _i32, _i32, _P, _i32, _vp, _vp, _i32, _i32, _vp, _vp],
+                                              _i32),
+    "ds4g_zero_fill": ([_vp, _sz, _vp], _i32),
     "ds4g_permute_static_max_bytes": ([], _sz),
     "ds4g_moe_permute_static": ([_vp, _i32, _i32, _i32, _P, _vp, _vp, _vp, _P, _vp], _i32),
 }
@@ -255,6 +258,24 @@ def ds4g_grouped_gemm_fp4_combine(a, offsets, E, max_rows_per_expert, w, N, row_
                                               ctypes.byref(wc), N, row_to_slot.data_ptr(), route_w.data_ptr(), T, k,
                                               out.data_ptr(), _stream()))
     return out
+
+
+def ds4g_grouped_gemm_fp4_combine_chained(a, offsets, E, max_rows_per_expert, w, N, row_to_slot, route_w, out):
+    """FC2 with the combine added into out [T][N] (not zeroed), launched to
+    overlap the previous kernel on the stream (the FC1 call that wrote a)."""
+    T, k = route_w.shape
+    ac, wc = a.c(), w.c()
+    _check("ds4g_grouped_gemm_fp4_combine_chained",
+           _lib.ds4g_grouped_gemm_fp4_combine_chained(ctypes.byref(ac), offsets.data_ptr(), E, max_rows_per_expert,
+                                                      ctypes.byref(wc), N, row_to_slot.data_ptr(),
+                                                      route_w.data_ptr(), T, k, out.data_ptr(), _stream()))
+    return out
+
+
+def ds4g_zero_fill(t):
+    """zero-fills a device tensor on the current stream"""
+    _check("ds4g_zero_fill", _lib.ds4g_zero_fill(t.data_ptr(), t.numel() * t.element_size(), _stream()))
+    return t
 
 
 def ds4g_swiglu_requant(y1, fmt, h_q=None, h_debug=None, g_h=None):

@@ -13,15 +13,19 @@ from .ds4g import EPI_NONE, EPI_SWIGLU_REQUANT, NVFP4, Fp4Tensor
 
 
 class MoeLayer:
-    def __init__(self, w1, w2, E, k, d, I, fmt, g_h=None, fused=True, fused_combine=True, fused_dispatch=True):
+    def __init__(self, w1, w2, E, k, d, I, fmt, g_h=None, fused=True, fused_combine=True, fused_dispatch=True,
+                 chained=True):
         """w1: Fp4Tensor [E*2I][d] (gate rows then up rows per expert),
         w2: Fp4Tensor [E*d][I]; NVFP4 weights carry one tensor scale per
-        expert (w.g has E floats); g_h: the static NVFP4 tensor scale of h."""
+        expert (w.g has E floats); g_h: the static NVFP4 tensor scale of h.
+        chained: the output is zeroed before the dispatch and FC2 + combine
+        is launched to overlap the end of FC1 (decode sizes)."""
         self.w1, self.w2 = w1, w2
         self.E, self.k, self.d, self.I, self.fmt = E, k, d, I, fmt
         self.fused = fused
         self.fused_combine = fused_combine
         self.fused_dispatch = fused_dispatch
+        self.chained = chained and fused_combine
         self.g_h = None
         if fmt == NVFP4:
             dev = w1.data.device
@@ -61,14 +65,16 @@ class MoeLayer:
         (written into `out` when given, else into the layer's own buffer)"""
         T = x.shape[0]
         b = self.buffers(T, x.device)
-        self.dispatch(x, logits, b)
+        self.dispatch(x, logits, b, out)
         self.fc1(b, T, h_debug)
         return self.fc2(b, T, out)
 
-    def dispatch(self, x, logits, b):
+    def dispatch(self, x, logits, b, out=None):
         """routing, activation quantisation and the expert-contiguous
         permutation (one library call; self.fused_dispatch=False issues the
-        three separate calls)"""
+        three separate calls); chained: the output is zeroed first"""
+        if self.chained:
+            ds4g.ds4g_zero_fill(b["out"] if out is None else out)
         if self.fused_dispatch:
             ds4g.ds4g_moe_dispatch(logits, x, self.k, self.fmt, idx=b["idx"], w=b["w"], x_q=b["xq"],
                                    offsets=b["offsets"], row_to_slot=b["r2s"], slot_to_row=b["s2r"], a_perm=b["a"],
@@ -91,7 +97,10 @@ class MoeLayer:
     def fc2(self, b, T, out=None):
         """grouped FC2 and the routing-weighted combine into out [T][d]"""
         out = b["out"] if out is None else out
-        if self.fused_combine:
+        if self.chained:
+            ds4g.ds4g_grouped_gemm_fp4_combine_chained(b["hq"], b["offsets"], self.E, T, self.w2, self.d, b["r2s"],
+                                                       b["w"], out)
+        elif self.fused_combine:
             ds4g.ds4g_grouped_gemm_fp4_combine(b["hq"], b["offsets"], self.E, T, self.w2, self.d, b["r2s"],
                                                b["w"], out=out)
         else:

@@ -12,7 +12,8 @@
  *   ds4g_swiglu_requant   the same epilogue as a separate step
  *   ds4g_grouped_gemm_fp4 FC2
  *   ds4g_moe_combine      routing-weighted sum of each token's k expert rows
- *     (ds4g_grouped_gemm_fp4_combine does FC2 and the combine in one call)
+ *     (ds4g_grouped_gemm_fp4_combine does FC2 and the combine in one call;
+ *      ds4g_grouped_gemm_fp4_combine_chained does it overlapping FC1's end)
  *
  * Sources: "DGX Spark native FP4 matrix instructions: how DwarfStar uses
  * Blackwell" (sec. 1 FP4 formats and the block-scaled MMA, sec. 2 MoE
@@ -220,6 +221,29 @@ ds4g_status ds4g_grouped_gemm_fp4_combine(const ds4g_fp4* a, const int32_t* offs
                                           int max_rows_per_expert, const ds4g_fp4* w, int N,
                                           const int32_t* row_to_slot, const float* route_w, int T, int k,
                                           float* out, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * ds4g_grouped_gemm_fp4_combine chained to the kernel just before it on the
+ * stream (normally the FC1 call that writes a):
+ *   - out is NOT zeroed: the weighted rows are added to what it holds (zero
+ *     it before the FC1 call, e.g. with ds4g_zero_fill, or leave in it what
+ *     the routed experts' sum should be added to);
+ *   - with decode-sized segments the launch may start while that previous
+ *     kernel still runs, so that the FC2 weights stream in while its last
+ *     tiles finish.  The kernel waits for the previous kernel (programmatic
+ *     dependent launch, griddepcontrol.wait) before it reads a; every other
+ *     input (offsets, row_to_slot, route_w, w and out's contents) must be
+ *     complete before that previous kernel started.
+ * Other shapes launch the same kernels as ds4g_grouped_gemm_fp4_combine, in
+ * stream order.  Arguments, results within the same bound and errors as
+ * ds4g_grouped_gemm_fp4_combine. */
+ds4g_status ds4g_grouped_gemm_fp4_combine_chained(const ds4g_fp4* a, const int32_t* offsets, int E,
+                                                  int max_rows_per_expert, const ds4g_fp4* w, int N,
+                                                  const int32_t* row_to_slot, const float* route_w, int T, int k,
+                                                  float* out, void* stream);
+
+/* Zero-fills bytes of device memory at p on the stream (cudaMemsetAsync). */
+ds4g_status ds4g_zero_fill(void* p, size_t bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
  * The SwiGLU + requantisation epilogue as its own step ("Moore Threads ..."

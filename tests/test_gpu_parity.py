@@ -416,6 +416,59 @@ def test_fc2_combine_fused(fmt, T, k, E, N, K, tc_mode):
     assert np.all(np.abs(got - ref) <= bound), f"worst excess {(np.abs(got - ref) - bound).max():.3e}"
 
 
+@pytest.mark.parametrize("fmt", [MX, NV])
+@pytest.mark.parametrize("T,k,E,d,I", [(1, 6, 32, 2048, 1024),     # decode kernel, FC1 split over CTA pairs
+                                       (3, 6, 64, 1024, 512),      # decode kernel
+                                       (300, 6, 16, 512, 512),     # tensor-core kernel (no overlap)
+                                       (4, 2, 8, 256, 128)])       # dp4a kernel (MX)
+def test_fc2_combine_chained(fmt, T, k, E, d, I):
+    """FC1 writes h, then the chained FC2 + combine, launched right after it
+    on the same stream, adds into out: out = (what it held) + the oracle's
+    FC2 + combine of the h codes FC1 produced"""
+    lg = synth.logits(T, E, 7, 1.5)
+    idx, rw = oracle.route_topk(lg, k)
+    offsets, r2s, s2r = oracle.moe_permute(idx, E)
+    S = T * k
+    touched = [e for e in range(E) if offsets[e + 1] > offsets[e]]
+    W = []
+    for n_rows, K, stream in ((2 * I, d, 82), (d, I, 83)):
+        blk = oracle.BLOCK[fmt]
+        data = np.zeros((E * n_rows, K // 2), np.uint8)
+        scales = np.zeros((E * n_rows, K // blk), np.uint8)
+        gw = [1.0] * E
+        for e in touched:          # weights of the touched experts only (no row reads the others)
+            q = oracle.quantize(synth.normal_f32((n_rows, K), e, stream, 0.02), fmt)
+            data[e * n_rows:(e + 1) * n_rows], scales[e * n_rows:(e + 1) * n_rows] = q.data, q.scales
+            gw[e] = q.g if fmt == NV else 1.0
+        W.append((oracle.Fp4(data, scales, 1.0, fmt), gw if fmt == NV else None))
+    (W1, g1), (W2, g2) = W
+    a = oracle.quantize(_x_f32(S, d, 81), fmt)
+    offs_d, r2s_d = torch.from_numpy(offsets).to(dev()), torch.from_numpy(r2s).to(dev())
+    rw32 = rw.astype(np.float32)
+    hq = ds4g.Fp4Tensor.empty(S, I, fmt, dev())
+    if fmt == NV:
+        hq.g.fill_(G_H)
+    base = synth.normal_f32((T, d), 0, 84, 1.0)
+    out = torch.from_numpy(base).to(dev())
+    torch.cuda.synchronize()
+    ds4g.ds4g_grouped_gemm_fp4(to_dev(a), offs_d, E, T, to_dev(W1, g_per_expert=g1), 2 * I, ds4g.EPI_SWIGLU_REQUANT,
+                               out_q=hq)
+    ds4g.ds4g_grouped_gemm_fp4_combine_chained(hq, offs_d, E, T, to_dev(W2, g_per_expert=g2), d, r2s_d,
+                                               torch.from_numpy(rw32).to(dev()), out)
+    ds4g.ds4g_check_device()
+    hq_host = from_dev(hq)
+    y1, ab1 = _ref_gemm(a, offsets, W1, g1, 2 * I)
+    h_ref, dh = _h_bound(y1, ab1, I)
+    check_requant(hq_host, h_ref, dh, fmt, g=G_H)
+    y2, ab2 = _ref_gemm(hq_host, offsets, W2, g2, d)
+    w64 = rw32.astype(np.float64)
+    ref = base.astype(np.float64) + oracle.moe_combine(y2, s2r, w64)
+    bound = (oracle.moe_combine(1e-5 * ab2 + 1e-6, s2r, np.abs(w64)) +
+             1e-6 * (oracle.moe_combine(np.abs(y2), s2r, np.abs(w64)) + np.abs(base)) + 1e-7)
+    got = out.cpu().numpy()
+    assert np.all(np.abs(got - ref) <= bound), f"worst excess {(np.abs(got - ref) - bound).max():.3e}"
+
+
 # ---- combine -----------------------------------------------------------------------
 
 def test_combine():
