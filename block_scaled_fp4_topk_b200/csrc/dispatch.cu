@@ -33,6 +33,10 @@ k_dispatch_small(const float* __restrict__ logits, const T* __restrict__ x, int 
                  uint8_t* __restrict__ ad, uint8_t* __restrict__ as, float* __restrict__ ag)
 {
     extern __shared__ int32_t sh[];
+    // the next kernel on the stream (FC1) may launch now and set itself up
+    // on the SMs this one-CTA kernel leaves idle; it reads nothing of ours
+    // before this grid has finished
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int S = Tn * k;
     int32_t* sidx = sh;               // [S]  picked expert of each slot
     int32_t* cnt = sidx + S;          // [E]  picks per expert, then running ranks

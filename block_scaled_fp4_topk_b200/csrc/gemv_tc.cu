@@ -210,6 +210,12 @@ k_gemv_tc(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUt
         *abort_flag = 0;
         fence_barrier_init();
     }
+    // Every launch may begin while the previous kernel on the stream ends
+    // (programmatic serialization): the set-up above touches no input, and
+    // this wait holds every read of one until that kernel has finished.
+    // A chained FC2 (p.chained) reads its offsets now and waits only before
+    // its activation rows (the producers below).
+    if (!p.chained) asm volatile("griddepcontrol.wait;" ::: "memory");
     // the expert offsets -> shared memory in one parallel pass (a loop of
     // dependent global loads here cost about 2 us per launch)
     for (int e = threadIdx.x; e <= E; e += kThreads) soff[e] = p.offsets[e];
@@ -586,13 +592,10 @@ static cudaError_t run_dtc(const GemmArgs& a, cudaStream_t st)
     if (e != cudaSuccess) return e;
     int dev = 0, sms = kNumSMs;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (SPLIT == 1 && !a.chained) {
-        kern<<<sms, dtc::kThreads, shm, st>>>(mw, mx, msw, msx, a);
-        return cudaGetLastError();
-    }
     if (SPLIT == 1) {
-        // chained: may start while the previous kernel on the stream runs
-        // (the kernel waits for it before loading activation rows)
+        // may start while the previous kernel on the stream runs (the kernel
+        // waits for it before reading any input; a chained FC2 before its
+        // activation rows)
         cudaLaunchConfig_t cfg = {};
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -607,24 +610,28 @@ static cudaError_t run_dtc(const GemmArgs& a, cudaStream_t st)
         if (e != cudaSuccess) return e;
         return cudaGetLastError();
     }
-    // CTA pairs: clusters of two, as many as can be resident at once
+    // CTA pairs: clusters of two, as many as can be resident at once; may
+    // start while the previous kernel runs, as above
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.gridDim = dim3((unsigned)(sms & ~1));
     cfg.blockDim = dim3(dtc::kThreads);
     cfg.dynamicSmemBytes = shm;
     cfg.stream = st;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 1;                          // the occupancy query sees the cluster shape only
     int nclusters = 0;
     e = cudaOccupancyMaxActiveClusters(&nclusters, kern, &cfg);
     if (e != cudaSuccess) return e;
     if (nclusters < 1) return cudaErrorInvalidConfiguration;
     cfg.gridDim = dim3((unsigned)(2 * (nclusters < sms / 2 ? nclusters : sms / 2)));
+    cfg.numAttrs = 2;
     e = cudaLaunchKernelEx(&cfg, kern, mw, mx, msw, msx, a);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();

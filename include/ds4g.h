@@ -188,7 +188,9 @@ ds4g_status ds4g_moe_dispatch(const float* logits, const void* x, int dtype, int
  *     about two weight tiles per SM (min(E, rows) x I / 64 <= 296) each
  *     tile's K range is split over a CTA pair whose follower sends its
  *     partial sums to the leader (DS4G_DTC_SPLIT=0 / 1 in the environment
- *     forces this off / on);
+ *     forces this off / on).  This kernel is launched with programmatic
+ *     stream serialization: it may start while the previous kernel on the
+ *     stream ends, and reads no input before that kernel has finished;
  *   > 16 rows and the same K rule, N % 224 == 0 (NONE): tensor-core kernel
  *     with 128-row x 224-column tiles and two accumulators (the epilogue of
  *     one tile overlaps the next tile's MMAs); else N % 256 == 0 (NONE):
