@@ -96,6 +96,27 @@ def test_grouped_gemm_shapes_rejected_on_the_host():
                                            None) == 1
 
 
+def test_chained_combine_and_zero_fill_rejected_on_the_host():
+    import numpy as np
+    from block_scaled_fp4_topk_b200 import ds4g
+    L = ds4g._lib
+    buf = np.zeros(1 << 16, np.uint8)              # 64-byte aligned host buffer, never read
+    offs = np.zeros(5, np.int32)
+    op = offs.ctypes.data_as(ctypes.c_void_p)
+    out = buf.ctypes.data_as(ctypes.c_void_p)
+    a, w = _fp4(8, 128, buf=buf), _fp4(4 * 128, 128, buf=buf)
+    # a must have T * k rows; k >= 1; T >= 0; the routing arrays when T > 0
+    assert L.ds4g_grouped_gemm_fp4_combine_chained(ctypes.byref(a), op, 4, 8, ctypes.byref(w), 128, op, out, 3, 2,
+                                                   out, None) == 2
+    assert L.ds4g_grouped_gemm_fp4_combine_chained(ctypes.byref(a), op, 4, 8, ctypes.byref(w), 128, op, out, 8, 0,
+                                                   out, None) == 1
+    assert L.ds4g_grouped_gemm_fp4_combine_chained(ctypes.byref(a), op, 4, 8, ctypes.byref(w), 128, None, out, 4, 2,
+                                                   out, None) == 1
+    # zero-fill: nothing to do for 0 bytes; a null pointer otherwise is rejected
+    assert L.ds4g_zero_fill(None, 0, None) == 0
+    assert L.ds4g_zero_fill(None, 64, None) == 1
+
+
 def test_empty_combine_is_a_no_op():
     from block_scaled_fp4_topk_b200 import ds4g
     # zero tokens: validated, nothing to launch
