@@ -25,7 +25,10 @@
 //           rows through shared memory and quantises h along 32-column blocks
 // Items (expert, group of 16 activation rows, weight tile) come from the
 // expert offsets on the device; empty experts have none.  Every mbarrier
-// wait is bounded.
+// wait is bounded.  Launches use programmatic stream serialization: the
+// set-up overlaps the previous kernel, and no input is read before
+// griddepcontrol.wait (a chained FC2 reads its offsets first and waits only
+// before its activation rows).
 #include <cuda.h>
 #include <cuda_runtime.h>
 
