@@ -262,13 +262,15 @@ def _ref_gemm(a, offsets, w, gw, N):
 # decode-sized segments: the swapped tensor-core kernel where the tiling fits
 # (K % 512 MX / % 256 NV), the dp4a kernel otherwise
 GEMV_CASES = [([3, 0, 1, 8, 5], 512, 7168), ([1, 1, 1, 1, 1, 1], 256, 2048), ([2, 0, 0, 7], 256, 256),
-              ([8], 4096, 256), ([1], 128, 128), ([16, 9, 0, 13], 256, 1024), ([1, 2], 384, 1024)]
+              ([8], 4096, 256), ([1], 128, 128), ([16, 9, 0, 13], 256, 1024), ([1, 2], 384, 1024),
+              ([1], 4096, 7168)]                      # the dense configuration at M = 1 (one expert)
 # tensor-core kernel cases (MX needs K % 512, NV K % 256; others take the
 # GEMV kernel with long segments, which is covered as well)
 TC_CASES = [([300, 0, 1, 129, 77], 512, 512), ([256, 128], 256, 1024), ([9, 200, 0, 0, 1000], 256, 512),
             ([130], 512, 7168), ([17, 140], 256, 768), ([40, 12], 256, 384),
             # N a multiple of 224: 224-column tiles, two accumulators
-            ([300, 0, 1, 129, 77], 448, 512), ([130, 20], 224, 2048), ([17, 600], 672, 1024)]
+            ([300, 0, 1, 129, 77], 448, 512), ([130, 20], 224, 2048), ([17, 600], 672, 1024),
+            ([64], 4096, 7168)]                       # the dense configuration at M = 64 (one expert)
 
 
 # the prefill tensor-core kernel runs with one CTA per 128-row tile
