@@ -20,7 +20,6 @@ enum DeviceError : unsigned int {
     kErrNone = 0,
     kErrWaitTimeout = 1u,      // an mbarrier wait exceeded its iteration cap
     kErrBadOffsets = 2u,       // offsets[E] larger than the row count
-    kErrSegmentTooLong = 4u,   // a segment longer than the GEMV row bound
 };
 
 __device__ __forceinline__ void raise_error(unsigned int e) { atomicOr(&g_device_error, e); }
@@ -121,6 +120,16 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel)
     uint32_t d;
     asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
     return d;
+}
+
+// SwiGLU element ("Moore Threads full-link adaptation of DeepSeek-V4", the
+// fused SwiGLU + quantisation step): silu(g) * u with silu(x) = x / (1 + e^-x),
+// in fp32 with IEEE-rounded add, divide and multiply and CUDA's expf (2 ulp),
+// so every kernel that computes h (fused epilogues and the standalone step)
+// gives the same bits for the same g and u
+__device__ __forceinline__ float swiglu_f32(float g, float u)
+{
+    return __fmul_rn(__fdiv_rn(g, __fadd_rn(1.0f, expf(-g))), u);
 }
 
 // internal epilogue mode: FC2 with the weighted combine fused (adds into the

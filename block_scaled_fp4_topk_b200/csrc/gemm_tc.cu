@@ -915,8 +915,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
                     float h[32];
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
-                        const float g = gv[i] * gscale, u = uv[i] * gscale;
-                        h[i] = __fdividef(g * u, 1.0f + __expf(-g));    // silu(g) * u
+                        h[i] = swiglu_f32(__fmul_rn(gv[i], gscale), __fmul_rn(uv[i], gscale));
                     }
                     if (valid) {
                         if (p.h_debug) {
@@ -949,10 +948,11 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
                                     for (int i = 0; i < 16; ++i)
                                         wq[2 * hb + (i >> 3)] |= ((__float_as_uint(h[16 * hb + i]) >> 28) & 8u) << (4 * (i & 7));
                                 } else {
-                                    const float rcp = __frcp_rn(__fmul_rn(ds, gh));
+                                    const float den = __fmul_rn(ds, gh);
 #pragma unroll
                                     for (int i = 0; i < 16; i += 2)
-                                        wq[2 * hb + (i >> 3)] |= e2m1x2(h[16 * hb + i] * rcp, h[16 * hb + i + 1] * rcp)
+                                        wq[2 * hb + (i >> 3)] |= e2m1x2(__fdiv_rn(h[16 * hb + i], den),
+                                                                        __fdiv_rn(h[16 * hb + i + 1], den))
                                                                  << (4 * (i & 7));
                                 }
                                 sb[hb] = s;

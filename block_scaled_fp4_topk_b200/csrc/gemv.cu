@@ -253,7 +253,7 @@ k_gemv(const GemmArgs p)
             for (int rr = warp; rr < nr; rr += NW) {
                 const float g = red[(0 * MAXR + rr) * 32 + lane];
                 const float u = red[(1 * MAXR + rr) * 32 + lane];
-                const float h = __fmul_rn(__fdiv_rn(g, __fadd_rn(1.0f, expf(-g))), u);
+                const float h = swiglu_f32(g, u);
                 const int64_t row = rg + rr;
                 const int col = blockIdx.x * 32 + lane;
                 if (p.h_debug) p.h_debug[row * I + col] = h;

@@ -28,7 +28,8 @@
 // wait is bounded.  Launches use programmatic stream serialization: the
 // set-up overlaps the previous kernel, and no input is read before
 // griddepcontrol.wait (a chained FC2 reads its offsets first and waits only
-// before its activation rows).
+// before its activation rows).  A launch releases the next kernel on the
+// stream only after its own wait has returned.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -174,9 +175,6 @@ k_gemv_tc(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUt
     int32_t* soff = prefix + C::EARR_BYTES / 4;      // the expert offsets, staged once
     float* xred = reinterpret_cast<float*>(soff + C::EARR_BYTES / 4);   // split: [128][16] partial sums
 
-    // a chained launch of the next kernel on the stream may start now: its
-    // CTAs take the SMs this grid's CTAs leave
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int E = p.E;
     const int64_t K = p.K;
@@ -216,12 +214,22 @@ k_gemv_tc(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUt
     // Every launch may begin while the previous kernel on the stream ends
     // (programmatic serialization): the set-up above touches no input, and
     // this wait holds every read of one until that kernel has finished.
-    // A chained FC2 (p.chained) reads its offsets now and waits only before
-    // its activation rows (the producers below).
-    if (!p.chained) asm volatile("griddepcontrol.wait;" ::: "memory");
+    // The next kernel on the stream is released only after this wait has
+    // returned, so when any kernel of a chain starts, every kernel before
+    // its immediate predecessor has completed.
+    // A chained FC2 (p.chained) reads its offsets now (written before its
+    // predecessor, FC1, started: complete by the rule above); its producers
+    // wait only before its activation rows, its other threads once the
+    // set-up below is done.
+    if (!p.chained) {
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    }
     // the expert offsets -> shared memory in one parallel pass (a loop of
-    // dependent global loads here cost about 2 us per launch)
-    for (int e = threadIdx.x; e <= E; e += kThreads) soff[e] = p.offsets[e];
+    // dependent global loads here cost about 2 us per launch); L2 loads, so
+    // that a chained launch, which may start before its predecessor ends,
+    // never reads a line its SM cached earlier
+    for (int e = threadIdx.x; e <= E; e += kThreads) soff[e] = __ldcg(p.offsets + e);
     if (warp == 0 && lane == 0) {
         asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&map_w) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&map_x) : "memory");
@@ -273,6 +281,13 @@ k_gemv_tc(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUt
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const int64_t nitems = *total_items;
+    if (p.chained && !((warp == 0 || warp == 8) && lane == 0)) {
+        // a chained launch: every thread but the two producers (which load
+        // weights first) waits for the previous kernel here, before any role
+        // reads an input it writes
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    }
 
     // A thread that has issued asynchronous work (TMA copies, tensor-core
     // instructions) and then waits on a barrier, or branches on anything it
@@ -312,6 +327,7 @@ k_gemv_tc(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUt
             };
             auto release_deferred = [&]() {
                 asm volatile("griddepcontrol.wait;" ::: "memory");
+                asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
                 for (uint32_t i = 0; i < ndef; ++i) load_x((uint32_t)pi + 2 * i);
                 waited = true;
             };
@@ -535,9 +551,8 @@ k_gemv_tc(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUt
                     const int col = itm.wt * 64 + 32 * q + lane;    // h column (gate row within I)
 #pragma unroll 1
                     for (int tt = 0; tt < itm.nr; ++tt) {
-                        const float g = v[tt] * gscale;
-                        const float u = xch[(q * 32 + lane) * BNT + tt] * gscale;
-                        const float h = __fdividef(g * u, 1.0f + __expf(-g));
+                        const float h = swiglu_f32(__fmul_rn(v[tt], gscale),
+                                                   __fmul_rn(xch[(q * 32 + lane) * BNT + tt], gscale));
                         const int64_t row = itm.x0 + tt;
                         if (p.h_debug) p.h_debug[row * I + col] = h;
                         uint32_t code;
@@ -555,7 +570,7 @@ k_gemv_tc(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUt
                             const uint32_t s = ue4m3_encode(__fdiv_rn(m, __fmul_rn(6.0f, gh)));
                             const float ds = ue4m3_value(s);
                             code = (ds == 0.0f) ? ((__float_as_uint(h) >> 28) & 8u)
-                                                : e2m1_code(h * __frcp_rn(__fmul_rn(ds, gh)));
+                                                : e2m1_code(__fdiv_rn(h, __fmul_rn(ds, gh)));
                             if ((lane & 15) == 0) p.oq_scales[row * (I / 16) + col / 16] = (uint8_t)s;
                         }
                         const uint32_t hi_code = __shfl_down_sync(0xffffffffu, code, 1);
@@ -642,15 +657,12 @@ static cudaError_t run_dtc(const GemmArgs& a, cudaStream_t st)
 
 // FC1 with few items (at most about two per SM: decode T = 1) splits each
 // item's K range over a CTA pair, so that no SM streams two whole items while
-// others idle.  DS4G_DTC_SPLIT=0 / 1 in the environment forces it off / on.
+// others idle.  Chosen from the shape alone.
 static bool use_split(const GemmArgs& a)
 {
     const int64_t K = a.K;
     const int npairs = (int)((ceil_div(K, 256) + 1) / 2);
     if (a.epilogue != DS4G_EPI_SWIGLU_REQUANT || npairs < 2) return false;
-    const char* env = getenv("DS4G_DTC_SPLIT");
-    if (env && env[0] == '0') return false;
-    if (env && env[0] == '1') return true;
     const int64_t wtiles = (a.N / 2) / 64;
     const int64_t experts = a.E < a.S ? a.E : a.S;       // experts that can hold rows
     return experts * wtiles <= 2 * kNumSMs;

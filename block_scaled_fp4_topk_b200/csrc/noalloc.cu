@@ -12,32 +12,38 @@
 namespace ds4g {
 
 // scratch of the multi-CTA permutation (per-chunk expert histograms), E * B
-// 32-bit counters with B = ceil(T * k / 1024); the single-CTA path used for
-// T * k <= 512 needs none
+// 32-bit counters with B = ceil(T * k / 256) (256 slots per chunk); the
+// single-CTA path used for T * k <= 512 needs none
 constexpr size_t kStaticPermuteScratchBytes = 256 * 1024;
 static __device__ __align__(256) int32_t g_permute_scratch[kStaticPermuteScratchBytes / sizeof(int32_t)];
 
 constexpr int kMaxDevices = 64;
 static void* g_scratch_ptr[kMaxDevices];
-static std::once_flag g_scratch_once[kMaxDevices];
-static cudaError_t g_scratch_err[kMaxDevices];
+static std::mutex g_scratch_mutex;
 
-// device address of the scratch array on the current device, looked up once
-// per device (the array's host-side name is only a stand-in, never a device
-// address)
+// device address of the scratch array on the current device (the array's
+// host-side name is only a stand-in, never a device address).  Looked up on
+// the first call on each device and kept only once a lookup has succeeded: a
+// lookup that fails (for example one attempted during a stream capture) is
+// reported to that caller and tried again on the next call.
 static cudaError_t static_scratch(void** out)
 {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::call_once(g_scratch_once[dev], [dev]() {
+    std::lock_guard<std::mutex> lock(g_scratch_mutex);
+    if (!g_scratch_ptr[dev]) {
         void* p = nullptr;
-        g_scratch_err[dev] = cudaGetSymbolAddress(&p, g_permute_scratch);
-        g_scratch_ptr[dev] = (g_scratch_err[dev] == cudaSuccess) ? p : nullptr;
-    });
+        e = cudaGetSymbolAddress(&p, g_permute_scratch);
+        if (e != cudaSuccess) {
+            cudaGetLastError();   // the failure is returned here, not left for the next CUDA call
+            return e;
+        }
+        g_scratch_ptr[dev] = p;
+    }
     *out = g_scratch_ptr[dev];
-    return g_scratch_err[dev];
+    return cudaSuccess;
 }
 
 }  // namespace ds4g

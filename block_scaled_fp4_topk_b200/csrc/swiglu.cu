@@ -21,7 +21,7 @@ __global__ void k_swiglu_requant(const float* __restrict__ y1, int64_t rows, int
     const int col = (int)(b * 32) + lane;
     const float g = y1[row * 2 * I + col];
     const float u = y1[row * 2 * I + I + col];
-    const float h = __fmul_rn(__fdiv_rn(g, __fadd_rn(1.0f, expf(-g))), u);
+    const float h = swiglu_f32(g, u);
     if (h_debug) h_debug[row * I + col] = h;
     uint32_t code;
     if (FMT == DS4G_MXFP4) {

@@ -142,38 +142,3 @@ class MoeLayer:
         with torch.cuda.graph(graphs[2]):
             out = self.fc2(b, T)
         return list(zip(names, graphs)), out
-
-    # -- synthetic weights -----------------------------------------------------
-    @staticmethod
-    def synthetic_weights(E, d, I, fmt, seed=0, device="cuda", rows_w1=None, chunk=8):
-        """Expert weights drawn on the device by the seeded generator
-        (W1[e] ~ N(0, 0.02) [2I][d], W2[e] ~ N(0, 0.02) [d][I]) and quantised
-        with the library's own quantiser (offline, not part of a step)."""
-        import synth
-        from synth.workloads import W_SIGMA
-        r1 = rows_w1 if rows_w1 is not None else 2 * I
-        st = torch.cuda.current_stream().cuda_stream
-        w1 = Fp4Tensor.empty(E * r1, d, fmt, device)
-        w2 = Fp4Tensor.empty(E * d, I, fmt, device)
-        if fmt == NVFP4:
-            w1.g = torch.empty(E, dtype=torch.float32, device=device)
-            w2.g = torch.empty(E, dtype=torch.float32, device=device)
-        ws = torch.empty(16, dtype=torch.uint8, device=device)
-        for dst, rows, cols, base in ((w1, r1, d, synth.STREAM_W1), (w2, d, I, synth.STREAM_W2)):
-            buf = torch.empty((chunk * rows, cols), dtype=torch.float32, device=device)
-            for e0 in range(0, E, chunk):
-                n = min(chunk, E - e0)
-                for j in range(n):
-                    synth.cuda_fill_normal_f32(buf[j * rows:(j + 1) * rows].data_ptr(), rows * cols, seed,
-                                               base + e0 + j, W_SIGMA, 0, st)
-                if fmt == NVFP4:
-                    for j in range(n):
-                        e = e0 + j
-                        part = Fp4Tensor(dst.data[e * rows:(e + 1) * rows], dst.scales[e * rows:(e + 1) * rows],
-                                         dst.g[e:e + 1], fmt)
-                        ds4g.ds4g_quantize_mx(buf[j * rows:(j + 1) * rows], fmt, out=part, workspace=ws)
-                else:
-                    part = dst.view_rows(e0 * rows, (e0 + n) * rows)
-                    ds4g.ds4g_quantize_mx(buf[:n * rows], fmt, out=part)
-            del buf
-        return w1, w2

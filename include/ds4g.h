@@ -187,8 +187,7 @@ ds4g_status ds4g_moe_dispatch(const float* logits, const void* x, int dtype, int
  *     weights as the MMA's M side (decode); with SWIGLU_REQUANT and at most
  *     about two weight tiles per SM (min(E, rows) x I / 64 <= 296) each
  *     tile's K range is split over a CTA pair whose follower sends its
- *     partial sums to the leader (DS4G_DTC_SPLIT=0 / 1 in the environment
- *     forces this off / on).  This kernel is launched with programmatic
+ *     partial sums to the leader.  This kernel is launched with programmatic
  *     stream serialization: it may start while the previous kernel on the
  *     stream ends, and reads no input before that kernel has finished;
  *   > 16 rows and the same K rule, N % 224 == 0 (NONE): tensor-core kernel
@@ -233,9 +232,15 @@ ds4g_status ds4g_grouped_gemm_fp4_combine(const ds4g_fp4* a, const int32_t* offs
  *   - with decode-sized segments the launch may start while that previous
  *     kernel still runs, so that the FC2 weights stream in while its last
  *     tiles finish.  The kernel waits for the previous kernel (programmatic
- *     dependent launch, griddepcontrol.wait) before it reads a; every other
- *     input (offsets, row_to_slot, route_w, w and out's contents) must be
- *     complete before that previous kernel started.
+ *     dependent launch, griddepcontrol.wait) before it reads a, row_to_slot,
+ *     route_w or out; it reads offsets (and w) before that wait.  So a may be
+ *     written by the previous kernel, and every other input must be written
+ *     by work that comes before that previous kernel on the stream.  The
+ *     layer's own sequence -- ds4g_moe_dispatch (offsets, row_to_slot,
+ *     route_w), then FC1 (a = h), then this call -- satisfies it: each
+ *     decode-kernel launch of this library releases the next kernel on the
+ *     stream only after it has itself waited for its predecessor, so when
+ *     this kernel starts, everything before FC1 has completed.
  * Other shapes launch the same kernels as ds4g_grouped_gemm_fp4_combine, in
  * stream order.  Arguments, results within the same bound and errors as
  * ds4g_grouped_gemm_fp4_combine. */
@@ -273,8 +278,9 @@ ds4g_status ds4g_moe_combine(const float* y2, const int32_t* slot_to_row, const 
  * whose ds4g_permute_workspace_bytes(T, k, E) exceeds it returns
  * DS4G_ERR_WORKSPACE.  The first call on a device looks the array's device
  * address up for that device (make that first call before any stream
- * capture).  All calls share the one array: calls that overlap on the GPU
- * (concurrent streams, or several host threads) race on it and must be
+ * capture); a lookup that fails returns DS4G_ERR_CUDA and is tried again on
+ * the next call.  All calls share the one array: calls that overlap on the
+ * GPU (concurrent streams, or several host threads) race on it and must be
  * serialised by the caller. */
 size_t ds4g_permute_static_max_bytes(void);
 ds4g_status ds4g_moe_permute_static(const int32_t* idx, int T, int k, int E, const ds4g_fp4* x_q,

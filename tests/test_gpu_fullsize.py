@@ -1,7 +1,7 @@
 """Parity at the full problem sizes, in the configuration the bench times
-(E = 256, top-6, d = 7168, I = 2048; MXFP4 decode T = 1 / 8, MXFP4 prefill
-T = 2048 with the skewed router bias, NVFP4 prefill T = 16384), through the
-library's C ABI with the same layer code the bench uses.
+(E = 256, top-6, d = 7168, I = 2048; MXFP4 decode T = 1 / 4 / 8, MXFP4
+prefill T = 2048 with the skewed router bias, NVFP4 prefill T = 16384),
+through the library's C ABI with the same layer code the bench uses.
 
 What is checked against the oracle, which runs its own chain from the same
 seeded inputs:
@@ -12,7 +12,18 @@ seeded inputs:
   - FC2 on sampled rows whose FP4 input matches the oracle's byte for byte
     (rows where a code legitimately rounded the other way were validated in
     the FC1 check): per-element GEMM bound;
-  - combine on sampled tokens; and for decode T = 1 the whole layer."""
+  - FC2 + combine on sampled tokens (all tokens at decode sizes; 32 at
+    prefill sizes, among them tokens of the heaviest and of a one-row
+    expert), from the GPU's own upstream tensors (its h codes and routing
+    weights): per-element bound;
+  - the whole layer on the same token sample against the oracle's own chain
+    (routing, quantisation, FC1, SwiGLU, requantisation, FC2, combine):
+    relative L2 <= 1e-2.
+And the captured decode layer (split FC1 at T = 1, plain at T = 4) replayed
+back to back with different inputs and routing on every replay, each replay
+against the oracle's chain (offsets bit-exact, output relative L2 <= 1e-2):
+routing-dependent ordering errors between the layer's kernels only show when
+the routing changes between steps."""
 import numpy as np
 import pytest
 import torch
@@ -26,9 +37,11 @@ pytestmark = pytest.mark.gpu
 
 ds4g = pytest.importorskip("block_scaled_fp4_topk_b200.ds4g")
 from block_scaled_fp4_topk_b200.layer import MoeLayer  # noqa: E402
+from bench import synthetic_weights  # noqa: E402
 
 MX, NV = oracle.MX, oracle.NV
 _LAYERS = {}
+L2_MAX = 1e-2
 
 
 def _layer(fmt):
@@ -37,7 +50,7 @@ def _layer(fmt):
             del _LAYERS[k]
         torch.cuda.empty_cache()
         wl = workloads.WORKLOADS["prefill" if fmt == MX else "prefill16k"]
-        w1, w2 = MoeLayer.synthetic_weights(wl.E, wl.d, wl.I, fmt, device=dev())
+        w1, w2 = synthetic_weights(wl.E, wl.d, wl.I, fmt, device=dev())
         _LAYERS[fmt] = MoeLayer(w1, w2, wl.E, wl.k, wl.d, wl.I, fmt, g_h=workloads.G_H)
     return _LAYERS[fmt]
 
@@ -59,11 +72,50 @@ def _h_bound(g, u, ag, au):
     dg, du = 1e-5 * ag + 1e-6, 1e-5 * au + 1e-6
     sig = 1.0 / (1.0 + np.exp(-g))
     h = g * sig * u
-    fast = (4e-6 + 2.0 ** -23 * np.abs(g)) * np.abs(h)
-    return h, np.abs(sig * (1 + g * (1 - sig))) * np.abs(u) * dg + np.abs(g * sig) * du + fast + 1e-30
+    # fp32 rounding of (g / (1 + expf(-g))) * u: expf within 2 ulp (CUDA C
+    # Programming Guide, mathematical functions appendix), add / divide /
+    # multiply IEEE round-to-nearest: at most 3.5 ulp, below 8 |h| 2^-24
+    return h, np.abs(sig * (1 + g * (1 - sig))) * np.abs(u) * dg + np.abs(g * sig) * du + 8 * np.abs(h) * 2.0 ** -24 + 1e-30
 
 
-def _run(name, rng_seed=0):
+def _chain(wl, xq, idx, w, toks, gpu=None):
+    """For the tokens `toks`, the layer output by the oracle's own chain from
+    the quantised activations xq and the routing (idx, w): FC1 of each token's
+    k rows, SwiGLU on the fp32-rounded result, requantisation, FC2, and the
+    weighted sum in fp64.  With gpu = (hq, s2r, w_gpu) (the GPU's h codes, its
+    slot -> row map and its routing weights) also FC2 + combine from those
+    upstream tensors and the per-element bound of that result.  Each expert's
+    weights are quantised once, for all sample rows routed to it."""
+    g_h = workloads.G_H if wl.fmt == NV else None
+    n = len(toks)
+    ref = np.zeros((n, wl.d))
+    up = np.zeros((n, wl.d))
+    bound = np.full((n, wl.d), 1e-7)
+    sel = idx[toks]                                   # [n][k] experts
+    for e in np.unique(sel):
+        ii, jj = np.nonzero(sel == e)                 # sample token i, slot j
+        W1, W2 = _expert_weights(wl, int(e))
+        y1, _ = oracle.expert_gemm_rows(xq, toks[ii], W1, (0, 2 * wl.I))
+        hq = oracle.quantize(oracle.swiglu(y1.astype(np.float32)), wl.fmt, g=g_h)
+        y2, _ = oracle.expert_gemm_rows(hq, np.arange(len(ii)), W2, (0, wl.d))
+        ref[ii] += w[toks[ii], jj][:, None] * y2.astype(np.float32)
+        if gpu is not None:
+            ghq, s2r, wg = gpu
+            rows = s2r[toks[ii] * wl.k + jj]
+            y2u, ab = oracle.expert_gemm_rows(ghq, rows, W2, (0, wl.d))
+            wt = wg[toks[ii], jj].astype(np.float64)[:, None]
+            up[ii] += wt * y2u
+            # FC2 bound of each row carried by its routing weight, plus the
+            # fp32 rounding of the weighted terms and of their sum
+            bound[ii] += np.abs(wt) * (1e-5 * ab + 1e-6) + 1e-6 * np.abs(wt * y2u)
+    return ref, up, bound
+
+
+def _rel_l2(got, ref):
+    return float(np.linalg.norm(got - ref) / np.linalg.norm(ref))
+
+
+def _run(name):
     wl = workloads.WORKLOADS[name]
     layer = _layer(wl.fmt)
     xb = workloads.host_x_bits(wl)
@@ -77,7 +129,23 @@ def _run(name, rng_seed=0):
     return wl, layer, xb, lg, b, hdbg, out
 
 
-@pytest.mark.parametrize("name", ["decode_t1", "decode_t8", "prefill", "prefill16k"])
+def _token_sample(wl, idx, offsets, r2s, rng, n=32):
+    """all tokens up to n; else tokens of the heaviest expert, of a one-row
+    expert (if any) and random ones, n in all"""
+    if wl.T <= n:
+        return np.arange(wl.T)
+    counts = np.diff(offsets)
+    heavy = int(np.argmax(counts))
+    picks = set(int(s) // wl.k for s in r2s[offsets[heavy]:offsets[heavy] + 2])
+    ones = np.nonzero(counts == 1)[0]
+    for e in ones[:2]:
+        picks.add(int(r2s[offsets[e]]) // wl.k)
+    rest = np.setdiff1d(np.arange(wl.T), np.array(sorted(picks)))
+    picks.update(int(t) for t in rng.choice(rest, size=n - len(picks), replace=False))
+    return np.array(sorted(picks))
+
+
+@pytest.mark.parametrize("name", ["decode_t1", "decode_t4", "decode_t8", "prefill", "prefill16k"])
 def test_fullsize_layer(name):
     wl, layer, xb, lg, b, hdbg, out = _run(name)
     rng = np.random.default_rng(123)
@@ -86,7 +154,8 @@ def test_fullsize_layer(name):
     # routing, quantisation, permutation: whole tensors, bit-exact
     idx, w = oracle.route_topk(lg, wl.k)
     assert np.array_equal(b["idx"].cpu().numpy(), idx)
-    assert np.allclose(b["w"].cpu().numpy(), w, rtol=0, atol=2e-6)
+    w_gpu = b["w"].cpu().numpy()
+    assert np.allclose(w_gpu, w, rtol=0, atol=2e-6)
     xq = oracle.quantize(x, wl.fmt)
     gxq = from_dev(b["xq"])
     assert np.array_equal(gxq.scales, xq.scales) and np.array_equal(gxq.data, xq.data)
@@ -110,7 +179,6 @@ def test_fullsize_layer(name):
     picks.update(int(e) for e in rng.choice(touched, size=min(2, len(touched)), replace=False))
     g_h = workloads.G_H if wl.fmt == NV else None
     hq_gpu = from_dev(b["hq"])
-    y2_rows, y2_ref_rows, y2_ab = [], [], []
     for e in sorted(picks):
         r0, r1 = int(offsets[e]), int(offsets[e + 1])
         rows = np.arange(r0, r1)
@@ -148,45 +216,51 @@ def test_fullsize_layer(name):
         for i in np.nonzero(same)[0]:
             assert_gemm_close(y2_gpu[i, n_cols], y2_ref[i, n_cols], y2_abs[i, n_cols], f"FC2 expert {e} row {rows[i]}")
 
-    # combine on sampled tokens, from the oracle's own FC2 rows
-    toks = rng.choice(wl.T, size=min(2, wl.T), replace=False)
-    out_gpu = out.cpu().numpy() if wl.T <= 64 else out[torch.from_numpy(toks).to(dev())].cpu().numpy()
-    for ti, t in enumerate(toks):
-        acc = np.zeros(wl.d)
-        bound = np.full(wl.d, 1e-7)
-        exact_inputs = True
-        for j in range(wl.k):
-            r = int(s2r[t * wl.k + j])
-            e = int(idx[t, j])
-            W1, W2 = _expert_weights(wl, e)
-            hrow = oracle.swiglu(oracle.expert_gemm_rows(a, np.array([r]), W1, (0, 2 * wl.I))[0].astype(np.float32))
-            hq_ref = oracle.quantize(hrow, wl.fmt, g=g_h)
-            exact_inputs &= bool(np.array_equal(hq_gpu.data[r], hq_ref.data[0]) and
-                                 np.array_equal(hq_gpu.scales[r], hq_ref.scales[0]))
-            y, yab = oracle.expert_gemm_rows(hq_ref, np.array([0]), W2, (0, wl.d))
-            acc += w[t, j] * y[0].astype(np.float32)
-            # FC2 bound of the row, carried by the routing weight, plus the
-            # fp32 rounding of the weighted sum
-            bound += abs(w[t, j]) * (1e-5 * yab[0] + 1e-6) + 1e-6 * abs(w[t, j] * y[0])
-        got = out_gpu[t] if wl.T <= 64 else out_gpu[ti]
-        if exact_inputs:
-            assert np.all(np.abs(got - acc) <= bound), f"combine token {t}"
+    # the sampled tokens: FC2 + combine from the GPU's own h codes and routing
+    # weights (per element), and the whole layer against the oracle's chain
+    toks = _token_sample(wl, idx, offsets, r2s, rng)
+    assert len(toks) >= min(wl.T, 32)
+    ref, up, bound = _chain(wl, xq, idx, w, toks, gpu=(hq_gpu, s2r, w_gpu))
+    got = out[torch.from_numpy(toks).to(dev())].cpu().numpy().astype(np.float64)
+    err = np.abs(got - up)
+    assert np.all(err <= bound), f"combine: worst excess {(err - bound).max():.3e} over {len(toks)} tokens"
+    rel = _rel_l2(got, ref)
+    assert rel <= L2_MAX, f"layer relative L2 {rel:.3e} over {len(toks)} tokens"
 
 
-def test_fullsize_decode_t1_layer_l2():
-    """the whole decode layer (one token, six experts) against the oracle's
-    independent chain: relative L2 <= 1e-2"""
-    wl, layer, xb, lg, b, hdbg, out = _run("decode_t1")
-    x = synth.bf16_bits_to_f32(xb)
-    idx, w = oracle.route_topk(lg, wl.k)
-    xq = oracle.quantize(x, wl.fmt)
-    ref = np.zeros(wl.d)
-    for j in range(wl.k):
-        W1, W2 = _expert_weights(wl, int(idx[0, j]))
-        y1, _ = oracle.expert_gemm_rows(xq, np.array([0]), W1, (0, 2 * wl.I))
-        hq = oracle.quantize(oracle.swiglu(y1.astype(np.float32)), wl.fmt)
-        y2, _ = oracle.expert_gemm_rows(hq, np.array([0]), W2, (0, wl.d))
-        ref += w[0, j] * y2[0].astype(np.float32)
-    got = out.cpu().numpy()[0]
-    rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
-    assert rel <= 1e-2, rel
+@pytest.mark.parametrize("name,replays", [("decode_t1", 4), ("decode_t4", 3)])
+def test_decode_graph_replays_with_changing_routing(name, replays):
+    """The decode layer captured once (MoeLayer.capture, FC2 chained to FC1;
+    FC1 split over CTA pairs at T = 1) and replayed back to back with new
+    activations and router logits before every replay, no host sync in
+    between; each replay's offsets bit-exact and its output within relative
+    L2 1e-2 of the oracle's chain on that replay's inputs"""
+    wl = workloads.WORKLOADS[name]
+    layer = _layer(MX)
+    x = bf16_dev(workloads.host_x_bits(wl, 0))
+    lg = torch.from_numpy(workloads.host_logits(wl, 0)).to(dev())
+    graph, out = layer.capture(x, lg)
+    b = layer.buffers(wl.T, dev())
+    inputs, outs, offs = [], [], []
+    for r in range(1, replays + 1):
+        xb, lr = workloads.host_x_bits(wl, r), workloads.host_logits(wl, r)
+        inputs.append((xb, lr))
+        x.copy_(bf16_dev(xb))
+        lg.copy_(torch.from_numpy(lr).to(dev()))
+        graph.replay()
+        outs.append(out.clone())
+        offs.append(b["offsets"].clone())
+    torch.cuda.synchronize()
+    ds4g.ds4g_check_device()
+    prev = None
+    for r, ((xb, lr), o, of) in enumerate(zip(inputs, outs, offs)):
+        idx, w = oracle.route_topk(lr, wl.k)
+        offsets, _, _ = oracle.moe_permute(idx, wl.E)
+        assert np.array_equal(of.cpu().numpy(), offsets), f"replay {r}: offsets"
+        if prev is not None:
+            assert not np.array_equal(offsets, prev), "the routing did not change between replays"
+        prev = offsets
+        xq = oracle.quantize(synth.bf16_bits_to_f32(xb), wl.fmt)
+        ref, _, _ = _chain(wl, xq, idx, w, np.arange(wl.T))
+        rel = _rel_l2(o.cpu().numpy().astype(np.float64), ref)
+        assert rel <= L2_MAX, f"replay {r}: layer relative L2 {rel:.3e}"

@@ -1,10 +1,10 @@
 """ds4g_moe_permute_static -- the expert permutation for callers that cannot
 allocate device memory (not even a workspace of their own), whose scratch is
 the library's file-scope device array.  Checked through the C ABI against
-the workspace-taking ds4g_moe_permute on the same inputs, on two calls in a
-row (the array keeps the previous call's contents), on problems that take
-the multi-CTA path (the one that uses the scratch) and the single-CTA path.
-Collected last on purpose."""
+the workspace-taking ds4g_moe_permute and against the oracle's permutation of
+the same inputs, on two calls in a row (the array keeps the previous call's
+contents), on problems that take the multi-CTA path (the one that uses the
+scratch) and the single-CTA path.  Collected last on purpose."""
 import numpy as np
 import pytest
 import torch
@@ -36,6 +36,14 @@ def test_permute_static_matches_workspace_version(T, k, E):
         for r, g in zip(ref[:3], got[:3]):
             assert torch.equal(r, g), f"call {call}"
         assert torch.equal(ref[3].data, got[3].data) and torch.equal(ref[3].scales, got[3].scales)
+        # and against the oracle's permutation and gather, bit for bit
+        offs, r2s, s2r = oracle.moe_permute(idx, E)
+        assert np.array_equal(got[0].cpu().numpy(), offs), f"call {call}: offsets"
+        assert np.array_equal(got[1].cpu().numpy(), r2s), f"call {call}: row_to_slot"
+        assert np.array_equal(got[2].cpu().numpy(), s2r), f"call {call}: slot_to_row"
+        a = oracle.gather_rows(xq, r2s, k)
+        assert np.array_equal(got[3].data.cpu().numpy(), a.data) and np.array_equal(got[3].scales.cpu().numpy(),
+                                                                                   a.scales), f"call {call}: rows"
 
 
 def test_permute_static_rejects_too_large():
