@@ -7,8 +7,10 @@ It is a numpy front end over the plain-C fp64 oracle in ``ds4g_oracle.c``
 the CUDA library.
 
 Formats: ``MX`` = E2M1 + UE8M0 scale per 32 along K; ``NV`` = E2M1 + UE4M3
-scale per 16 along K + an fp32 tensor scale ``g``.  An FP4 tensor is the tuple
-``Fp4(data uint8 [rows][K/2], scales uint8 [rows][K/blk], g float, fmt)``.
+scale per 16 along K + an fp32 tensor scale ``g``; ``MX8`` = E4M3 (one byte
+per element) + UE8M0 scale per 32 (the FP8 activations of the FP8 x FP4
+variant).  A block-scaled tensor is the tuple
+``Fp4(data uint8 [rows][K/2] (K for MX8), scales uint8 [rows][K/blk], g float, fmt)``.
 """
 import ctypes
 from collections import namedtuple
@@ -19,7 +21,16 @@ from . import build as _build
 
 MX = 0
 NV = 1
-BLOCK = {MX: 32, NV: 16}
+MX8 = 2
+BLOCK = {MX: 32, NV: 16, MX8: 32}
+
+
+def _row_bytes(fmt, K):
+    return K if fmt == MX8 else K // 2
+
+
+def _K_of(t):
+    return t.data.shape[1] if t.fmt == MX8 else t.data.shape[1] * 2
 
 Fp4 = namedtuple("Fp4", ["data", "scales", "g", "fmt"])
 
@@ -44,6 +55,15 @@ def _L():
         L.orc_ue4m3_encode.argtypes = [dbl]
         L.orc_lut_decode_check.restype = i32
         L.orc_lut_decode_check.argtypes = []
+        L.orc_e4m3_decode.restype = dbl
+        L.orc_e4m3_decode.argtypes = [i32]
+        L.orc_e4m3_encode.restype = i32
+        L.orc_e4m3_encode.argtypes = [dbl]
+        L.orc_quantize_mx8.argtypes = [vp, i64, i64, vp, vp]
+        L.orc_quantize_mx8.restype = None
+        L.orc_expert_gemm_rows_mixed.argtypes = [vp, vp, dbl, i32, vp, i64, vp, vp, dbl, i32, i32, i32, i64, vp,
+                                                 vp]
+        L.orc_expert_gemm_rows_mixed.restype = None
         L.orc_quantize_mx.argtypes = [vp, i64, i64, vp, vp]
         L.orc_quantize_nv.argtypes = [vp, i64, i64, vp, vp, vp, vp]
         L.orc_dequantize.argtypes = [vp, vp, i32, dbl, i64, i64, vp]
@@ -97,6 +117,14 @@ def lut_decode_check():
     return _L().orc_lut_decode_check()
 
 
+def e4m3_decode(code):
+    return _L().orc_e4m3_decode(int(code))
+
+
+def e4m3_encode(y):
+    return _L().orc_e4m3_encode(float(y))
+
+
 # ---- quantisation ----------------------------------------------------------
 
 def quantize(x, fmt, g=None):
@@ -104,8 +132,11 @@ def quantize(x, fmt, g=None):
     x = _c(x, np.float32)
     rows, K = x.shape
     blk = BLOCK[fmt]
-    data = np.zeros((rows, K // 2), np.uint8)
+    data = np.zeros((rows, _row_bytes(fmt, K)), np.uint8)
     scales = np.zeros((rows, K // blk), np.uint8)
+    if fmt == MX8:
+        _L().orc_quantize_mx8(_p(x), rows, K, _p(data), _p(scales))
+        return Fp4(data, scales, 1.0, MX8)
     if fmt == MX:
         _L().orc_quantize_mx(_p(x), rows, K, _p(data), _p(scales))
         return Fp4(data, scales, 1.0, MX)
@@ -117,7 +148,7 @@ def quantize(x, fmt, g=None):
 
 def dequantize(t):
     rows = t.data.shape[0]
-    K = t.data.shape[1] * 2
+    K = _K_of(t)
     out = np.empty((rows, K), np.float64)
     _L().orc_dequantize(_p(_c(t.data, np.uint8)), _p(_c(t.scales, np.uint8)), t.fmt, float(t.g),
                         rows, K, _p(out))
@@ -149,7 +180,7 @@ def moe_permute(idx, E):
 def gather_rows(t, row_to_slot, k):
     data = _c(t.data, np.uint8)
     scales = _c(t.scales, np.uint8)
-    K = data.shape[1] * 2
+    K = _K_of(t)
     r2s = _c(row_to_slot, np.int32)
     S = r2s.shape[0]
     od = np.zeros((S, data.shape[1]), np.uint8)
@@ -184,12 +215,16 @@ def expert_gemm_rows(a, rows, w_e, cols):
     ad, as_ = _c(a.data, np.uint8), _c(a.scales, np.uint8)
     wd, ws = _c(w_e.data, np.uint8), _c(w_e.scales, np.uint8)
     rows = _c(rows, np.int64)
-    K = ad.shape[1] * 2
+    K = _K_of(a)
     c0, c1 = cols
     out = np.empty((rows.shape[0], c1 - c0))
     ab = np.empty((rows.shape[0], c1 - c0))
-    _L().orc_expert_gemm_rows(_p(ad), _p(as_), float(a.g), _p(rows), rows.shape[0], _p(wd), _p(ws),
-                              float(w_e.g), c0, c1, K, a.fmt, _p(out), _p(ab))
+    if a.fmt == w_e.fmt:
+        _L().orc_expert_gemm_rows(_p(ad), _p(as_), float(a.g), _p(rows), rows.shape[0], _p(wd), _p(ws),
+                                  float(w_e.g), c0, c1, K, a.fmt, _p(out), _p(ab))
+    else:
+        _L().orc_expert_gemm_rows_mixed(_p(ad), _p(as_), float(a.g), a.fmt, _p(rows), rows.shape[0], _p(wd),
+                                        _p(ws), float(w_e.g), w_e.fmt, c0, c1, K, _p(out), _p(ab))
     return out, ab
 
 

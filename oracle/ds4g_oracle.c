@@ -9,7 +9,11 @@
 #include <stdlib.h>
 #include <string.h>
 
-enum { ORC_MX = 0, ORC_NV = 1 };
+enum { ORC_MX = 0, ORC_NV = 1, ORC_MX8 = 2 };
+
+/* bytes of one row of K elements, and its block length, per format */
+static int64_t row_bytes(int fmt, int64_t K) { return fmt == ORC_MX8 ? K : K / 2; }
+static int block_of(int fmt) { return fmt == ORC_NV ? 16 : 32; }
 
 /* ---------------------------------------------------------------------------
  * E2M1 element, [P1] sec. 1: 1 sign bit, 2 exponent bits, 1 mantissa bit,
@@ -34,6 +38,7 @@ int orc_e2m1_encode(double y)
     static const double grid[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
     int sign = signbit(y) ? 8 : 0;
     double a = fabs(y);
+    if (a >= 6.0) return sign | 7;    /* 6 is the nearest value to anything beyond it */
     int best = 0;
     double best_d = INFINITY;
     for (int c = 0; c < 8; ++c) {
@@ -68,6 +73,7 @@ double orc_ue4m3_decode(int b)
 /* Nearest finite UE4M3 value to r >= 0, ties to the even code, saturating. */
 int orc_ue4m3_encode(double r)
 {
+    if (r >= 448.0) return 0x7E;      /* saturation, as for the elements */
     int best = 0;
     double best_d = INFINITY;
     for (int c = 0; c <= 0x7E; ++c) {
@@ -93,6 +99,43 @@ int orc_lut_decode_check(void)
         if (orc_e2m1_encode(a) != c) return 2;
     }
     return 0;
+}
+
+/* ---------------------------------------------------------------------------
+ * E4M3 element (the FP8 activations of [P2] "Step 0",
+ * m_grouped_fp8_fp4_gemm_nt_contiguous: FP8 activations x FP4 weights; the
+ * E4M3 format of [P5] sec. 1: 4 exponent bits, 3 mantissa bits): code =
+ * s*128 + e*8 + m, bias 7; e = 0 is the subnormal m * 2^-9, otherwise
+ * 2^(e-7) * (1 + m/8); e = 15, m = 7 is NaN (no infinities), so the largest
+ * finite magnitude is 0x7E = 448.
+ * ------------------------------------------------------------------------- */
+double orc_e4m3_decode(int code)
+{
+    int s = (code >> 7) & 1;
+    int e = (code >> 3) & 15;
+    int m = code & 7;
+    if (e == 15 && m == 7) return NAN;
+    double mag = (e == 0) ? ldexp((double)m, -9) : ldexp(1.0 + m / 8.0, e - 7);
+    return s ? -mag : mag;
+}
+
+/* Nearest finite E4M3 value to y, ties to the even code, beyond 448 the
+ * nearest finite value (saturation); the code's sign bit is y's sign bit. */
+int orc_e4m3_encode(double y)
+{
+    int sign = signbit(y) ? 0x80 : 0;
+    double a = fabs(y);
+    if (a >= 448.0) return sign | 0x7E;   /* 448 is the nearest finite value to anything beyond it */
+    int best = 0;
+    double best_d = INFINITY;
+    for (int c = 0; c <= 0x7E; ++c) {
+        double d = fabs(a - orc_e4m3_decode(c));
+        if (d < best_d || (d == best_d && (c & 1) == 0 && (best & 1) == 1)) {
+            best = c;
+            best_d = d;
+        }
+    }
+    return sign | best;
 }
 
 /* packed byte layout, [P2] "Step 2": element k sits in byte k/2, even k in
@@ -200,15 +243,51 @@ void orc_quantize_nv(const float* x, int64_t rows, int64_t K, const float* g_in,
     }
 }
 
+/* ---------------------------------------------------------------------------
+ * MXFP8 quantisation, [OCP] sec. 6.3 with the E4M3 element: per block of 32
+ * along K, shared exponent X = floor(log2(amax)) - 8 (8 = largest E4M3
+ * exponent, 448 = 1.75 * 2^8), clamped to [-127, 127], scale byte X + 127,
+ * element code = E4M3_RNE(v * 2^-X) saturating at 448; one byte per element.
+ * ------------------------------------------------------------------------- */
+void orc_quantize_mx8(const float* x, int64_t rows, int64_t K, uint8_t* data, uint8_t* scales)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        const float* xr = x + r * K;
+        for (int64_t b = 0; b < K / 32; ++b) {
+            double amax = 0.0;
+            for (int i = 0; i < 32; ++i) {
+                double v = fabs((double)xr[b * 32 + i]);
+                if (v > amax) amax = v;
+            }
+            int X;
+            if (amax == 0.0) {
+                X = -127;
+            } else {
+                int e2;
+                frexp(amax, &e2);          /* amax = f * 2^e2, f in [0.5, 1) */
+                X = (e2 - 1) - 8;
+                if (X < -127) X = -127;
+                if (X > 127) X = 127;
+            }
+            scales[r * (K / 32) + b] = (uint8_t)(X + 127);
+            for (int i = 0; i < 32; ++i)
+                data[r * K + b * 32 + i] = (uint8_t)orc_e4m3_encode(ldexp((double)xr[b * 32 + i], -X));
+        }
+    }
+}
+
 void orc_dequantize(const uint8_t* data, const uint8_t* scales, int fmt, double g,
                     int64_t rows, int64_t K, double* out)
 {
-    int blk = (fmt == ORC_MX) ? 32 : 16;
+    int blk = block_of(fmt);
     for (int64_t r = 0; r < rows; ++r) {
         for (int64_t k = 0; k < K; ++k) {
             int sb = scales[r * (K / blk) + k / blk];
-            double sc = (fmt == ORC_MX) ? orc_ue8m0_decode(sb) : orc_ue4m3_decode(sb) * g;
-            out[r * K + k] = orc_e2m1_decode(get_nibble(data + r * (K / 2), k)) * sc;
+            double sc = (fmt == ORC_NV) ? orc_ue4m3_decode(sb) * g : orc_ue8m0_decode(sb);
+            double v = (fmt == ORC_MX8) ? orc_e4m3_decode(data[r * K + k])
+                                        : orc_e2m1_decode(get_nibble(data + r * (K / 2), k));
+            out[r * K + k] = v * sc;
         }
     }
 }
@@ -276,10 +355,11 @@ void orc_gather_rows(const uint8_t* src_data, const uint8_t* src_scales, int64_t
                      const int32_t* row_to_slot, int64_t S, int k,
                      uint8_t* dst_data, uint8_t* dst_scales)
 {
-    int blk = (fmt == ORC_MX) ? 32 : 16;
+    int blk = block_of(fmt);
+    int64_t rb = row_bytes(fmt, K);
     for (int64_t r = 0; r < S; ++r) {
         int64_t t = row_to_slot[r] / k;
-        memcpy(dst_data + r * (K / 2), src_data + t * (K / 2), (size_t)(K / 2));
+        memcpy(dst_data + r * rb, src_data + t * rb, (size_t)rb);
         memcpy(dst_scales + r * (K / blk), src_scales + t * (K / blk), (size_t)(K / blk));
     }
 }
@@ -294,8 +374,7 @@ void orc_gather_rows(const uint8_t* src_data, const uint8_t* src_scales, int64_t
 static void decode_row(const uint8_t* data, const uint8_t* scales, int64_t row, int64_t K,
                        int fmt, double* out)
 {
-    orc_dequantize(data + row * (K / 2), scales + row * (K / (fmt == ORC_MX ? 32 : 16)), fmt,
-                   1.0, 1, K, out);
+    orc_dequantize(data + row * row_bytes(fmt, K), scales + row * (K / block_of(fmt)), fmt, 1.0, 1, K, out);
 }
 
 void orc_expert_gemm_rows(const uint8_t* a_data, const uint8_t* a_scales, double g_a,
@@ -304,16 +383,30 @@ void orc_expert_gemm_rows(const uint8_t* a_data, const uint8_t* a_scales, double
                           int n_begin, int n_end, int64_t K, int fmt,
                           double* out, double* abssum)
 {
+    orc_expert_gemm_rows_mixed(a_data, a_scales, g_a, fmt, rows, nrows, w_e_data, w_e_scales, g_w, fmt,
+                               n_begin, n_end, K, out, abssum);
+}
+
+/* The same with activations and weights in their own formats: the FP8
+ * activation x FP4 weight GEMM of [P2] "Step 0" (a_fmt MX8, w_fmt MX).  A
+ * product of an E4M3 and an E2M1 value with their power-of-two scales has at
+ * most 6 significant bits, so it is exact in fp64 as well. */
+void orc_expert_gemm_rows_mixed(const uint8_t* a_data, const uint8_t* a_scales, double g_a, int a_fmt,
+                                const int64_t* rows, int64_t nrows,
+                                const uint8_t* w_e_data, const uint8_t* w_e_scales, double g_w, int w_fmt,
+                                int n_begin, int n_end, int64_t K, double* out, double* abssum)
+{
     int ncols = n_end - n_begin;
+    int fmt = w_fmt;
     double* arows = (double*)malloc(sizeof(double) * (size_t)(nrows * K));
-    for (int64_t i = 0; i < nrows; ++i) decode_row(a_data, a_scales, rows[i], K, fmt, arows + i * K);
-    double gg = (fmt == ORC_NV) ? g_a * g_w : 1.0;
+    for (int64_t i = 0; i < nrows; ++i) decode_row(a_data, a_scales, rows[i], K, a_fmt, arows + i * K);
+    double gg = (a_fmt == ORC_NV ? g_a : 1.0) * (w_fmt == ORC_NV ? g_w : 1.0);
 #pragma omp parallel
     {
         double* wrow = (double*)malloc(sizeof(double) * (size_t)K);
 #pragma omp for schedule(dynamic, 4)
         for (int n = n_begin; n < n_end; ++n) {
-            decode_row(w_e_data, w_e_scales, n, K, fmt, wrow);
+            decode_row(w_e_data, w_e_scales, n, K, w_fmt, wrow);
             for (int64_t i = 0; i < nrows; ++i) {
                 const double* ar = arows + i * K;
                 double acc = 0.0, aacc = 0.0;
@@ -338,7 +431,7 @@ void orc_grouped_gemm(const uint8_t* a_data, const uint8_t* a_scales, double g_a
                       int64_t row_begin, int64_t row_end, int n_begin, int n_end,
                       double* out, double* abssum)
 {
-    int blk = (fmt == ORC_MX) ? 32 : 16;
+    int blk = block_of(fmt);
     int ncols = n_end - n_begin;
     for (int e = 0; e < E; ++e) {
         int64_t lo = offsets[e] > row_begin ? offsets[e] : row_begin;

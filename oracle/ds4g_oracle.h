@@ -52,6 +52,10 @@
 extern "C" {
 #endif
 
+/* formats: 0 = MXFP4 (E2M1 + UE8M0 per 32), 1 = NVFP4 (E2M1 + UE4M3 per 16
+ * + tensor scale), 2 = MXFP8 (E4M3 + UE8M0 per 32, one byte per element;
+ * the FP8 activations of the FP8 x FP4 variant) */
+
 /* element / scale codecs */
 double orc_e2m1_decode(int code);
 int orc_e2m1_encode(double y);          /* RNE on the E2M1 grid, sign kept, saturating */
@@ -59,11 +63,14 @@ double orc_ue8m0_decode(int b);
 double orc_ue4m3_decode(int b);         /* unsigned E4M3: bias 7, subnormal m*2^-9 */
 int orc_ue4m3_encode(double r);         /* RNE over the 127 finite codes, saturating at 448 */
 int orc_lut_decode_check(void);         /* 16-entry-table decode == field decode, 0 = ok */
+double orc_e4m3_decode(int code);       /* E4M3: bias 7, subnormal m*2^-9, 0x7F / 0xFF NaN, max 448 */
+int orc_e4m3_encode(double y);          /* RNE over the finite codes, sign kept, saturating at 448 */
 
 /* quantisation of fp32 values (bf16 inputs are widened exactly first) */
 void orc_quantize_mx(const float* x, int64_t rows, int64_t K, uint8_t* data, uint8_t* scales);
 void orc_quantize_nv(const float* x, int64_t rows, int64_t K, const float* g_in,
                      uint8_t* data, uint8_t* scales, float* g_out);
+void orc_quantize_mx8(const float* x, int64_t rows, int64_t K, uint8_t* data, uint8_t* scales);
 void orc_dequantize(const uint8_t* data, const uint8_t* scales, int fmt, double g,
                     int64_t rows, int64_t K, double* out);
 
@@ -95,6 +102,13 @@ void orc_expert_gemm_rows(const uint8_t* a_data, const uint8_t* a_scales, double
                           const uint8_t* w_e_data, const uint8_t* w_e_scales, double g_w,
                           int n_begin, int n_end, int64_t K, int fmt,
                           double* out, double* abssum);
+
+/* the same with the activations and the weights each in its own format
+ * (FP8 activations x FP4 weights: a_fmt 2, w_fmt 0) */
+void orc_expert_gemm_rows_mixed(const uint8_t* a_data, const uint8_t* a_scales, double g_a, int a_fmt,
+                                const int64_t* rows, int64_t nrows,
+                                const uint8_t* w_e_data, const uint8_t* w_e_scales, double g_w, int w_fmt,
+                                int n_begin, int n_end, int64_t K, double* out, double* abssum);
 
 /* SwiGLU on fp32 FC1 outputs: h[r][i] = fp32(silu(y1[r][i]) * y1[r][I + i]) */
 void orc_swiglu(const float* y1, int64_t rows, int I, float* h);

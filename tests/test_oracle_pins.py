@@ -368,3 +368,115 @@ def test_layer_reduces_to_dense_chain():
     Hq = golden_dequant(oracle.quantize(h, oracle.MX))
     y2 = (Hq @ golden_dequant(w2).T).astype(np.float32)
     assert np.allclose(res["out"], y2.astype(np.float64), rtol=1e-6, atol=1e-9)
+
+
+# ---- FP8 (E4M3) activations: the MXFP8 format of the FP8 x FP4 variant ------
+
+def test_e4m3_against_torch_float8():
+    """all 256 codes decode as torch's float8_e4m3fn; every finite code
+    re-encodes to itself (sign of zero kept); the RNE encode of in-range fp32
+    values agrees with torch's conversion; beyond 448 the encode saturates"""
+    codes = np.arange(256, dtype=np.uint8)
+    tv = torch.from_numpy(codes).view(torch.float8_e4m3fn).double().numpy()
+    for c in range(256):
+        v = oracle.e4m3_decode(c)
+        if np.isnan(tv[c]):
+            assert np.isnan(v) and c in (0x7F, 0xFF)
+            continue
+        assert v == tv[c] and np.signbit(v) == np.signbit(tv[c])
+        assert oracle.e4m3_encode(v) == c
+    rng = np.random.default_rng(5)
+    r = np.concatenate([rng.uniform(-448, 448, 4000), rng.choice([-1, 1], 4000) * np.exp(rng.uniform(-14, 6, 4000)),
+                        rng.normal(0, 1e-3, 1000)]).astype(np.float32)
+    ref = torch.from_numpy(r).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([oracle.e4m3_encode(float(v)) for v in r])
+    assert np.array_equal(got, ref)
+    # saturation: 464 is halfway between 448 and the NaN code's 480, so the
+    # nearest finite value is 448 either way
+    assert oracle.e4m3_encode(464.0) == 0x7E and oracle.e4m3_encode(1e6) == 0x7E
+    assert oracle.e4m3_encode(-1e30) == 0xFE and oracle.e4m3_encode(-0.0) == 0x80
+
+
+def test_mx8_block_cases():
+    for line in _read("mx8_block_cases.txt"):
+        vals, sbyte, codes = (p.strip() for p in line.split(";"))
+        v = np.zeros((1, 32), np.float32)
+        listed = np.array([float(t) for t in vals.split()], np.float32)
+        v[0, :len(listed)] = listed
+        q = oracle.quantize(v, oracle.MX8)
+        assert q.data.shape == (1, 32) and q.scales.shape == (1, 1)
+        assert int(q.scales[0, 0]) == int(sbyte), line
+        assert [int(c) for c in q.data[0, :len(listed)]] == [int(c, 16) for c in codes.split()], line
+
+
+def test_mx8_quantize_matches_independent_restatement():
+    """numpy restatement: X from np.frexp, codes from torch's E4M3 conversion
+    of the scaled values clipped to the largest finite magnitude"""
+    x = synth.normal_f32((8, 256), seed=0, stream=93, sigma=2.0)
+    x[0, :32] = 0.0
+    x[1, 32:64] *= 1e-30
+    x[2, 64] = 1e30
+    q = oracle.quantize(x, oracle.MX8)
+    for r in range(8):
+        for b in range(8):
+            v = x[r, b * 32:(b + 1) * 32]
+            amax = np.abs(v).max()
+            X = -127 if amax == 0 else int(np.clip(np.frexp(amax)[1] - 1 - 8, -127, 127))
+            assert q.scales[r, b] == X + 127
+            y = np.clip(np.ldexp(v.astype(np.float64), -X), -448, 448).astype(np.float32)
+            ref = torch.from_numpy(y).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+            assert np.array_equal(q.data[r, b * 32:(b + 1) * 32], ref)
+
+
+def test_quantize_laws_mx8():
+    x = synth.normal_f32((16, 512), seed=0, stream=92, sigma=3.0)
+    q = oracle.quantize(x, oracle.MX8)
+    sc = np.ldexp(1.0, np.repeat(q.scales.astype(np.int64), 32, axis=1) - 127)
+    deq = torch.from_numpy(q.data).view(torch.float8_e4m3fn).double().numpy() * sc
+    assert np.array_equal(deq, oracle.dequantize(q))
+    q2 = oracle.quantize(deq.astype(np.float32), oracle.MX8)
+    assert np.array_equal(oracle.dequantize(q2), deq)
+    # error within half an E4M3 step (3 mantissa bits: step 2^(e-10) of the
+    # scaled value, or the subnormal step 2^-9) unless saturated
+    y = np.abs(x.astype(np.float64)) / sc
+    e = np.floor(np.log2(np.maximum(y, 2.0 ** -6)))
+    step = np.ldexp(1.0, (e - 3).astype(np.int64)) * sc
+    err = np.abs(x - deq)
+    sat = (q.data & 0x7F) == 0x7E
+    assert np.all((err <= 0.5 * step * (1 + 1e-9)) | sat)
+
+
+@pytest.mark.parametrize("K", [64, 128])
+def test_gemm_mixed_fp8_fp4_bruteforce_tiny(K):
+    """FP8 (MXFP8) activations x FP4 (MXFP4) weights: each product of an E4M3
+    and an E2M1 value with power-of-two scales is exact in fp64, so the
+    result equals numpy's matmul of the dequantised operands bit for bit"""
+    N = 8
+    a = synth.normal_f32((5, K), seed=0, stream=91, sigma=1.0)
+    w = synth.normal_f32((N, K), seed=0, stream=90, sigma=0.5)
+    aq, wq = oracle.quantize(a, oracle.MX8), oracle.quantize(w, oracle.MX)
+    out, ab = oracle.expert_gemm_rows(aq, np.arange(5), wq, (0, N))
+    A = torch.from_numpy(aq.data).view(torch.float8_e4m3fn).double().numpy() * \
+        np.ldexp(1.0, np.repeat(aq.scales.astype(np.int64), 32, axis=1) - 127)
+    W = golden_dequant(wq, with_g=False)
+    assert np.array_equal(out, A @ W.T)
+    assert np.array_equal(ab, np.abs(A) @ np.abs(W).T)
+
+
+def test_gather_mx8_rows():
+    x = synth.normal_f32((5, 128), seed=0, stream=89, sigma=1.0)
+    q = oracle.quantize(x, oracle.MX8)
+    r2s = np.array([4, 0, 9, 2, 7, 5], np.int32)        # k = 2: token = slot // 2
+    g = oracle.gather_rows(q, r2s, 2)
+    assert np.array_equal(g.data, q.data[r2s // 2]) and np.array_equal(g.scales, q.scales[r2s // 2])
+
+
+def test_encoders_saturate_far_beyond_the_range():
+    """the nearest representable value to anything beyond the largest finite
+    one is that value, also where the distances themselves round (|y| near
+    1e30 and beyond)"""
+    for y in (6.0, 7.0, 1e10, 1e30, 1e300):
+        assert oracle.e2m1_encode(y) == 0x7 and oracle.e2m1_encode(-y) == 0xF
+    for y in (448.0, 1e10, 1e30, 1e300):
+        assert oracle.e4m3_encode(y) == 0x7E and oracle.e4m3_encode(-y) == 0xFE
+        assert oracle.ue4m3_encode(y) == 0x7E
