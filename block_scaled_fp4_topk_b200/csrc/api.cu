@@ -13,7 +13,7 @@ using namespace ds4g;
 static inline cudaStream_t S(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 static inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 static inline ds4g_status cuda_status(cudaError_t e) { return e == cudaSuccess ? DS4G_OK : DS4G_ERR_CUDA; }
-static inline int block_of(int fmt) { return fmt == DS4G_MXFP4 ? 32 : 16; }
+static inline int block_of(int fmt) { return fmt == DS4G_NVFP4 ? 16 : 32; }
 
 static ds4g_status check_fp4(const ds4g_fp4* t, int64_t rows, int64_t K, int fmt, bool need_g)
 {
@@ -67,7 +67,7 @@ size_t ds4g_quantize_workspace_bytes(int fmt, int has_g_in)
 ds4g_status ds4g_quantize_mx(const void* x, int dtype, int64_t rows, int64_t K, int fmt, const float* g_in,
                              ds4g_fp4* out, void* workspace, size_t ws_bytes, void* stream)
 {
-    if (fmt != DS4G_MXFP4 && fmt != DS4G_NVFP4) return DS4G_ERR_INVALID_ARG;
+    if (fmt != DS4G_MXFP4 && fmt != DS4G_NVFP4 && fmt != DS4G_MXFP8) return DS4G_ERR_INVALID_ARG;
     if (dtype != DS4G_BF16 && dtype != DS4G_F32) return DS4G_ERR_INVALID_ARG;
     if (rows < 0 || K <= 0) return DS4G_ERR_SHAPE;
     if (K % 64 != 0) return DS4G_ERR_SHAPE;
@@ -167,22 +167,29 @@ static ds4g_status grouped_gemm(const ds4g_fp4* a, const int32_t* offsets, int E
 {
     if (!a || !w || !offsets || E < 1 || N < 1 || max_rows_per_expert < 0) return DS4G_ERR_INVALID_ARG;
     const int fmt = a->fmt;
-    if (fmt != DS4G_MXFP4 && fmt != DS4G_NVFP4) return DS4G_ERR_INVALID_ARG;
+    if (fmt != DS4G_MXFP4 && fmt != DS4G_NVFP4 && fmt != DS4G_MXFP8) return DS4G_ERR_INVALID_ARG;
     const int64_t K = a->K;
     if (K <= 0 || K % 64 != 0) return DS4G_ERR_SHAPE;
     ds4g_status st = check_fp4(a, a->rows, K, fmt, true);
     if (st != DS4G_OK) return st;
-    st = check_fp4(w, (int64_t)E * N, K, fmt, true);
+    // FP8 (MXFP8) activations multiply MXFP4 weights (routed experts) or
+    // MXFP8 weights (the shared expert); FP4 activations, weights of their own
+    // format
+    if (fmt == DS4G_MXFP8 && w->fmt != DS4G_MXFP4 && w->fmt != DS4G_MXFP8) return DS4G_ERR_SHAPE;
+    st = check_fp4(w, (int64_t)E * N, K, fmt == DS4G_MXFP8 ? w->fmt : fmt, true);
     if (st != DS4G_OK) return st;
+    const int mode = (fmt == DS4G_MXFP8 && w->fmt == DS4G_MXFP8) ? kFmtFp8Fp8 : fmt;   // the kernel's operand mode
     // kernel choice: decode-sized segments (<= 16 rows) take the swapped
     // tensor-core kernel (weights as the MMA's M side) when the tiling fits;
     // longer segments the 128 x 224 / 128 x 256 tensor-core kernel; shapes neither fits
-    // take the dp4a GEMV kernel (any segment length)
+    // take the dp4a GEMV kernel (any segment length).  FP8 activations run on
+    // the 128-row tensor-core kernel at every segment length.
     const bool swiglu = epilogue == DS4G_EPI_SWIGLU_REQUANT;
     const bool tc_shape = gemm_tc_supports(fmt, K) &&
                           (!swiglu ? (N % 256 == 0 || N % 224 == 0) : (N % 2 == 0 && (N / 2) % 32 == 0));
-    const bool dtc = max_rows_per_expert <= 16 && gemv_tc_supports(fmt, K, N, epilogue, E);
-    const bool gemv = !dtc && (max_rows_per_expert <= 8 || !tc_shape);
+    if (fmt == DS4G_MXFP8 && !tc_shape) return DS4G_ERR_SHAPE;
+    const bool dtc = fmt != DS4G_MXFP8 && max_rows_per_expert <= 16 && gemv_tc_supports(fmt, K, N, epilogue, E);
+    const bool gemv = fmt != DS4G_MXFP8 && !dtc && (max_rows_per_expert <= 8 || !tc_shape);
     const int64_t Sr = a->rows;
     if (!swiglu) {
         if (Sr > 0 && (!out || !aligned16(out))) return DS4G_ERR_INVALID_ARG;
@@ -208,7 +215,7 @@ static ds4g_status grouped_gemm(const ds4g_fp4* a, const int32_t* offsets, int E
     g.w_g = w->g;
     g.N = N;
     g.K = K;
-    g.fmt = fmt;
+    g.fmt = mode;
     g.epilogue = epilogue;
     g.out = out;
     g.oq_data = out_q ? out_q->data : nullptr;
@@ -220,6 +227,7 @@ static ds4g_status grouped_gemm(const ds4g_fp4* a, const int32_t* offsets, int E
     g.route_w = route_w;
     g.topk = k;
     g.chained = chained ? 1 : 0;
+    g.band_tiles = 0;
     if (epilogue == kEpiCombine && T > 0 && !chained) {
         cudaError_t e = cudaMemsetAsync(out, 0, sizeof(float) * (size_t)T * N, S(stream));
         if (e != cudaSuccess) return DS4G_ERR_CUDA;

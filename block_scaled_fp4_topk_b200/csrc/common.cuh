@@ -59,8 +59,19 @@ __device__ __forceinline__ uint32_t e2m1x2(float lo, float hi)
     return d;
 }
 
-// MX shared exponent X = floor(log2(amax)) - 2, clamped to [-127, 127]
-// (OCP MX rule with the E2M1 element's largest exponent 2), from the bits.
+// Two values as E4M3 bytes with the hardware conversion (round to nearest
+// even, saturating to +-448, sign kept): low byte = lo, high byte = hi.
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi)
+{
+    uint16_t d;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(d) : "f"(hi), "f"(lo));
+    return d;
+}
+
+// MX shared exponent X = floor(log2(amax)) - EMAX, clamped to [-127, 127]
+// (OCP MX rule; EMAX is the element's largest exponent: 2 for E2M1, 8 for
+// E4M3), from the bits.
+template <int EMAX = 2>
 __device__ __forceinline__ int mx_shared_exp(float amax)
 {
     uint32_t b = __float_as_uint(amax);
@@ -73,7 +84,7 @@ __device__ __forceinline__ int mx_shared_exp(float amax)
     } else {
         fl = ef - 127;
     }
-    int X = fl - 2;
+    int X = fl - EMAX;
     return X < -127 ? -127 : (X > 127 ? 127 : X);
 }
 
@@ -123,14 +134,26 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel)
 }
 
 // SwiGLU element ("Moore Threads full-link adaptation of DeepSeek-V4", the
-// fused SwiGLU + quantisation step): silu(g) * u with silu(x) = x / (1 + e^-x),
-// in fp32 with IEEE-rounded add, divide and multiply and CUDA's expf (2 ulp),
-// so every kernel that computes h (fused epilogues and the standalone step)
-// gives the same bits for the same g and u
+// fused SwiGLU + quantisation step): silu(g) * u = g u / (1 + e^-g) in fp32
+// with the hardware's fast exponential and division (__expf: at most
+// 2 + floor(1.173 |x|) ulp; __fdividef: at most 2 ulp for divisors in
+// [2^-126, 2^126]; CUDA C Programming Guide, intrinsic functions), so h is
+// within (5 + 1.173 |g|) 2^-23 |h| of silu(g) u for the fp32 g, u it gets.
+// The IEEE-rounded form costs a fifth of the prefill FC1 kernel's time
+// (measured), because this epilogue runs between two tiles' mainloops.
+// Every kernel that computes h (fused epilogues and the standalone step) uses
+// this one function, so they give the same bits for the same g and u.
 __device__ __forceinline__ float swiglu_f32(float g, float u)
 {
-    return __fmul_rn(__fdiv_rn(g, __fadd_rn(1.0f, expf(-g))), u);
+    return __fdividef(__fmul_rn(g, u), __fadd_rn(1.0f, __expf(-g)));
 }
+
+// internal GEMM operand mode: MXFP8 activations with MXFP8 weights (the
+// shared expert's FP8 weights); DS4G_MXFP8 as a GEMM mode means MXFP8
+// activations with MXFP4 weights
+constexpr int kFmtFp8Fp8 = 3;
+// FP8 (E4M3) activations, either weight format
+__host__ __device__ constexpr bool fp8_act(int fmt) { return fmt == DS4G_MXFP8 || fmt == kFmtFp8Fp8; }
 
 // internal epilogue mode: FC2 with the weighted combine fused (adds into the
 // token outputs instead of storing per-row results)

@@ -8,19 +8,23 @@
 // practice", "Step 0" (each expert's rows form one segment).  The page's
 // kernel is the warp-level mma.sync m16n8k64 form of sm_12x; on sm_100a the
 // same math is tcgen05.mma kind::mxf4 (.block32, UE8M0) / kind::mxf4nvf4
-// (.block16, UE4M3) with the accumulator in tensor memory.
+// (.block16, UE4M3) with the accumulator in tensor memory.  FP8 activations
+// (MXFP8: E4M3 + UE8M0 per 32, the FP8 x FP4 GEMM of the same page's "Step
+// 0") run the same kernel with kind::mxf8f6f4, against MXFP4 weights (loaded
+// unpacked, one byte per element) or MXFP8 weights (a shared expert's).
 //
 // Design (one persistent CTA per SM, 384 threads, warp-specialised):
-//   warp 0   TMA producer: packed FP4 tiles of A (128 rows x 256 K) and W
-//            (256 rows x 256 K) into 128B-swizzled shared memory (4 stages),
-//            and the row-major scale bytes of 512 K (two stages) of both as
-//            16 / 32-byte row boxes (2 scale stages)
+//   warp 0   TMA producer: tiles of A (128 rows x 128 bytes of K) and W
+//            (up to 256 rows x 128 bytes) into 128B-swizzled shared memory
+//            (4 stages), and the row-major scale bytes of two (FP4) or four
+//            (FP8) K stages of both as 16 / 32-byte row boxes
 //   warp 1   MMA issuer: the stage's scale words shared -> TMEM with
-//            tcgen05.cp (32x128b.warpx4), 4 x tcgen05.mma (M128 N256 K64),
-//            tcgen05.commit releases the stage / publishes the accumulator
+//            tcgen05.cp (32x128b.warpx4), 4 x tcgen05.mma (M128, K64 FP4 or
+//            K32 FP8), tcgen05.commit releases the stage / publishes the
+//            accumulator
 //   warp 2   scale transposer: rewrites each scale stage in place from row
 //            order into the 32-line x 16-byte chunks tcgen05.cp expects
-//   warp 3   TMEM allocator
+//   warp 3   TMEM allocator (and, with two accumulators, the second issuer)
 //   warps 4-11  epilogue: two warps per TMEM lane quarter, each reading half
 //            of the tile's columns with tcgen05.ld (thread = tile row), then
 //            the fp32 store or SwiGLU + requantisation
@@ -41,10 +45,8 @@ namespace tc {
 
 constexpr int BM = 128;            // tile rows (tokens)
 constexpr int BKB = 128;           // bytes of K per stage per row (256 FP4)
-constexpr int BK = 256;            // K elements per stage
 constexpr int STAGES = 4;
 constexpr int kEpiWarps = 8;
-constexpr int kThreads = 32 * (4 + kEpiWarps);
 constexpr int A_BYTES = BM * BKB;  // 16 KB
 constexpr int kTmemCols = 512;
 constexpr int kColAcc = 0;
@@ -55,29 +57,36 @@ constexpr unsigned long long kWaitNs = 4000000000ull;
 // multiple of 224, e.g. FC2 with N = 7168) with two, so that the epilogue of
 // one tile overlaps the MMAs of the next: 2 x 224 accumulator columns plus
 // the scale columns fit the 512 TMEM columns, 2 x 256 do not.
-// CTAS: 1 = one CTA per tile (M = 128); 2 = a CTA pair per tile
-// (tcgen05 cta_group::2, M = 256): each CTA of the pair loads its own 128
-// activation rows and half of the TBN weight rows, the pair's MMA reads both
-// halves, and each CTA's tensor memory receives its own 128 rows x TBN
-// columns.  Per unit of MMA work a CTA then moves half the weight bytes
-// through its shared memory.
-template <int FMT, int TBN, int NISS, int CTAS = 1>
+template <int FMT, int TBN, int NISS>
 struct Cfg {
     static_assert(TBN == 256 || TBN == 224 || TBN == 192, "tile width");
     static_assert(NISS == 1 || (NISS == 2 && TBN < 256), "two issuers need two accumulators");
-    static_assert(CTAS == 1 || CTAS == 2, "one CTA or a CTA pair per tile");
     static constexpr int NACC = (TBN == 256) ? 1 : 2;               // accumulator buffers
     static constexpr int HALF = TBN / 2;                             // weight rows per TMA box
-    static constexpr int BMT = BM * CTAS;                            // activation rows per tile
-    static constexpr int B_BYTES = (CTAS == 1 ? TBN : HALF) * BKB;   // weight bytes per stage in this CTA
-    static constexpr int WPS = (FMT == DS4G_MXFP4) ? 2 : 4;         // 4-scale words per row per K stage
+    static constexpr int B_BYTES = TBN * BKB;                        // weight bytes per stage
+    // bytes the weight loads of a stage count on its barrier: the shared
+    // memory they fill, except for FP4 weights unpacked next to FP8
+    // activations, whose loads write only the packed half of each 16-byte
+    // chunk (the other half is a gap they leave untouched)
+    static constexpr int B_TX = (FMT == DS4G_MXFP8) ? B_BYTES / 2 : B_BYTES;
+    // K elements per K stage: 128 bytes of each operand row in shared
+    // memory, i.e. 256 FP4 elements, or 128 for FP8 activations (their FP4
+    // weight rows are unpacked to one byte per element on the way in)
+    static constexpr int KE = fp8_act(FMT) ? 128 : 256;
+    // 4-scale words per row per K stage (MX: 8 scales of 32, NV: 16 of 16,
+    // FP8 activations: 4 of 32)
+    static constexpr int WPS = (FMT == DS4G_MXFP4) ? 2 : (FMT == DS4G_NVFP4 ? 4 : 1);
+    // K stages per scale stage, so that a row's scale box is at least the
+    // 16 bytes a TMA copy moves
+    static constexpr int KPS = fp8_act(FMT) ? 4 : 2;
     // TMEM scale columns per issuer: A (4 per word) then W (8 per word)
     static constexpr int SF_COLS = 12 * WPS;
-    // scale stages, each covering two K stages (512 K): two per issuer
+    // scale stages in shared memory, each covering KPS K stages: two per issuer
     static constexpr int SF_STAGES = 2 * NISS;
     static constexpr int COL_SFA = NACC * TBN;
     static_assert(COL_SFA + NISS * SF_COLS <= 512, "TMEM columns");
-    static constexpr int SF_ROW = 2 * WPS * 4;                       // scale bytes per row per scale stage
+    static constexpr int THREADS = 32 * (4 + kEpiWarps);
+    static constexpr int SF_ROW = KPS * WPS * 4;                     // scale bytes per row per scale stage
     static constexpr int SFA_BYTES = BM * SF_ROW;                    // one scale stage of A
     static constexpr int SFB_BYTES = 256 * SF_ROW;                   // one scale stage of W (two 128-row groups)
     static constexpr int SF_BYTES = SF_STAGES * (SFA_BYTES + SFB_BYTES);
@@ -88,15 +97,11 @@ struct Cfg {
     // shared-memory bandwidth and the staging traffic slows it more than the
     // wider reductions gain (measured: FC2 0.389 -> 0.448 ms at T = 2048), so
     // that configuration stores straight from registers.
-    static constexpr bool STAGED = (TBN == 224 && NISS == 1 && CTAS == 1);
-    static constexpr int BAR_BYTES = (CTAS == 1) ? 256 : 512;        // barriers + TMEM slot + flags
+    static constexpr bool STAGED = (TBN == 224 && NISS == 1);
+    static constexpr int BAR_BYTES = 256;                            // barriers + TMEM slot + flags
     static constexpr int PREFIX_BYTES = ((kMaxE + 1) * 4 + 15) / 16 * 16;
     static constexpr int STAGE_BYTES = STAGED ? kEpiWarps * 16 * 33 * 4 : 0;
-    // data ring: 4 stages with one CTA per tile; a pair's stages are smaller,
-    // so as many as fit (at most 8)
-    static constexpr int PAIR_STAGES =
-        (232448 - 1024 - SF_BYTES - BAR_BYTES - 2 * PREFIX_BYTES - STAGE_BYTES) / (A_BYTES + B_BYTES);
-    static constexpr int NST = (CTAS == 1) ? STAGES : (PAIR_STAGES > 8 ? 8 : PAIR_STAGES);
+    static constexpr int NST = STAGES;                               // data ring
     static constexpr int DATA_BYTES = NST * (A_BYTES + B_BYTES);
     // tile prefix, then the expert offsets staged once ([E + 1] int32 each)
     static constexpr int STAGE_OFF = DATA_BYTES + SF_BYTES + BAR_BYTES + 2 * PREFIX_BYTES;
@@ -175,7 +180,7 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
         : "memory");
 }
 
-// ---- CTA-pair (cluster of two) wrappers
+// ---- cluster (CTA pair) wrappers, used by the decode kernel's split mode
 __device__ __forceinline__ uint32_t cluster_ctarank()
 {
     uint32_t r;
@@ -213,17 +218,6 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr)
 {
     asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
-// tile load into this CTA's shared memory whose completion is counted on an
-// mbarrier of the pair's leader CTA
-__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, uint32_t mbar_cluster, int x,
-                                                 int y)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
-        ::"r"(dst), "l"((uint64_t)map), "r"(mbar_cluster), "r"(x), "r"(y)
-        : "memory");
-}
-
 // shared-memory matrix descriptor (tcgen05): K-major, 128-byte swizzle,
 // 8-row core groups 1024 bytes apart
 __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr)
@@ -247,71 +241,57 @@ __device__ __forceinline__ uint64_t desc_sf(uint32_t saddr)
     return d;
 }
 
-// instruction descriptor: E2M1 x E2M1, fp32 accumulate, K-major A and B,
-// N = TBN, M = 128 (one CTA) or 256 (a CTA pair); scale format UE8M0 (MX) or
-// UE4M3 (NV)
-template <int FMT, int TBN, int CTAS = 1>
+// instruction descriptor: fp32 accumulate, K-major A and B, M = 128,
+// N = TBN.  FP4 formats (kind::mxf4 / mxf4nvf4): E2M1 x E2M1 (type code 1),
+// scale format UE8M0 (MX) or UE4M3 (NV).  FP8 activations (kind::mxf8f6f4):
+// A E4M3 (code 0) x B E2M1 (code 5) or, with FP8 weights, E4M3 (code 0);
+// UE8M0.
+template <int FMT, int TBN>
 __device__ __forceinline__ uint32_t idesc_base()
 {
-    return (1u << 7) | (1u << 10) | ((uint32_t)(TBN >> 3) << 17) | ((FMT == DS4G_MXFP4 ? 1u : 0u) << 23) |
-           ((uint32_t)((BM * CTAS) >> 4) << 24);
+    const uint32_t at = fp8_act(FMT) ? 0u : 1u;
+    const uint32_t bt = (FMT == DS4G_MXFP8) ? 5u : (FMT == kFmtFp8Fp8 ? 0u : 1u);
+    return (at << 7) | (bt << 10) | ((uint32_t)(TBN >> 3) << 17) | ((FMT == DS4G_NVFP4 ? 0u : 1u) << 23) |
+           ((uint32_t)(BM >> 4) << 24);
 }
 
-template <int FMT, int CTAS = 1>
+template <int FMT>
 __device__ __forceinline__ void mma(uint32_t d_tmem, uint64_t ad, uint64_t bd, uint32_t idesc, uint32_t acc,
                                     uint32_t sfa, uint32_t sfb)
 {
-    if (FMT == DS4G_MXFP4 && CTAS == 1) {
+    if (fp8_act(FMT)) {
         asm volatile(
             "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-            "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+            "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
             ::"r"(d_tmem), "l"(ad), "l"(bd), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb)
             : "memory");
     } else if (FMT == DS4G_MXFP4) {
         asm volatile(
             "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-            "tcgen05.mma.cta_group::2.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
-            ::"r"(d_tmem), "l"(ad), "l"(bd), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb)
-            : "memory");
-    } else if (CTAS == 1) {
-        asm volatile(
-            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-            "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+            "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
             ::"r"(d_tmem), "l"(ad), "l"(bd), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb)
             : "memory");
     } else {
         asm volatile(
             "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-            "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+            "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
             ::"r"(d_tmem), "l"(ad), "l"(bd), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb)
             : "memory");
     }
 }
 
 // shared -> tensor memory copy of one 32 x 16-byte scale chunk into all four
-// lane quarters; with a CTA pair each CTA copies its own chunk into its own
-// tensor memory
-template <int CTAS = 1>
+// lane quarters
 __device__ __forceinline__ void utccp(uint32_t taddr, uint64_t sdesc)
 {
-    if (CTAS == 1)
-        asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
-    else
-        asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
-// arrive on `mbar` once the thread's earlier tensor-core operations are done;
-// with a CTA pair on the mbarrier at the same offset in both CTAs
-template <int CTAS = 1>
+// arrive on `mbar` once the thread's earlier tensor-core operations are done
 __device__ __forceinline__ void tc_commit(uint32_t mbar)
 {
-    if (CTAS == 1)
-        asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(mbar)
-                     : "memory");
-    else
-        asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
-                     ::"r"(mbar), "h"((uint16_t)3)
-                     : "memory");
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(mbar)
+                 : "memory");
 }
 
 // 16 TMEM lanes x 16 columns: thread t gets lanes t/4 and t/4 + 8, columns
@@ -416,23 +396,35 @@ struct Tile {
     int64_t end;  // end of the expert's segment
 };
 
-template <int BMT = BM>
+// Tiles are numbered band by band: a band is nb consecutive column tiles
+// (the last band may be narrower), and within a band expert by expert, then
+// column tile, then row tile.  prefix[e] counts the row tiles of the experts
+// before e (prefix[E] of all of them).  With one band (nb = n_tiles) this is
+// expert-major order.  The combine epilogue uses several bands when the
+// output is larger than L2: the reductions of all experts into one band's
+// columns of the output then happen while those columns are in L2.
 __device__ __forceinline__ Tile tile_of(int64_t t, const int32_t* prefix, const int32_t* offsets, int E,
-                                        int n_tiles)
+                                        int n_tiles, int nb)
 {
-    int lo = 0, hi = E - 1;   // largest e with prefix[e] <= t (prefix non-decreasing)
+    const int64_t U = prefix[E];
+    const int nbands = (n_tiles + nb - 1) / nb;
+    int64_t band = t / (U * nb);
+    if (band > nbands - 1) band = nbands - 1;
+    const int nbb = min(nb, n_tiles - (int)band * nb);          // column tiles of this band
+    const int64_t local = t - band * U * nb;
+    int lo = 0, hi = E - 1;   // largest e with prefix[e] * nbb <= local (prefix non-decreasing)
     while (lo < hi) {
         int mid = (lo + hi + 1) >> 1;
-        if (prefix[mid] <= t) lo = mid; else hi = mid - 1;
+        if ((int64_t)prefix[mid] * nbb <= local) lo = mid; else hi = mid - 1;
     }
     Tile r;
     r.e = lo;
     const int64_t beg = offsets[lo];
     r.end = offsets[lo + 1];
-    const int64_t mt_cnt = ceil_div(r.end - beg, BMT);
-    const int64_t local = t - prefix[lo];
-    r.nt = (int)(local / mt_cnt);
-    r.m0 = beg + (local % mt_cnt) * BMT;
+    const int64_t mt_cnt = ceil_div(r.end - beg, BM);
+    const int64_t le = local - (int64_t)prefix[lo] * nbb;
+    r.nt = (int)(band * nb + le / mt_cnt);
+    r.m0 = beg + (le % mt_cnt) * BM;
     return r;
 }
 
@@ -450,13 +442,12 @@ __device__ __forceinline__ void w_rows(const Tile& tl, int N, int I, int64_t& y0
     }
 }
 
-template <int FMT, int EPI, int TBN, int NISS, int CTAS>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int FMT, int EPI, int TBN, int NISS>
+__global__ void __launch_bounds__(Cfg<FMT, TBN, NISS>::THREADS, 1)
 k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
           const __grid_constant__ CUtensorMap map_sfa, const __grid_constant__ CUtensorMap map_sfb, const GemmArgs p)
 {
-    using C = Cfg<FMT, TBN, NISS, CTAS>;
-    constexpr bool PAIR = (CTAS == 2);
+    using C = Cfg<FMT, TBN, NISS>;
     constexpr int STAGES = C::NST;
     constexpr int SF_STAGES = C::SF_STAGES;
     static_assert(EPI != DS4G_EPI_SWIGLU_REQUANT || TBN == 256 || TBN == 192,
@@ -486,17 +477,17 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int E = p.E;
     const int64_t K = p.K;
-    const int nks = (int)ceil_div(K, BK);
-    const int npairs = (nks + 1) / 2;
+    constexpr int KPS = C::KPS;
+    const int nks = (int)ceil_div(K, C::KE);
+    const int nsfs = (nks + KPS - 1) / KPS;      // scale stages per tile
     const int I = p.N / 2;
     // SwiGLU: the last tile may be ragged (I % (TBN/2) != 0); its columns past
     // I are computed from other rows and never stored
     const int n_tiles = (EPI == DS4G_EPI_SWIGLU_REQUANT) ? (int)ceil_div(I, TBN / 2) : (int)ceil_div(p.N, TBN);
-    // A CTA pair walks the tiles of its cluster; rank 0 (the leader) issues
-    // the pair's MMAs, rank 1 only loads its halves and drains its rows.
-    const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
-    const int64_t tile0 = PAIR ? (int64_t)cluster_id_x() : (int64_t)blockIdx.x;
-    const int64_t tstride = PAIR ? (int64_t)nclusters_x() : (int64_t)gridDim.x;
+    // column tiles per band of the tile order (see tile_of)
+    const int nb = (EPI == kEpiCombine && p.band_tiles > 0 && p.band_tiles < n_tiles) ? p.band_tiles : n_tiles;
+    const int64_t tile0 = blockIdx.x;
+    const int64_t tstride = gridDim.x;
 
     // ---- prologue
     if (threadIdx.x == 0) {
@@ -506,20 +497,19 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
         }
         for (int r = 0; r < SF_STAGES; ++r) {
             mbar_init(smem_u32(&sf_full[r]), 1);
-            mbar_init(smem_u32(&sf_ready[r]), PAIR ? 2 : 1);     // pair: both CTAs' transposers
+            mbar_init(smem_u32(&sf_ready[r]), 1);
             mbar_init(smem_u32(&sf_empty[r]), 1);
         }
         for (int b2 = 0; b2 < NACC; ++b2) {
             mbar_init(smem_u32(&tmem_full[b2]), 1);
-            // pair: one arrival per epilogue warp of either CTA
-            mbar_init(smem_u32(&tmem_empty[b2]), PAIR ? 2 * kEpiWarps : 32 * kEpiWarps);
+            mbar_init(smem_u32(&tmem_empty[b2]), 32 * kEpiWarps);
         }
         *abort_flag = 0;
         fence_barrier_init();
     }
     // the expert offsets -> shared memory in one parallel pass (a loop of
     // dependent global loads here cost about 2 us per launch)
-    for (int e = threadIdx.x; e <= E; e += kThreads) soff[e] = p.offsets[e];
+    for (int e = threadIdx.x; e <= E; e += C::THREADS) soff[e] = p.offsets[e];
     if (warp == 0 && lane == 0) {
         asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&map_a) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&map_b) : "memory");
@@ -527,27 +517,19 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
         asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&map_sfb) : "memory");
     }
     if (warp == 3) {
-        if (PAIR) {
-            // both CTAs' warp 3 allocate together: the same columns in each
-            asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                         "r"(kTmemCols)
-                         : "memory");
-            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
-        } else {
-            asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                         "r"(kTmemCols)
-                         : "memory");
-            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-        }
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     __syncthreads();
     if (warp == 0) {
-        // tiles per expert, exclusive scan by one warp
+        // row tiles per expert, exclusive scan by one warp
         const int per = (E + 31) / 32;
         int32_t sum = 0;
         for (int i = 0; i < per; ++i) {
             const int e = lane * per + i;
-            if (e < E) sum += (int32_t)(ceil_div((int64_t)soff[e + 1] - soff[e], C::BMT) * n_tiles);
+            if (e < E) sum += (int32_t)ceil_div((int64_t)soff[e + 1] - soff[e], BM);
         }
         int32_t incl = sum;
 #pragma unroll
@@ -560,12 +542,12 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
             const int e = lane * per + i;
             if (e < E) {
                 prefix[e] = run;
-                run += (int32_t)(ceil_div((int64_t)soff[e + 1] - soff[e], C::BMT) * n_tiles);
+                run += (int32_t)ceil_div((int64_t)soff[e + 1] - soff[e], BM);
             }
         }
         if (lane == 31) {
             prefix[E] = incl;
-            int32_t tot = incl;
+            int32_t tot = incl * n_tiles;
             if ((int64_t)soff[E] > p.S) {   // inconsistent offsets: do nothing
                 raise_error(kErrBadOffsets);
                 tot = 0;
@@ -574,8 +556,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
         }
     }
     tc_fence_before();
-    // a pair: the peer's barriers must be initialised before anything arrives on them
-    if (PAIR) cluster_sync_all(); else __syncthreads();
+    __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const int64_t ntiles = *total_tiles;
@@ -585,10 +566,6 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
         // This CTA's tiles in groups of NISS consecutive ones; the stages of a
         // group are interleaved (K stage by K stage, member by member) so that
         // each MMA issuer finds its next stage while the other works.
-        // A pair: each CTA loads its own 128 activation rows and its half of
-        // the weight rows, counted on the leader's `full` barrier (the leader
-        // expects both CTAs' bytes); the scales of its own activation rows and
-        // of all TBN weight rows go to its own shared memory.
         if (lane == 0) {
             uint32_t it = 0, sit = 0;
             bool ok = true;
@@ -601,7 +578,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
 #pragma unroll
                 for (int u = 0; u < NISS; ++u) {
                     if (u < gsz) {
-                        tls[u] = tile_of<C::BMT>(t0 + u * tstride, prefix, soff, E, n_tiles);
+                        tls[u] = tile_of(t0 + u * tstride, prefix, soff, E, n_tiles, nb);
                         w_rows<EPI, TBN>(tls[u], p.N, I, y0s[u], y1s[u]);
                     }
                 }
@@ -610,79 +587,50 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
                     for (int u = 0; u < NISS; ++u) {
                         if (u >= gsz || !ok) continue;
                         const Tile& tl = tls[u];
-                        const int64_t arow = tl.m0 + (int64_t)BM * rank;   // this CTA's first activation row
-                        if ((ks & 1) == 0) {
+                        if ((ks % KPS) == 0) {
                             const int r = sit % SF_STAGES;
                             if (!mbar_wait(smem_u32(&sf_empty[r]), ((sit / SF_STAGES) & 1) ^ 1, abort_flag)) { ok = false; break; }
                             const uint32_t fb = smem_u32(&sf_full[r]);
                             mbar_arrive_tx(fb, C::SFA_BYTES + TBN * C::SF_ROW);
-                            const int x = (ks >> 1) * C::SF_ROW;
-                            tma_load_2d(smem_u32(sSFA + r * C::SFA_BYTES), &map_sfa, fb, x, (int)arow);
+                            const int x = (ks / KPS) * C::SF_ROW;
+                            tma_load_2d(smem_u32(sSFA + r * C::SFA_BYTES), &map_sfa, fb, x, (int)tl.m0);
                             tma_load_2d(smem_u32(sSFB + r * C::SFB_BYTES), &map_sfb, fb, x, (int)y0s[u]);
                             tma_load_2d(smem_u32(sSFB + r * C::SFB_BYTES + C::HALF * C::SF_ROW), &map_sfb, fb, x, (int)y1s[u]);
                             ++sit;
                         }
                         const int s = it % STAGES;
                         if (!mbar_wait(smem_u32(&empty[s]), ((it / STAGES) & 1) ^ 1, abort_flag)) { ok = false; break; }
-                        if (PAIR) {
-                            // the second CTA's activation rows may lie wholly
-                            // past the expert's segment: then they are not
-                            // loaded (the MMA computes rows that are never stored)
-                            const bool peer_live = tl.m0 + BM < tl.end;
-                            const uint32_t fb = mapa_shared(smem_u32(&full[s]), 0);
-                            if (rank == 0)
-                                mbar_arrive_tx(smem_u32(&full[s]), (peer_live ? 2 * A_BYTES : A_BYTES) + 2 * B_BYTES);
-                            if (rank == 0 || peer_live)
-                                tma_load_2d_pair(smem_u32(sA + s * A_BYTES), &map_a, fb, ks * BKB, (int)arow);
-                            tma_load_2d_pair(smem_u32(sB + s * B_BYTES), &map_b, fb, ks * BKB,
-                                             (int)(rank == 0 ? y0s[u] : y1s[u]));
-                        } else {
-                            const uint32_t fb = smem_u32(&full[s]);
-                            mbar_arrive_tx(fb, A_BYTES + B_BYTES);
-                            tma_load_2d(smem_u32(sA + s * A_BYTES), &map_a, fb, ks * BKB, (int)tl.m0);
-                            tma_load_2d(smem_u32(sB + s * B_BYTES), &map_b, fb, ks * BKB, (int)y0s[u]);
-                            tma_load_2d(smem_u32(sB + s * B_BYTES + B_BYTES / 2), &map_b, fb, ks * BKB, (int)y1s[u]);
-                        }
+                        const uint32_t fb = smem_u32(&full[s]);
+                        mbar_arrive_tx(fb, A_BYTES + C::B_TX);
+                        tma_load_2d(smem_u32(sA + s * A_BYTES), &map_a, fb, ks * BKB, (int)tl.m0);
+                        tma_load_2d(smem_u32(sB + s * B_BYTES), &map_b, fb, ks * BKB, (int)y0s[u]);
+                        tma_load_2d(smem_u32(sB + s * B_BYTES + B_BYTES / 2), &map_b, fb, ks * BKB, (int)y1s[u]);
                         ++it;
                     }
                 }
             }
             if (!ok) {
                 // let the copies already issued land before the CTA goes away
-                // (a pair's data copies count on the leader's barriers, which
-                // only the leader can wait on)
                 volatile int never = 0;
-                if (!PAIR || rank == 0)
-                    for (uint32_t j = (it > STAGES ? it - STAGES : 0); j < it; ++j)
-                        mbar_wait(smem_u32(&full[j % STAGES]), (j / STAGES) & 1, &never);
+                for (uint32_t j = (it > STAGES ? it - STAGES : 0); j < it; ++j)
+                    mbar_wait(smem_u32(&full[j % STAGES]), (j / STAGES) & 1, &never);
                 for (uint32_t j = (sit > SF_STAGES ? sit - SF_STAGES : 0); j < sit; ++j)
                     mbar_wait(smem_u32(&sf_full[j % SF_STAGES]), (j / SF_STAGES) & 1, &never);
-            } else if (PAIR) {
-                // the leader's last commits arrive on this CTA's barriers:
-                // wait for them so that none lands after the CTA has exited
-                for (uint32_t j = (it > STAGES ? it - STAGES : 0); j < it; ++j)
-                    if (!mbar_wait(smem_u32(&empty[j % STAGES]), (j / STAGES) & 1, abort_flag)) break;
-                for (uint32_t j = (sit > SF_STAGES ? sit - SF_STAGES : 0); j < sit; ++j)
-                    if (!mbar_wait(smem_u32(&sf_empty[j % SF_STAGES]), (j / SF_STAGES) & 1, abort_flag)) break;
             }
         }
         __syncwarp();
-    } else if ((warp == 1 || (NISS == 2 && warp == 3)) && rank == 0) {
+    } else if (warp == 1 || (NISS == 2 && warp == 3)) {
         // ================= MMA issuer(s) =================
         // Issuer pi takes member pi of each tile group, accumulating into
         // accumulator pi (two issuers) with its own scale columns.  An issuing
         // thread that waits on a barrier first drains its own tensor-core
         // work; with two issuers the other one's MMAs fill that gap.
-        // A pair: only the leader issues; its scale copies, MMAs and commits
-        // act on both CTAs (each CTA's own shared and tensor memory at the
-        // same addresses, the commits arrive on both CTAs' barriers).
         if (lane == 0) {
             const int pi = (warp == 1) ? 0 : 1;
-            const uint32_t ibase = idesc_base<FMT, TBN, CTAS>();
+            const uint32_t ibase = idesc_base<FMT, TBN>();
             const uint32_t col_sfa = tmem + C::COL_SFA + pi * C::SF_COLS;
             const uint32_t col_sfb = col_sfa + 4 * C::WPS;
             uint32_t it_base = 0, sit_base = 0;
-            uint32_t uses[2] = {0, 0};
             bool ok = true;
             for (int64_t j0 = 0; ok; j0 += NISS) {
                 const int64_t t0 = tile0 + j0 * tstride;
@@ -693,80 +641,73 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
                     const int buf = (NISS == 2) ? pi : (int)(jt % NACC);
                     const uint32_t use = (NISS == 2) ? (uint32_t)(j0 / 2) : (uint32_t)(jt / NACC);
                     if (!mbar_wait(smem_u32(&tmem_empty[buf]), (use & 1) ^ 1, abort_flag)) { ok = false; break; }
-                    uses[buf] = use + 1;
                     const uint32_t acc = tmem + kColAcc + buf * TBN;
                     tc_fence_after();
                     for (int ks = 0; ks < nks; ++ks) {
                         const uint32_t it = it_base + (uint32_t)(ks * gsz + pi);
-                        const uint32_t sit = sit_base + (uint32_t)((ks >> 1) * gsz + pi);
+                        const uint32_t sit = sit_base + (uint32_t)((ks / KPS) * gsz + pi);
                         const int r = sit % SF_STAGES;
-                        if ((ks & 1) == 0) {
+                        if ((ks % KPS) == 0) {
                             if (!mbar_wait(smem_u32(&sf_ready[r]), (sit / SF_STAGES) & 1, abort_flag)) { ok = false; break; }
                         }
                         const int s = it % STAGES;
                         if (!mbar_wait(smem_u32(&full[s]), (it / STAGES) & 1, abort_flag)) { ok = false; break; }
                         tc_fence_after();
                         // this K stage's scale words -> TMEM
-                        const int w0 = (ks & 1) * C::WPS;
+                        const int w0 = (ks % KPS) * C::WPS;
                         const uint32_t sfa_s = smem_u32(sSFA + r * C::SFA_BYTES);
                         const uint32_t sfb_s = smem_u32(sSFB + r * C::SFB_BYTES);
 #pragma unroll
                         for (int c = 0; c < C::WPS; ++c) {
-                            utccp<CTAS>(col_sfa + 4 * c, desc_sf(sfa_s + (w0 + c) * 512));
-                            utccp<CTAS>(col_sfb + 8 * c, desc_sf(sfb_s + ((w0 + c) * 2 + 0) * 512));
-                            utccp<CTAS>(col_sfb + 8 * c + 4, desc_sf(sfb_s + ((w0 + c) * 2 + 1) * 512));
+                            utccp(col_sfa + 4 * c, desc_sf(sfa_s + (w0 + c) * 512));
+                            utccp(col_sfb + 8 * c, desc_sf(sfb_s + ((w0 + c) * 2 + 0) * 512));
+                            utccp(col_sfb + 8 * c + 4, desc_sf(sfb_s + ((w0 + c) * 2 + 1) * 512));
                         }
-                        const int64_t krem = K - (int64_t)ks * BK;
-                        const int nmma = krem >= BK ? 4 : (int)(krem / 64);
+                        const int64_t krem = K - (int64_t)ks * C::KE;
+                        const int nmma = krem >= C::KE ? 4 : (int)(krem / (C::KE / 4));
                         const uint32_t a_s = smem_u32(sA + s * A_BYTES);
                         const uint32_t b_s = smem_u32(sB + s * B_BYTES);
 #pragma unroll
                         for (int j = 0; j < 4; ++j) {
                             if (j < nmma) {
-                                const int c = (FMT == DS4G_MXFP4) ? (j >> 1) : j;
-                                const uint32_t sfid = (FMT == DS4G_MXFP4) ? (uint32_t)((j & 1) * 2) : 0u;
+                                // scale word (4 TMEM columns) and byte of MMA j:
+                                // MX K = 64 takes 2 scales (bytes 0-1 / 2-3 of
+                                // word j / 2), NV K = 64 all 4 of word j, MXFP8
+                                // K = 32 byte j of the stage's one word
+                                const int c = (FMT == DS4G_MXFP4) ? (j >> 1) : (FMT == DS4G_NVFP4 ? j : 0);
+                                const uint32_t sfid = (FMT == DS4G_MXFP4) ? (uint32_t)((j & 1) * 2)
+                                                                         : (FMT == DS4G_NVFP4 ? 0u : (uint32_t)j);
                                 const uint32_t idesc = ibase | (sfid << 4) | (sfid << 29);
-                                mma<FMT, CTAS>(acc, desc_sw128(a_s + 32 * j), desc_sw128(b_s + 32 * j), idesc,
-                                               (ks > 0 || j > 0) ? 1u : 0u, col_sfa + 4 * c, col_sfb + 8 * c);
+                                mma<FMT>(acc, desc_sw128(a_s + 32 * j), desc_sw128(b_s + 32 * j), idesc,
+                                         (ks > 0 || j > 0) ? 1u : 0u, col_sfa + 4 * c, col_sfb + 8 * c);
                             }
                         }
-                        tc_commit<CTAS>(smem_u32(&empty[s]));
-                        if ((ks & 1) == 1 || ks == nks - 1) tc_commit<CTAS>(smem_u32(&sf_empty[r]));
+                        tc_commit(smem_u32(&empty[s]));
+                        if ((ks % KPS) == KPS - 1 || ks == nks - 1) tc_commit(smem_u32(&sf_empty[r]));
                     }
                     if (!ok) break;
-                    tc_commit<CTAS>(smem_u32(&tmem_full[buf]));
+                    tc_commit(smem_u32(&tmem_full[buf]));
                 }
                 it_base += (uint32_t)(nks * gsz);
-                sit_base += (uint32_t)(npairs * gsz);
-            }
-            if (PAIR && ok) {
-                // both CTAs' epilogues have released the last accumulators
-                // (their arrivals on this CTA's barriers have landed)
-                for (int b2 = 0; b2 < NACC; ++b2)
-                    if ((NISS == 1 || b2 == pi) && uses[b2] > 0)
-                        if (!mbar_wait(smem_u32(&tmem_empty[b2]), (uses[b2] & 1) ^ 1, abort_flag)) break;
+                sit_base += (uint32_t)(nsfs * gsz);
             }
         }
         __syncwarp();
     } else if (warp == 2) {
         // ================= scale transposer =================
-        // (a pair: each CTA transposes its own scales and tells the leader)
         uint32_t sit = 0;
         for (int64_t t = tile0; t < ntiles; t += tstride) {
             bool ok = true;
-            for (int pr = 0; pr < npairs; ++pr, ++sit) {
+            for (int pr = 0; pr < nsfs; ++pr, ++sit) {
                 const int r = sit % SF_STAGES;
                 bool w_ok = true;
                 if (lane == 0) w_ok = mbar_wait(smem_u32(&sf_full[r]), (sit / SF_STAGES) & 1, abort_flag);
                 if (!__shfl_sync(0xffffffffu, w_ok ? 1 : 0, 0)) { ok = false; break; }
-                sf_transpose<2 * C::WPS, 1>(sSFA + r * C::SFA_BYTES, lane);
-                sf_transpose<2 * C::WPS, 2>(sSFB + r * C::SFB_BYTES, lane);
+                sf_transpose<KPS * C::WPS, 1>(sSFA + r * C::SFA_BYTES, lane);
+                sf_transpose<KPS * C::WPS, 2>(sSFB + r * C::SFB_BYTES, lane);
                 fence_proxy_async();
                 __syncwarp();
-                if (lane == 0) {
-                    if (PAIR) mbar_arrive_cluster(mapa_shared(smem_u32(&sf_ready[r]), 0));
-                    else mbar_arrive(smem_u32(&sf_ready[r]));
-                }
+                if (lane == 0) mbar_arrive(smem_u32(&sf_ready[r]));
             }
             if (!ok) break;
         }
@@ -782,8 +723,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
             // epilogue) the output rows of this thread's four tile rows are
             // looked up before waiting for the accumulator, so that their
             // global loads overlap the tile's mainloop
-            Tile tl = tile_of<C::BMT>(t, prefix, soff, E, n_tiles);
-            tl.m0 += (int64_t)BM * rank;           // a pair: this CTA's 128 rows of the tile
+            const Tile tl = tile_of(t, prefix, soff, E, n_tiles, nb);
             const float gscale = (FMT == DS4G_NVFP4) ? __fmul_rn(p.a_g[0], p.w_g[tl.e]) : 1.0f;
             constexpr bool kDirect = (EPI != DS4G_EPI_SWIGLU_REQUANT) && !C::STAGED;
             float* dk[2][2];
@@ -810,10 +750,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
                         }
                     }
             }
-            const bool got = mbar_wait(smem_u32(&tmem_full[buf]), (tcount / NACC) & 1, abort_flag);
-            // a pair's teardown is a warp-aligned cluster barrier: the whole
-            // warp leaves the loop together
-            if (PAIR ? !__all_sync(0xffffffffu, got) : !got) break;
+            if (!mbar_wait(smem_u32(&tmem_full[buf]), (tcount / NACC) & 1, abort_flag)) break;
             tc_fence_after();
             const int64_t row = tl.m0 + 32 * q + lane;
             const bool valid = row < tl.end;
@@ -924,7 +861,24 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
                             for (int i = 0; i < 8; ++i) hd[i] = make_float4(h[4 * i], h[4 * i + 1], h[4 * i + 2], h[4 * i + 3]);
                         }
                         uint32_t wq[4] = {0, 0, 0, 0};
-                        if (FMT == DS4G_MXFP4) {
+                        if (fp8_act(FMT)) {
+                            // "SwiGLU + FP8 quant": h -> E4M3 with a UE8M0
+                            // scale per 32 (OCP MX rule, largest exponent 8)
+                            float m = 0.f;
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) m = fmaxf(m, fabsf(h[i]));
+                            const int X = mx_shared_exp<8>(m);
+                            const float inv = exp2i(-X);
+                            uint32_t w8[8];
+#pragma unroll
+                            for (int i = 0; i < 8; ++i)
+                                w8[i] = e4m3x2(__fmul_rn(h[4 * i], inv), __fmul_rn(h[4 * i + 1], inv)) |
+                                        (e4m3x2(__fmul_rn(h[4 * i + 2], inv), __fmul_rn(h[4 * i + 3], inv)) << 16);
+                            p.oq_scales[row * (I / 32) + col0 / 32] = (uint8_t)(X + 127);
+                            uint4* dq = reinterpret_cast<uint4*>(p.oq_data + row * I + col0);
+                            dq[0] = make_uint4(w8[0], w8[1], w8[2], w8[3]);
+                            dq[1] = make_uint4(w8[4], w8[5], w8[6], w8[7]);
+                        } else if (FMT == DS4G_MXFP4) {
                             float m = 0.f;
 #pragma unroll
                             for (int i = 0; i < 32; ++i) m = fmaxf(m, fabsf(h[i]));
@@ -948,11 +902,16 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
                                     for (int i = 0; i < 16; ++i)
                                         wq[2 * hb + (i >> 3)] |= ((__float_as_uint(h[16 * hb + i]) >> 28) & 8u) << (4 * (i & 7));
                                 } else {
-                                    const float den = __fmul_rn(ds, gh);
+                                    // h / (dec(s) g_h) as h times the correctly
+                                    // rounded reciprocal (within 1.5 ulp of the
+                                    // quotient; a code can then differ from the
+                                    // divided one only for a quotient that close
+                                    // to a rounding boundary of the E2M1 grid)
+                                    const float rcp = __frcp_rn(__fmul_rn(ds, gh));
 #pragma unroll
                                     for (int i = 0; i < 16; i += 2)
-                                        wq[2 * hb + (i >> 3)] |= e2m1x2(__fdiv_rn(h[16 * hb + i], den),
-                                                                        __fdiv_rn(h[16 * hb + i + 1], den))
+                                        wq[2 * hb + (i >> 3)] |= e2m1x2(__fmul_rn(h[16 * hb + i], rcp),
+                                                                        __fmul_rn(h[16 * hb + i + 1], rcp))
                                                                  << (4 * (i & 7));
                                 }
                                 sb[hb] = s;
@@ -960,32 +919,23 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
                             *reinterpret_cast<uint16_t*>(p.oq_scales + row * (I / 16) + col0 / 16) =
                                 (uint16_t)(sb[0] | (sb[1] << 8));
                         }
-                        *reinterpret_cast<uint4*>(p.oq_data + row * (I / 2) + col0 / 2) =
-                            make_uint4(wq[0], wq[1], wq[2], wq[3]);
+                        if (!fp8_act(FMT))
+                            *reinterpret_cast<uint4*>(p.oq_data + row * (I / 2) + col0 / 2) =
+                                make_uint4(wq[0], wq[1], wq[2], wq[3]);
                     }
                 }
             }
             tc_fence_before();
-            if (PAIR) {
-                __syncwarp();
-                if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tmem_empty[buf]), 0));
-            } else {
-                mbar_arrive(smem_u32(&tmem_empty[buf]));
-            }
+            mbar_arrive(smem_u32(&tmem_empty[buf]));
         }
     }
 
-    // ---- teardown (a pair: neither CTA leaves while the other may still
-    // touch its shared or tensor memory)
+    // ---- teardown
     tc_fence_before();
-    if (PAIR) cluster_sync_all(); else __syncthreads();
+    __syncthreads();
     tc_fence_after();
-    if (warp == 3) {
-        if (PAIR)
-            asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
-        else
-            asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
-    }
+    if (warp == 3)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
 }
 
 }  // namespace tc
@@ -1008,6 +958,27 @@ static PFN_encodeTiled get_encode()
     return fn;
 }
 
+// 2-D map over [rows][K] packed E2M1 codes (K / 2 bytes per row) that lands
+// each 128-element box row in shared memory as the 8-bit-per-element layout
+// kind::mxf8f6f4 reads for FP4 operands: every 16 codes (8 bytes) followed by
+// an 8-byte gap, so 128 elements fill a 128-byte row (CUDA's
+// CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B; needs K % 128 == 0, a 32-byte
+// aligned base and a row pitch that is a multiple of 32 bytes), 128-byte
+// swizzle, box 128 elements x box_h rows
+static bool make_map_fp4_unpacked(CUtensorMap* m, const uint8_t* base, int64_t rows, int64_t K, uint32_t box_h)
+{
+    PFN_encodeTiled enc = get_encode();
+    if (!enc || (reinterpret_cast<uintptr_t>(base) & 31) != 0 || K % 128 != 0 || (K / 2) % 32 != 0) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
+    cuuint32_t box[2] = {128, box_h};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, const_cast<uint8_t*>(base), dims, strides, box,
+                     estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 // 2-D byte map over [rows][width] bytes with a box of box_w bytes x box_h rows
 static bool make_map(CUtensorMap* m, const uint8_t* base, int64_t rows, int64_t width, uint32_t box_w,
                      uint32_t box_h, bool swizzle)
@@ -1024,113 +995,94 @@ static bool make_map(CUtensorMap* m, const uint8_t* base, int64_t rows, int64_t 
     return r == CUDA_SUCCESS;
 }
 
-template <int FMT, int EPI, int TBN, int NISS, int CTAS = 1>
+template <int FMT, int EPI, int TBN, int NISS>
 static cudaError_t run_tc(const GemmArgs& a, cudaStream_t st)
 {
-    using C = tc::Cfg<FMT, TBN, NISS, CTAS>;
-    const int blk = (FMT == DS4G_MXFP4) ? 32 : 16;
+    using C = tc::Cfg<FMT, TBN, NISS>;
+    const int blk = (FMT == DS4G_NVFP4) ? 16 : 32;
+    const bool fp8 = fp8_act(FMT);
     CUtensorMap ma, mb, msa, msb;
-    if (!make_map(&ma, a.a_data, a.S, a.K / 2, 128, 128, true) ||
-        !make_map(&mb, a.w_data, (int64_t)a.E * a.N, a.K / 2, 128, C::HALF, true) ||
+    // activations: 128 bytes of K per box row (256 FP4 or 128 FP8 elements);
+    // weights: 256 packed FP4 elements, 128 unpacked FP4 elements next to FP8
+    // activations, or 128 FP8 elements
+    if (!make_map(&ma, a.a_data, a.S, fp8 ? a.K : a.K / 2, 128, 128, true) ||
+        !(FMT == DS4G_MXFP8 ? make_map_fp4_unpacked(&mb, a.w_data, (int64_t)a.E * a.N, a.K, C::HALF)
+                            : make_map(&mb, a.w_data, (int64_t)a.E * a.N, FMT == kFmtFp8Fp8 ? a.K : a.K / 2, 128,
+                                       C::HALF, true)) ||
         !make_map(&msa, a.a_scales, a.S, a.K / blk, C::SF_ROW, 128, false) ||
         !make_map(&msb, a.w_scales, (int64_t)a.E * a.N, a.K / blk, C::SF_ROW, C::HALF, false))
         return cudaErrorInvalidValue;
-    auto kern = tc::k_gemm_tc<FMT, EPI, TBN, NISS, CTAS>;
+    auto kern = tc::k_gemm_tc<FMT, EPI, TBN, NISS>;
     const size_t shm = C::SMEM;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)shm);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = kNumSMs;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (CTAS == 1) {
-        kern<<<sms, tc::kThreads, shm, st>>>(ma, mb, msa, msb, a);
-        return cudaGetLastError();
-    }
-    // CTA pairs: clusters of two, as many as can be resident at once (the
-    // grid is persistent, so a cluster that had to wait for another to finish
-    // would double the time)
-    cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.gridDim = dim3((unsigned)(sms & ~1));
-    cfg.blockDim = dim3(tc::kThreads);
-    cfg.dynamicSmemBytes = shm;
-    cfg.stream = st;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    int nclusters = 0;
-    e = cudaOccupancyMaxActiveClusters(&nclusters, kern, &cfg);
-    if (e != cudaSuccess) return e;
-    if (nclusters < 1) return cudaErrorInvalidConfiguration;
-    cfg.gridDim = dim3((unsigned)(2 * (nclusters < sms / 2 ? nclusters : sms / 2)));
-    e = cudaLaunchKernelEx(&cfg, kern, ma, mb, msa, msb, a);
-    if (e != cudaSuccess) return e;
+    kern<<<sms, C::THREADS, shm, st>>>(ma, mb, msa, msb, a);
     return cudaGetLastError();
 }
 
 // plain and combine epilogues, N % 224 == 0 (FC2, N = 7168): 224-column
-// tiles with two accumulators; MXFP4 with two MMA issuers, NVFP4 (whose scale
-// columns do not fit beside them twice) with one issuer and the staged
-// epilogue.  (NVFP4 192-column tiles with two issuers measured slower: FC2
-// at T = 16384 2.18 ms against 1.97 ms, with the current epilogues on one
-// box.  A variant that copied one scale
-// word at a time, so that two NVFP4 issuers fit in tensor memory, left
-// shared memory for only three data stages and faulted on the T = 16384
-// layer, cause not found; it is not used.)
-// Other N: 256-column tiles, one accumulator.
+// tiles with two accumulators; MXFP4 and FP8 activations with two MMA
+// issuers, NVFP4 (whose scale columns do not fit beside them twice) with one
+// issuer and the staged epilogue.  Other N: 256-column tiles, one accumulator.
 template <int FMT, int EPI>
-static cudaError_t run_tc_plain(const GemmArgs& a, cudaStream_t st, bool pair)
+static cudaError_t run_tc_plain(const GemmArgs& a, cudaStream_t st)
 {
-    if (a.N % 224 != 0) return pair ? run_tc<FMT, EPI, 256, 1, 2>(a, st) : run_tc<FMT, EPI, 256, 1>(a, st);
-    if constexpr (FMT == DS4G_MXFP4)
-        return pair ? run_tc<FMT, EPI, 224, 2, 2>(a, st) : run_tc<FMT, EPI, 224, 2>(a, st);
-    else
-        return pair ? run_tc<FMT, EPI, 224, 1, 2>(a, st) : run_tc<FMT, EPI, 224, 1>(a, st);
+    if (a.N % 224 != 0) return run_tc<FMT, EPI, 256, 1>(a, st);
+    if constexpr (FMT != DS4G_NVFP4) return run_tc<FMT, EPI, 224, 2>(a, st);
+    else return run_tc<FMT, EPI, 224, 1>(a, st);
 }
 
+// FC1 + SwiGLU: 96 gate + 96 up columns per tile, two accumulators, two issuers
 template <int FMT>
-static cudaError_t run_tc_swiglu(const GemmArgs& a, cudaStream_t st, bool pair)
+static cudaError_t run_tc_swiglu(const GemmArgs& a, cudaStream_t st)
 {
-    return pair ? run_tc<FMT, DS4G_EPI_SWIGLU_REQUANT, 192, 2, 2>(a, st)
-                : run_tc<FMT, DS4G_EPI_SWIGLU_REQUANT, 192, 2>(a, st);
+    return run_tc<FMT, DS4G_EPI_SWIGLU_REQUANT, 192, 2>(a, st);
 }
 
 bool gemm_tc_supports(int fmt, int64_t K)
 {
-    // the scale rows are loaded by TMA in 16 (MX) / 32 (NV) byte boxes, whose
-    // row pitch K / block must be a multiple of 16 bytes
-    return fmt == DS4G_MXFP4 ? (K % 512 == 0) : (K % 256 == 0);
+    // the scale rows are loaded by TMA in 16 (MX, FP8) / 32 (NV) byte boxes,
+    // whose row pitch K / block must be a multiple of 16 bytes
+    return fmt == DS4G_NVFP4 ? (K % 256 == 0) : (K % 512 == 0);
 }
 
-// One CTA per 128-row tile (default), or CTA pairs per 256-row tile (tcgen05
-// cta_group::2) when DS4G_TC_PAIR=1 is set in the environment.  Pairs halve
-// the MMA instructions and the weight bytes per SM of a tile, but each SM
-// still runs all of its scale-factor copies, and the tensor pipe executes
-// copies and MMAs one after another (about 60 cycles per copy, N/2 per MMA):
-// per SM a K stage costs the same in both modes, and 256-row tiles waste
-// more rows on short expert segments.  Measured on the prefill layers, FC1
-// T = 2048 MXFP4 0.516 ms (one CTA) vs 0.698 ms (pairs), T = 16384 NVFP4
-// 2.44 vs 2.64 ms; FC2 + combine 0.377 vs 0.520 ms and 1.94 vs 2.14 ms.
-static bool use_pairs(const GemmArgs&)
+// Column tiles per band of the combine epilogue's tile order: as many as keep
+// one band's columns of the fp32 output (T rows) within about 60 MB, half of
+// L2, so that a token's k reductions into those columns find them in L2.
+// An output that fits in L2 (decode, T = 2048) is one band: expert-major order.
+static int combine_band_tiles(const GemmArgs& a, int tbn)
 {
-    const char* env = getenv("DS4G_TC_PAIR");
-    return env && env[0] == '1';
+    const int64_t T = a.topk > 0 ? a.S / a.topk : a.S;
+    const int64_t n_tiles = ceil_div(a.N, tbn);
+    const int64_t per_tile = T * tbn * 4;                 // output bytes of one column tile
+    int64_t nb = per_tile > 0 ? (int64_t)60000000 / per_tile : n_tiles;
+    if (nb < 1) nb = 1;
+    return (int)(nb < n_tiles ? nb : n_tiles);
 }
 
-cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st)
+cudaError_t launch_gemm_tc(const GemmArgs& a_in, cudaStream_t st)
 {
-    if (a.S == 0) return cudaSuccess;
-    if (a.E > tc::kMaxE || !gemm_tc_supports(a.fmt, a.K)) return cudaErrorInvalidValue;
-    const bool pair = use_pairs(a);
+    if (a_in.S == 0) return cudaSuccess;
+    if (a_in.E > tc::kMaxE || !gemm_tc_supports(a_in.fmt, a_in.K)) return cudaErrorInvalidValue;
+    GemmArgs a = a_in;
+    if (a.epilogue == kEpiCombine) a.band_tiles = combine_band_tiles(a, a.N % 224 == 0 ? 224 : 256);
+    if (a.fmt == DS4G_MXFP8)
+        return a.epilogue == DS4G_EPI_NONE ? run_tc_plain<DS4G_MXFP8, DS4G_EPI_NONE>(a, st)
+             : a.epilogue == kEpiCombine   ? run_tc_plain<DS4G_MXFP8, kEpiCombine>(a, st)
+                                           : run_tc_swiglu<DS4G_MXFP8>(a, st);
+    if (a.fmt == kFmtFp8Fp8)
+        return a.epilogue == DS4G_EPI_NONE ? run_tc_plain<kFmtFp8Fp8, DS4G_EPI_NONE>(a, st)
+             : a.epilogue == kEpiCombine   ? run_tc_plain<kFmtFp8Fp8, kEpiCombine>(a, st)
+                                           : run_tc_swiglu<kFmtFp8Fp8>(a, st);
     if (a.fmt == DS4G_MXFP4)
-        return a.epilogue == DS4G_EPI_NONE ? run_tc_plain<DS4G_MXFP4, DS4G_EPI_NONE>(a, st, pair)
-             : a.epilogue == kEpiCombine   ? run_tc_plain<DS4G_MXFP4, kEpiCombine>(a, st, pair)
-                                           : run_tc_swiglu<DS4G_MXFP4>(a, st, pair);
-    return a.epilogue == DS4G_EPI_NONE ? run_tc_plain<DS4G_NVFP4, DS4G_EPI_NONE>(a, st, pair)
-         : a.epilogue == kEpiCombine   ? run_tc_plain<DS4G_NVFP4, kEpiCombine>(a, st, pair)
-                                       : run_tc_swiglu<DS4G_NVFP4>(a, st, pair);
+        return a.epilogue == DS4G_EPI_NONE ? run_tc_plain<DS4G_MXFP4, DS4G_EPI_NONE>(a, st)
+             : a.epilogue == kEpiCombine   ? run_tc_plain<DS4G_MXFP4, kEpiCombine>(a, st)
+                                           : run_tc_swiglu<DS4G_MXFP4>(a, st);
+    return a.epilogue == DS4G_EPI_NONE ? run_tc_plain<DS4G_NVFP4, DS4G_EPI_NONE>(a, st)
+         : a.epilogue == kEpiCombine   ? run_tc_plain<DS4G_NVFP4, kEpiCombine>(a, st)
+                                       : run_tc_swiglu<DS4G_NVFP4>(a, st);
 }
 
 }  // namespace ds4g

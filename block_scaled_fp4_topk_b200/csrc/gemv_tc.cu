@@ -570,7 +570,7 @@ k_gemv_tc(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUt
                             const uint32_t s = ue4m3_encode(__fdiv_rn(m, __fmul_rn(6.0f, gh)));
                             const float ds = ue4m3_value(s);
                             code = (ds == 0.0f) ? ((__float_as_uint(h) >> 28) & 8u)
-                                                : e2m1_code(__fdiv_rn(h, __fmul_rn(ds, gh)));
+                                                : e2m1_code(__fmul_rn(h, __frcp_rn(__fmul_rn(ds, gh))));
                             if ((lane & 15) == 0) p.oq_scales[row * (I / 16) + col / 16] = (uint8_t)s;
                         }
                         const uint32_t hi_code = __shfl_down_sync(0xffffffffu, code, 1);

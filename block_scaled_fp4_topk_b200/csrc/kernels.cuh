@@ -48,6 +48,7 @@ struct GemmArgs {
     const float* route_w;
     int topk;
     int chained;             // decode kernel: launched to overlap the previous kernel on the stream
+    int band_tiles;          // prefill kernel, combine epilogue: column tiles per band of the tile order (0: all)
 };
 
 cudaError_t launch_gemv(const GemmArgs& a, cudaStream_t st);

@@ -119,9 +119,10 @@ __global__ void k_perm_rank(const int32_t* __restrict__ idx, int64_t S, int E, i
     }
 }
 
-// one warp per permuted row: copy data (K/2 bytes, 16-byte pieces) and scales
+// one warp per permuted row: copy data (rb bytes per row -- K/2 for FP4, K
+// for MXFP8 -- in 16-byte pieces) and the ns scale bytes (even)
 __global__ void k_perm_gather(const uint8_t* __restrict__ xd, const uint8_t* __restrict__ xs,
-                              const float* __restrict__ xg, int64_t S, int k, int64_t K, int blk,
+                              const float* __restrict__ xg, int64_t S, int k, int64_t rb, int64_t ns,
                               const int32_t* __restrict__ row_to_slot, uint8_t* __restrict__ ad,
                               uint8_t* __restrict__ as, float* __restrict__ ag)
 {
@@ -130,11 +131,10 @@ __global__ void k_perm_gather(const uint8_t* __restrict__ xd, const uint8_t* __r
     if (ag && r == 0 && lane == 0) *ag = *xg;
     if (r >= S) return;
     const int64_t t = row_to_slot[r] / k;
-    const int64_t nvec = K / 32;                         // 16-byte pieces of K/2 bytes
-    const uint4* src = reinterpret_cast<const uint4*>(xd + t * (K / 2));
-    uint4* dst = reinterpret_cast<uint4*>(ad + r * (K / 2));
+    const int64_t nvec = rb / 16;
+    const uint4* src = reinterpret_cast<const uint4*>(xd + t * rb);
+    uint4* dst = reinterpret_cast<uint4*>(ad + r * rb);
     for (int64_t i = lane; i < nvec; i += 32) dst[i] = src[i];
-    const int64_t ns = K / blk;                          // scale bytes per row (even)
     const uint16_t* ss = reinterpret_cast<const uint16_t*>(xs + t * ns);
     uint16_t* sd = reinterpret_cast<uint16_t*>(as + r * ns);
     for (int64_t i = lane; i < ns / 2; i += 32) sd[i] = ss[i];
@@ -145,7 +145,7 @@ __global__ void k_perm_gather(const uint8_t* __restrict__ xd, const uint8_t* __r
 constexpr int kSmallS = 512;
 
 __global__ void __launch_bounds__(512)
-k_perm_small(const int32_t* __restrict__ idx, int S, int E, int k, int64_t K, int blk,
+k_perm_small(const int32_t* __restrict__ idx, int S, int E, int k, int64_t rb, int64_t ns,
              const uint8_t* __restrict__ xd, const uint8_t* __restrict__ xs, const float* __restrict__ xg,
              int32_t* __restrict__ offsets, int32_t* __restrict__ row_to_slot, int32_t* __restrict__ slot_to_row,
              uint8_t* __restrict__ ad, uint8_t* __restrict__ as, float* __restrict__ ag)
@@ -207,12 +207,11 @@ k_perm_small(const int32_t* __restrict__ idx, int S, int E, int k, int64_t K, in
     }
     __syncthreads();
     // gather: one warp per permuted row
-    const int64_t nvec = K / 32;
-    const int64_t ns = K / blk;
+    const int64_t nvec = rb / 16;
     for (int r = warp; r < S; r += blockDim.x / 32) {
         const int64_t t = r2s[r] / k;
-        const uint4* src = reinterpret_cast<const uint4*>(xd + t * (K / 2));
-        uint4* dst = reinterpret_cast<uint4*>(ad + (int64_t)r * (K / 2));
+        const uint4* src = reinterpret_cast<const uint4*>(xd + t * rb);
+        uint4* dst = reinterpret_cast<uint4*>(ad + (int64_t)r * rb);
         for (int64_t i = lane; i < nvec; i += 32) dst[i] = src[i];
         const uint16_t* ss = reinterpret_cast<const uint16_t*>(xs + t * ns);
         uint16_t* sd = reinterpret_cast<uint16_t*>(as + (int64_t)r * ns);
@@ -235,18 +234,18 @@ cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, const uint8_
         if (fmt == DS4G_NVFP4 && ag) return cudaMemcpyAsync(ag, xg, sizeof(float), cudaMemcpyDeviceToDevice, st);
         return cudaSuccess;
     }
-    const int blk0 = (fmt == DS4G_MXFP4) ? 32 : 16;
+    const int64_t rb = (fmt == DS4G_MXFP8) ? K : K / 2;          // data bytes per row
+    const int64_t ns = K / (fmt == DS4G_NVFP4 ? 16 : 32);          // scale bytes per row
     if (S <= kSmallS) {
         const size_t shs = (size_t)(2 * E + 1 + S) * sizeof(int32_t);
-        k_perm_small<<<1, 512, shs, st>>>(idx, (int)S, E, k, K, blk0, xd, xs, xg, offsets, row_to_slot, slot_to_row,
+        k_perm_small<<<1, 512, shs, st>>>(idx, (int)S, E, k, rb, ns, xd, xs, xg, offsets, row_to_slot, slot_to_row,
                                           ad, as, fmt == DS4G_NVFP4 ? ag : nullptr);
         return cudaGetLastError();
     }
     k_perm_hist<<<B, 256, shm, st>>>(idx, S, E, B, ws);
     k_perm_scan<<<1, 1024, 0, st>>>(ws, E * B, E, B, S, offsets);
     k_perm_rank<<<B, 32, shm, st>>>(idx, S, E, B, ws, row_to_slot, slot_to_row);
-    const int blk = (fmt == DS4G_MXFP4) ? 32 : 16;
-    k_perm_gather<<<(unsigned)ceil_div(S, 8), 256, 0, st>>>(xd, xs, xg, S, k, K, blk, row_to_slot, ad, as,
+    k_perm_gather<<<(unsigned)ceil_div(S, 8), 256, 0, st>>>(xd, xs, xg, S, k, rb, ns, row_to_slot, ad, as,
                                                           fmt == DS4G_NVFP4 ? ag : nullptr);
     return cudaGetLastError();
 }

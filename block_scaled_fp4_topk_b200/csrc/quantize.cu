@@ -1,9 +1,11 @@
-// quantize.cu -- activations (bf16 / fp32) -> MXFP4 or NVFP4.
+// quantize.cu -- activations (bf16 / fp32) -> MXFP4, NVFP4 or MXFP8.
 //
 // MXFP4: "DGX Spark native FP4 matrix instructions ..." sec. 1 (E2M1 element
 // with a UE8M0 scale per 32) under the OCP MX shared-exponent rule.
 // NVFP4: same page, sec. 1 (kind::mxf4nvf4, UE4M3 scale per 16) with an fp32
-// tensor scale.  One thread quantises one block; its 32 (MX) or 16 (NV)
+// tensor scale.  MXFP8: the FP8 (E4M3) activations of the FP8 x FP4 GEMM
+// ("[DeepSeek V4] Triton FP4 optimisation in practice", "Step 0") with a
+// UE8M0 scale per 32 under the same OCP rule.  One thread quantises one block; its 32 (MX) or 16 (NV)
 // inputs are read with 16-byte loads, so a warp streams contiguous memory.
 #include "common.cuh"
 #include "kernels.cuh"
@@ -76,6 +78,39 @@ __device__ __forceinline__ void quant_nv_block(const float* v, float g, uint2& p
     packed = make_uint2(w[0], w[1]);
 }
 
+// one MXFP8 block of 32 values -> 32 E4M3 bytes + scale byte (OCP MX rule
+// with the E4M3 element, whose largest exponent is 8)
+__device__ __forceinline__ void quant_mx8_block(const float* v, uint4* codes, uint8_t& scale)
+{
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    const int X = mx_shared_exp<8>(amax);
+    scale = (uint8_t)(X + 127);
+    const float inv = exp2i(-X);
+    uint32_t w[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        w[i] = e4m3x2(__fmul_rn(v[4 * i], inv), __fmul_rn(v[4 * i + 1], inv)) |
+               (e4m3x2(__fmul_rn(v[4 * i + 2], inv), __fmul_rn(v[4 * i + 3], inv)) << 16);
+    codes[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    codes[1] = make_uint4(w[4], w[5], w[6], w[7]);
+}
+
+template <typename T>
+__global__ void k_quant_mx8(const T* __restrict__ x, int64_t nblocks, uint8_t* __restrict__ data,
+                            uint8_t* __restrict__ scales)
+{
+    for (int64_t b = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; b < nblocks;
+         b += (int64_t)gridDim.x * blockDim.x) {
+        float v[32];
+        load_block<T>(x + b * 32, v, 32);
+        uint8_t s;
+        quant_mx8_block(v, reinterpret_cast<uint4*>(data) + 2 * b, s);
+        scales[b] = s;
+    }
+}
+
 template <typename T>
 __global__ void k_quant_mx(const T* __restrict__ x, int64_t nblocks, int64_t K,
                            uint8_t* __restrict__ data, uint8_t* __restrict__ scales)
@@ -146,6 +181,14 @@ cudaError_t launch_quantize(const void* x, int dtype, int64_t rows, int64_t K, i
 {
     const int64_t n = rows * K;
     if (n == 0) return cudaSuccess;
+    if (fmt == DS4G_MXFP8) {
+        const int64_t nb = n / 32;
+        if (dtype == DS4G_BF16)
+            k_quant_mx8<uint16_t><<<grid_1d(nb, 256), 256, 0, st>>>((const uint16_t*)x, nb, data, scales);
+        else
+            k_quant_mx8<float><<<grid_1d(nb, 256), 256, 0, st>>>((const float*)x, nb, data, scales);
+        return cudaGetLastError();
+    }
     if (fmt == DS4G_MXFP4) {
         const int64_t nb = n / 32;
         if (dtype == DS4G_BF16)

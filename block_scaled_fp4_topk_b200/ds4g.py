@@ -13,11 +13,17 @@ from . import build as _build
 
 MXFP4 = 0
 NVFP4 = 1
+MXFP8 = 2
 BF16 = 0
 F32 = 1
 EPI_NONE = 0
 EPI_SWIGLU_REQUANT = 1
-BLOCK = {MXFP4: 32, NVFP4: 16}
+BLOCK = {MXFP4: 32, NVFP4: 16, MXFP8: 32}
+
+
+def row_bytes(fmt, K):
+    """bytes of one row of K elements: E4M3 (MXFP8) one per byte, E2M1 two"""
+    return K if fmt == MXFP8 else K // 2
 
 _STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "unsupported device", 4: "CUDA error",
            5: "device-side wait gave up", 6: "workspace missing or too small"}
@@ -86,8 +92,9 @@ def _check(name, st):
 
 
 class Fp4Tensor:
-    """Device FP4 tensor: data uint8 [rows][K/2], scales uint8 [rows][K/blk],
-    g float32 [1] (NVFP4 tensor scale) or None, fmt."""
+    """Device block-scaled tensor: data uint8 [rows][K/2] (FP4) or [rows][K]
+    (MXFP8), scales uint8 [rows][K/blk], g float32 [1] (NVFP4 tensor scale)
+    or None, fmt."""
 
     def __init__(self, data, scales, g, fmt):
         self.data, self.scales, self.g, self.fmt = data, scales, g, fmt
@@ -98,12 +105,12 @@ class Fp4Tensor:
 
     @property
     def K(self):
-        return self.data.shape[1] * 2
+        return self.data.shape[1] * (1 if self.fmt == MXFP8 else 2)
 
     @staticmethod
     def empty(rows, K, fmt, device="cuda"):
         g = torch.ones(1, dtype=torch.float32, device=device) if fmt == NVFP4 else None
-        return Fp4Tensor(torch.empty((rows, K // 2), dtype=torch.uint8, device=device),
+        return Fp4Tensor(torch.empty((rows, row_bytes(fmt, K)), dtype=torch.uint8, device=device),
                          torch.empty((rows, K // BLOCK[fmt]), dtype=torch.uint8, device=device), g, fmt)
 
     def c(self):

@@ -9,22 +9,36 @@ device buffers and issues the calls.
 import torch
 
 from . import ds4g
-from .ds4g import EPI_NONE, EPI_SWIGLU_REQUANT, NVFP4, Fp4Tensor
+from .ds4g import EPI_NONE, EPI_SWIGLU_REQUANT, MXFP4, MXFP8, NVFP4, Fp4Tensor
 
 
 class MoeLayer:
     def __init__(self, w1, w2, E, k, d, I, fmt, g_h=None, fused=True, fused_combine=True, fused_dispatch=True,
-                 chained=True):
+                 chained=True, act_fmt=None, shared=None):
         """w1: Fp4Tensor [E*2I][d] (gate rows then up rows per expert),
         w2: Fp4Tensor [E*d][I]; NVFP4 weights carry one tensor scale per
         expert (w.g has E floats); g_h: the static NVFP4 tensor scale of h.
         chained: the output is zeroed before the dispatch and FC2 + combine
-        is launched to overlap the end of FC1 (decode sizes)."""
+        is launched to overlap the end of FC1 (decode sizes).
+        act_fmt: the format of the activations and of h, fmt by default;
+        MXFP8 with MXFP4 weights is the FP8 x FP4 variant (its activations
+        take the separate routing / quantisation / permutation calls).
+        shared: (ws1 [2I_s][d], ws2 [d][I_s]) MXFP8 weights of a shared expert
+        that every token also goes through (FP8 activations only); its output
+        is added to the routed experts' sum with weight 1."""
         self.w1, self.w2 = w1, w2
         self.E, self.k, self.d, self.I, self.fmt = E, k, d, I, fmt
-        self.fused = fused
+        self.act_fmt = fmt if act_fmt is None else act_fmt
+        if self.act_fmt == MXFP8 and fmt != MXFP4:
+            raise ValueError("FP8 activations multiply MXFP4 weights")
+        self.fused = fused or self.act_fmt == MXFP8        # h is requantised in FC1's epilogue
         self.fused_combine = fused_combine
-        self.fused_dispatch = fused_dispatch
+        self.fused_dispatch = fused_dispatch and self.act_fmt != MXFP8
+        self.shared = shared
+        if shared is not None:
+            if self.act_fmt != MXFP8 or shared[0].fmt != MXFP8 or shared[1].fmt != MXFP8:
+                raise ValueError("the shared expert takes MXFP8 weights and FP8 activations")
+            self.I_s = shared[0].rows // 2
         self.chained = chained and fused_combine
         self.g_h = None
         if fmt == NVFP4:
@@ -40,12 +54,12 @@ class MoeLayer:
             b = dict(
                 idx=torch.empty((T, self.k), dtype=torch.int32, device=device),
                 w=torch.empty((T, self.k), dtype=torch.float32, device=device),
-                xq=Fp4Tensor.empty(T, self.d, self.fmt, device),
+                xq=Fp4Tensor.empty(T, self.d, self.act_fmt, device),
                 offsets=torch.empty(self.E + 1, dtype=torch.int32, device=device),
                 r2s=torch.empty(max(S, 1), dtype=torch.int32, device=device),
                 s2r=torch.empty(max(S, 1), dtype=torch.int32, device=device),
-                a=Fp4Tensor.empty(S, self.d, self.fmt, device),
-                hq=Fp4Tensor.empty(S, self.I, self.fmt, device),
+                a=Fp4Tensor.empty(S, self.d, self.act_fmt, device),
+                hq=Fp4Tensor.empty(S, self.I, self.act_fmt, device),
                 out=torch.empty((T, self.d), dtype=torch.float32, device=device),
                 pws=ds4g.permute_workspace(T, self.k, self.E, device),
                 dws=ds4g.dispatch_workspace(T, self.k, self.E, self.fmt, False, device),
@@ -53,6 +67,11 @@ class MoeLayer:
             )
             if self.fmt == NVFP4:
                 b["hq"].g = self.g_h
+            if self.shared is not None:
+                b["s_off"] = torch.tensor([0, T], dtype=torch.int32, device=device)
+                b["s_hq"] = Fp4Tensor.empty(T, self.I_s, MXFP8, device)
+                b["s_rows"] = torch.arange(max(T, 1), dtype=torch.int32, device=device)
+                b["s_w"] = torch.ones((T, 1), dtype=torch.float32, device=device)
             if not self.fused:
                 b["y1"] = torch.empty((S, 2 * self.I), dtype=torch.float32, device=device)
             if not self.fused_combine:
@@ -81,7 +100,7 @@ class MoeLayer:
                                    workspace=b["dws"])
             return
         ds4g.ds4g_route_topk(logits, self.k, idx=b["idx"], w=b["w"])
-        ds4g.ds4g_quantize_mx(x, self.fmt, out=b["xq"], workspace=b["qws"])
+        ds4g.ds4g_quantize_mx(x, self.act_fmt, out=b["xq"], workspace=b["qws"])
         ds4g.ds4g_moe_permute(b["idx"], self.E, b["xq"], offsets=b["offsets"], row_to_slot=b["r2s"],
                               slot_to_row=b["s2r"], a_perm=b["a"], workspace=b["pws"])
 
@@ -93,6 +112,15 @@ class MoeLayer:
         else:
             ds4g.ds4g_grouped_gemm_fp4(b["a"], b["offsets"], self.E, T, self.w1, 2 * self.I, EPI_NONE, out=b["y1"])
             ds4g.ds4g_swiglu_requant(b["y1"], self.fmt, h_q=b["hq"], h_debug=h_debug)
+
+    def shared_expert(self, b, T, out):
+        """the shared expert on every token's FP8 activations: FC1 with the
+        fused SwiGLU + FP8 requantisation, then FC2 adding each token's row
+        into out (the combine epilogue with one slot per token, weight 1)"""
+        ws1, ws2 = self.shared
+        ds4g.ds4g_grouped_gemm_fp4(b["xq"], b["s_off"], 1, T, ws1, 2 * self.I_s, EPI_SWIGLU_REQUANT, out_q=b["s_hq"])
+        ds4g.ds4g_grouped_gemm_fp4_combine_chained(b["s_hq"], b["s_off"], 1, T, ws2, self.d, b["s_rows"], b["s_w"],
+                                                   out)
 
     def fc2(self, b, T, out=None):
         """grouped FC2 and the routing-weighted combine into out [T][d]"""
@@ -106,6 +134,8 @@ class MoeLayer:
         else:
             ds4g.ds4g_grouped_gemm_fp4(b["hq"], b["offsets"], self.E, T, self.w2, self.d, EPI_NONE, out=b["y2"])
             ds4g.ds4g_moe_combine(b["y2"], b["s2r"][:T * self.k], b["w"], out=out)
+        if self.shared is not None:
+            self.shared_expert(b, T, out)
         return out
 
     def _warm(self, x, logits):

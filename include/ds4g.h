@@ -61,17 +61,20 @@ typedef enum {
     DS4G_ERR_WORKSPACE = 6      /* workspace missing or too small */
 } ds4g_status;
 
-typedef enum { DS4G_MXFP4 = 0, DS4G_NVFP4 = 1 } ds4g_fmt;
+typedef enum { DS4G_MXFP4 = 0, DS4G_NVFP4 = 1, DS4G_MXFP8 = 2 } ds4g_fmt;
 typedef enum { DS4G_BF16 = 0, DS4G_F32 = 1 } ds4g_dtype;
 typedef enum { DS4G_EPI_NONE = 0, DS4G_EPI_SWIGLU_REQUANT = 1 } ds4g_epilogue;
 
-/* An FP4 tensor of `rows` x `K` elements (row-major along K).
- *   data   [rows][K/2] bytes: E2M1 codes (sign, 2 exponent, 1 mantissa bit),
- *          element 2i in the low nibble of byte i, 2i+1 in the high nibble.
- *   scales [rows][K/32] UE8M0 bytes (MXFP4: value 2^(b-127)) or
+/* A block-scaled tensor of `rows` x `K` elements (row-major along K).
+ *   data   MXFP4 / NVFP4: [rows][K/2] bytes of E2M1 codes (sign, 2 exponent,
+ *          1 mantissa bit), element 2i in the low nibble of byte i, 2i+1 in
+ *          the high nibble.  MXFP8 (FP8 activations of the FP8 x FP4
+ *          variant): [rows][K] bytes of E4M3 codes (sign, 4 exponent bits
+ *          with bias 7, 3 mantissa bits; max 448, no infinities).
+ *   scales [rows][K/32] UE8M0 bytes (MXFP4, MXFP8: value 2^(b-127)) or
  *          [rows][K/16] UE4M3 bytes (NVFP4: unsigned E4M3, max 448).
  *   g      NVFP4 only: one fp32 tensor scale (device); element value =
- *          E2M1 * UE4M3 * g.  Ignored (may be NULL) for MXFP4.
+ *          E2M1 * UE4M3 * g.  Ignored (may be NULL) otherwise.
  *   data and scales must be 16-byte aligned. */
 typedef struct {
     uint8_t* data;
@@ -99,6 +102,10 @@ ds4g_status ds4g_check_device(void* stream);
  *     block, X = floor(log2(amax)) - 2 clamped to [-127, 127] (the OCP MX
  *     rule), scale byte X + 127, code = E2M1 round-to-nearest-even of
  *     v * 2^-X, saturating at 6, sign bit kept.
+ *   MXFP8 (the FP8 activations of "[DeepSeek V4] Triton FP4 ..." "Step 0",
+ *     m_grouped_fp8_fp4_gemm_nt_contiguous): per block of 32, X =
+ *     floor(log2(amax)) - 8 clamped to [-127, 127], scale byte X + 127, code
+ *     = E4M3 round-to-nearest-even of v * 2^-X, saturating at 448, sign kept.
  *   NVFP4 (sec. 1, kind::mxf4nvf4: E2M1 + UE4M3 per 16) with a tensor scale
  *     g: g = *g_in if g_in != NULL, else amax(x) / 2688 computed on the
  *     device (1 if amax is 0) and written to out->g; per block
@@ -155,7 +162,8 @@ ds4g_status ds4g_moe_permute(const int32_t* idx, int T, int k, int E, const ds4g
  * tensor scale is derived from amax |x| as ds4g_quantize_mx does).
  * Up to 512 slots (T*k) one kernel does all three steps (decode batches);
  * larger batches run the separate calls' kernels.  Limits as the separate
- * calls: E <= 1024, 1 <= k <= min(E, 32), K % 64 == 0.
+ * calls: E <= 1024, 1 <= k <= min(E, 32), K % 64 == 0.  fmt MXFP4 or NVFP4
+ * (FP8 activations take the three separate calls).
  * Workspace: ds4g_dispatch_workspace_bytes(T, k, E, fmt, g_in != NULL), 16-byte
  * aligned, owned by the caller. */
 size_t ds4g_dispatch_workspace_bytes(int T, int k, int E, int fmt, int has_g_in);
@@ -173,7 +181,11 @@ ds4g_status ds4g_moe_dispatch(const float* logits, const void* x, int dtype, int
  *             NVFP4: times a->g[0] * w->g[e])
  * w has E*N rows of K columns, same fmt as a; for NVFP4 w->g holds one fp32
  * tensor scale per expert ([E] floats, each expert's weight matrix being its
- * own tensor).
+ * own tensor).  FP8 activations (a->fmt DS4G_MXFP8, the FP8 x FP4 GEMM of
+ * "[DeepSeek V4] Triton FP4 ..." "Step 0") take MXFP4 weights (routed
+ * experts) or MXFP8 weights (a shared expert kept in 8 bits, "DGX Spark
+ * native FP4 ..." sec. 2); with them SWIGLU_REQUANT writes h as MXFP8 (the
+ * "SwiGLU + FP8 quant" step of "Moore Threads ...").
  * epilogue DS4G_EPI_NONE: out = y, fp32 [S][N].
  * epilogue DS4G_EPI_SWIGLU_REQUANT (FC1 with N = 2I): columns [0, I) are the
  *   gate and [I, 2I) the up projection; h = silu(gate) * up (fp32,
@@ -197,10 +209,8 @@ ds4g_status ds4g_moe_dispatch(const float* logits, const void* x, int dtype, int
  *     tiles of 96 gate + 96 up columns (the last one ragged), two
  *     accumulators;
  *   otherwise: a dp4a weight-streaming kernel (any segment length).
- *   With DS4G_TC_PAIR=1 in the environment the > 16-row tensor-core kernel
- *   runs on CTA pairs (tcgen05 cta_group::2, 256-row tiles, each CTA loading
- *   its own 128 rows and half of the weight rows); same results within the
- *   GEMM bound, slower on the layer shapes measured, so off by default.
+ *   FP8 activations always take the 128-row tensor-core kernel
+ *   (kind::mxf8f6f4): K % 512 == 0 and the N rule above, else DS4G_ERR_SHAPE.
  * Shapes: K % 64 == 0; NONE needs N % 64 == 0 unless a tensor-core kernel
  *   takes the call; SWIGLU_REQUANT needs I % 32 == 0.  offsets[E] must
  *   equal S. */
@@ -217,7 +227,11 @@ ds4g_status ds4g_grouped_gemm_fp4(const ds4g_fp4* a, const int32_t* offsets, int
  * order in which a token's k rows are summed is not fixed (results can
  * differ in the last bits from run to run; ds4g_moe_combine is the
  * deterministic alternative).  Kernel choice and shapes as for
- * ds4g_grouped_gemm_fp4 with DS4G_EPI_NONE. */
+ * ds4g_grouped_gemm_fp4 with DS4G_EPI_NONE.  When the output is larger than
+ * about half of L2 (T * N * 4 bytes over ~60 MB, prefill sizes) the
+ * tensor-core kernel walks its tiles in bands of output columns, all experts
+ * of a band before the next, so that a token's k additions to those columns
+ * meet in L2. */
 ds4g_status ds4g_grouped_gemm_fp4_combine(const ds4g_fp4* a, const int32_t* offsets, int E,
                                           int max_rows_per_expert, const ds4g_fp4* w, int N,
                                           const int32_t* row_to_slot, const float* route_w, int T, int k,
@@ -256,7 +270,8 @@ ds4g_status ds4g_zero_fill(void* p, size_t bytes, void* stream);
  * The SwiGLU + requantisation epilogue as its own step ("Moore Threads ..."
  * fused SwiGLU + quant pattern): y1 fp32 [rows][2I] -> h_q (fmt, [rows][I]);
  * h_debug (nullable) receives h fp32.  For NVFP4 *h_q->g is the static
- * tensor scale (input).  I % 32 == 0. */
+ * tensor scale (input).  I % 32 == 0; fmt MXFP4 or NVFP4 (with FP8
+ * activations h is requantised only in FC1's fused epilogue). */
 ds4g_status ds4g_swiglu_requant(const float* y1, int64_t rows, int I, int fmt, ds4g_fp4* h_q,
                                 float* h_debug, void* stream);
 

@@ -199,7 +199,7 @@ def grouped_gemm(a, offsets, w, N, rows=None, cols=None):
     offsets = _c(offsets, np.int32)
     E = offsets.shape[0] - 1
     S = ad.shape[0]
-    K = ad.shape[1] * 2
+    K = _K_of(a)
     r0, r1 = rows if rows is not None else (0, S)
     c0, c1 = cols if cols is not None else (0, N)
     out = np.full((S, N), np.nan)

@@ -443,7 +443,7 @@ void orc_grouped_gemm(const uint8_t* a_data, const uint8_t* a_scales, double g_a
         double* o = (double*)malloc(sizeof(double) * (size_t)(nr * ncols));
         double* s = abssum ? (double*)malloc(sizeof(double) * (size_t)(nr * ncols)) : NULL;
         orc_expert_gemm_rows(a_data, a_scales, g_a, rows, nr,
-                             w_data + (int64_t)e * N * (K / 2), w_scales + (int64_t)e * N * (K / blk),
+                             w_data + (int64_t)e * N * row_bytes(fmt, K), w_scales + (int64_t)e * N * (K / blk),
                              g_w, n_begin, n_end, K, fmt, o, s);
         for (int64_t i = 0; i < nr; ++i) {
             for (int c = 0; c < ncols; ++c) {

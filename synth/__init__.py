@@ -14,6 +14,7 @@ expert's weights can be regenerated on its own):
     STREAM_BIAS    per-expert router bias [E]
     STREAM_W1 + e  expert e FC1 weights [2I][d] (gate rows then up rows)
     STREAM_W2 + e  expert e FC2 weights [d][I]
+    STREAM_WS1 / STREAM_WS2  the shared expert's FC1 [2I][d] / FC2 [d][I] weights
 """
 import ctypes
 import os
@@ -28,6 +29,8 @@ STREAM_BIAS = 3
 STREAM_AUX = 4
 STREAM_W1 = 1 << 20
 STREAM_W2 = 2 << 20
+STREAM_WS1 = 1 << 22
+STREAM_WS2 = (1 << 22) + 1
 
 _host = None
 _cuda = None

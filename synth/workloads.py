@@ -19,13 +19,13 @@ from dataclasses import dataclass
 
 import numpy as np
 
-from . import STREAM_BIAS, STREAM_LOGITS, STREAM_W1, STREAM_W2, STREAM_X
+from . import STREAM_BIAS, STREAM_LOGITS, STREAM_W1, STREAM_W2, STREAM_WS1, STREAM_WS2, STREAM_X
 
 W_SIGMA = 0.02
 BIAS_SIGMA = 1.5
 H_CAL = 128.0
 G_H = float(np.float32(np.float32(H_CAL) / np.float32(2688.0)))
-MX, NV = 0, 1
+MX, NV, MX8 = 0, 1, 2
 
 
 @dataclass(frozen=True)
@@ -39,6 +39,11 @@ class Workload:
     fmt: int
     bias_sigma: float
     dense: bool = False   # one expert, FC1-shaped single GEMM only (N = I rows)
+    act_fmt: int = -1     # activations' format: the weights' by default; 2 = MXFP8 (FP8 x FP4)
+
+    @property
+    def afmt(self):
+        return self.fmt if self.act_fmt < 0 else self.act_fmt
 
     @property
     def S(self):
@@ -61,6 +66,14 @@ WORKLOADS = {
     # profiling stand-in for "prefill": same per-expert shapes and skew, 64
     # experts (1.5 GB of weights) so that ncu's multi-pass replay stays small
     "prof_prefill": Workload("prof_prefill", T=512, E=64, k=6, d=7168, I=2048, fmt=MX, bias_sigma=BIAS_SIGMA),
+    # FP8 activations (MXFP8: E4M3 + UE8M0 per 32) x MXFP4 weights, the
+    # m_grouped_fp8_fp4_gemm_nt_contiguous variant, at the prefill layer's shape
+    "prefill_fp8": Workload("prefill_fp8", T=2048, E=256, k=6, d=7168, I=2048, fmt=MX, bias_sigma=BIAS_SIGMA,
+                            act_fmt=MX8),
+    # the same for "prefill16k": NVFP4, 64 experts (1.6 GB of weights) and
+    # 4096 tokens, i.e. the same 384 rows per expert on average
+    "prof_prefill16k": Workload("prof_prefill16k", T=4096, E=64, k=6, d=7168, I=2048, fmt=NV,
+                                bias_sigma=BIAS_SIGMA),
 }
 
 
@@ -73,6 +86,18 @@ def host_w1(wl: Workload, e: int, seed: int = 0):
 def host_w2(wl: Workload, e: int, seed: int = 0):
     from . import normal_f32
     return normal_f32((wl.d, wl.I), seed, STREAM_W2 + e, W_SIGMA)
+
+
+def host_ws1(wl: Workload, seed: int = 0):
+    """the shared expert's FC1 weights, fp32 [2I][d] ~ N(0, 0.02)"""
+    from . import normal_f32
+    return normal_f32((2 * wl.I, wl.d), seed, STREAM_WS1, W_SIGMA)
+
+
+def host_ws2(wl: Workload, seed: int = 0):
+    """the shared expert's FC2 weights, fp32 [d][I] ~ N(0, 0.02)"""
+    from . import normal_f32
+    return normal_f32((wl.d, wl.I), seed, STREAM_WS2, W_SIGMA)
 
 
 def host_x_bits(wl: Workload, seed: int = 0):

@@ -46,6 +46,23 @@ def unpack(data):
     return out
 
 
+def swiglu_eval_bound(g, h):
+    """Bound on |h_gpu - silu(g) u| for the kernels' fp32 evaluation
+    g u / (1 + e^-g) from their own g and u, with the hardware's fast
+    exponential and division.  Documented bounds (CUDA C Programming Guide,
+    intrinsic functions): __expf(x) within 2 + floor(1.173 |x|) ulp,
+    __fdividef within 2 ulp for divisors in [2^-126, 2^126], 0 when the
+    divisor is beyond 2^126 (|g| above ~87, where |h| < 1e-36).  To first
+    order the relative error is (2 + 1.173 |g|) 2^-23 from e^-g, plus
+    2^-24 for the add, 2^-24 for g u and 2^-22 for the division:
+    (5 + 1.173 |g|) 2^-23; (6 + 1.2 |g|) 2^-23 leaves room for the
+    second-order terms.  A further 2^-22 |h| covers the NVFP4 codes, which
+    the fused epilogues take from h times the correctly rounded reciprocal of
+    the block's divisor (within 1.5 ulp of the quotient)."""
+    g = np.abs(np.asarray(g, np.float64))
+    return ((6.0 + 1.2 * g) * 2.0 ** -23 + 2.0 ** -22) * np.abs(h) + 1e-30
+
+
 def assert_gemm_close(gpu, ref, abssum, what=""):
     gpu = np.asarray(gpu, np.float64)
     bound = GEMM_REL * abssum + GEMM_ABS

@@ -50,3 +50,33 @@ def test_byte_accounting_per_expert():
     act_n = (d // 2 + d // 16) + (I // 2 + I // 16)
     w2_n = d * (I // 2 + I // 16)
     assert (n["fc1_bytes"] - act_n) + w2_n == 24_772_608   # NVFP4: UE4M3 per 16, W1 + W2 of one expert
+
+
+def test_reference_arm_dense_gemm():
+    """--workload dense_m1: the oracle's quantisation + GEMM, reported as time
+    per call (lower is better)"""
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload",
+                        "dense_m1", "--steps", "1", "--warmup", "0"], capture_output=True, text=True, timeout=600,
+                       cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.strip().startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["unit"] == "us" and d["higher_is_better"] is False and d["value"] > 0
+    assert d["config"]["workload"].startswith("dense FP4 GEMM M=1 N=4096 K=7168")
+
+
+def test_default_workload_is_the_largest_layer():
+    """with no flags the bench times the largest configuration, prefill
+    T = 16384 NVFP4"""
+    import argparse
+    old = sys.argv
+    sys.argv = ["bench.py"]
+    try:
+        a = bench.parse()
+    finally:
+        sys.argv = old
+    assert a.workload == "prefill16k" and a.steps is None and a.warmup >= 3
+    from synth import workloads
+    wl = workloads.WORKLOADS[a.workload]
+    assert (wl.T, wl.fmt) == (16384, 1)

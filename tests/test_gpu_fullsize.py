@@ -30,7 +30,7 @@ import torch
 
 import oracle
 import synth
-from parity_helpers import assert_gemm_close, bf16_dev, check_requant, dev, from_dev
+from parity_helpers import assert_gemm_close, bf16_dev, check_requant, dev, from_dev, swiglu_eval_bound
 from synth import workloads
 
 pytestmark = pytest.mark.gpu
@@ -72,10 +72,9 @@ def _h_bound(g, u, ag, au):
     dg, du = 1e-5 * ag + 1e-6, 1e-5 * au + 1e-6
     sig = 1.0 / (1.0 + np.exp(-g))
     h = g * sig * u
-    # fp32 rounding of (g / (1 + expf(-g))) * u: expf within 2 ulp (CUDA C
-    # Programming Guide, mathematical functions appendix), add / divide /
-    # multiply IEEE round-to-nearest: at most 3.5 ulp, below 8 |h| 2^-24
-    return h, np.abs(sig * (1 + g * (1 - sig))) * np.abs(u) * dg + np.abs(g * sig) * du + 8 * np.abs(h) * 2.0 ** -24 + 1e-30
+    # the GEMM's bound on g and u carried through silu(g) u, plus the fp32
+    # evaluation of h from the GPU's own g and u (swiglu_eval_bound)
+    return h, np.abs(sig * (1 + g * (1 - sig))) * np.abs(u) * dg + np.abs(g * sig) * du + swiglu_eval_bound(g, h)
 
 
 def _chain(wl, xq, idx, w, toks, gpu=None):

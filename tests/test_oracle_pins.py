@@ -480,3 +480,23 @@ def test_encoders_saturate_far_beyond_the_range():
     for y in (448.0, 1e10, 1e30, 1e300):
         assert oracle.e4m3_encode(y) == 0x7E and oracle.e4m3_encode(-y) == 0xFE
         assert oracle.ue4m3_encode(y) == 0x7E
+
+
+def test_grouped_gemm_fp8_weights_bruteforce_tiny():
+    """MXFP8 activations x MXFP8 weights (the shared expert's FP8 weights),
+    grouped over experts: numpy's matmul of the dequantised operands, exact"""
+    E, N, K = 3, 8, 128
+    a = synth.normal_f32((7, K), seed=0, stream=88, sigma=1.0)
+    w = synth.normal_f32((E * N, K), seed=0, stream=87, sigma=0.5)
+    aq, wq = oracle.quantize(a, oracle.MX8), oracle.quantize(w, oracle.MX8)
+    offsets = np.array([0, 2, 2, 7], np.int32)
+    out, ab = oracle.grouped_gemm(aq, offsets, wq, N)
+
+    def deq(t):
+        return torch.from_numpy(t.data).view(torch.float8_e4m3fn).double().numpy() * \
+            np.ldexp(1.0, np.repeat(t.scales.astype(np.int64), 32, axis=1) - 127)
+    A, W = deq(aq), deq(wq)
+    for e in range(E):
+        for r in range(offsets[e], offsets[e + 1]):
+            assert np.array_equal(out[r], W[e * N:(e + 1) * N] @ A[r])
+            assert np.array_equal(ab[r], np.abs(W[e * N:(e + 1) * N]) @ np.abs(A[r]))
