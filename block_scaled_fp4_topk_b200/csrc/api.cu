@@ -228,6 +228,7 @@ static ds4g_status grouped_gemm(const ds4g_fp4* a, const int32_t* offsets, int E
     g.topk = k;
     g.chained = chained ? 1 : 0;
     g.band_tiles = 0;
+    g.ksplit = 1;
     if (epilogue == kEpiCombine && T > 0 && !chained) {
         cudaError_t e = cudaMemsetAsync(out, 0, sizeof(float) * (size_t)T * N, S(stream));
         if (e != cudaSuccess) return DS4G_ERR_CUDA;
@@ -265,6 +266,78 @@ ds4g_status ds4g_grouped_gemm_fp4_combine_chained(const ds4g_fp4* a, const int32
     if (T > 0 && (!row_to_slot || !route_w || !out)) return DS4G_ERR_INVALID_ARG;
     return grouped_gemm(a, offsets, E, max_rows_per_expert, w, N, kEpiCombine, out, nullptr, nullptr, row_to_slot,
                         route_w, k, T, stream, true);
+}
+
+ds4g_status ds4g_moe_ffn_fp4(const ds4g_fp4* a, const int32_t* offsets, int E, int max_rows_per_expert,
+                             const ds4g_fp4* w1, const ds4g_fp4* w2, int d, int I, ds4g_fp4* h_q,
+                             const int32_t* row_to_slot, const float* route_w, int T, int k, float* out,
+                             int32_t* counters, void* stream)
+{
+    if (!a || !offsets || !w1 || !w2 || !h_q || E < 1 || d < 1 || I < 1 || T < 0 || k < 1 ||
+        max_rows_per_expert < 0)
+        return DS4G_ERR_INVALID_ARG;
+    const int fmt = a->fmt;
+    if (fmt != DS4G_MXFP4 && fmt != DS4G_NVFP4) return DS4G_ERR_INVALID_ARG;
+    if (a->rows != (int64_t)T * k) return DS4G_ERR_SHAPE;
+    if (max_rows_per_expert > 16 || !ffn_dtc_supports(fmt, d, I, E)) return DS4G_ERR_SHAPE;
+    ds4g_status st = check_fp4(a, a->rows, d, fmt, true);
+    if (st != DS4G_OK) return st;
+    st = check_fp4(w1, (int64_t)E * 2 * I, d, fmt, true);
+    if (st != DS4G_OK) return st;
+    st = check_fp4(w2, (int64_t)E * d, I, fmt, true);
+    if (st != DS4G_OK) return st;
+    st = check_fp4(h_q, a->rows, I, fmt, true);
+    if (st != DS4G_OK) return st;
+    if ((int64_t)E * 2 * I > 0x7FFFFFFF || (int64_t)E * d > 0x7FFFFFFF) return DS4G_ERR_SHAPE;
+    if (T > 0 && (!row_to_slot || !route_w || !out || !counters || !aligned16(out))) return DS4G_ERR_INVALID_ARG;
+    GemmArgs g1 = {};
+    g1.a_data = a->data;
+    g1.a_scales = a->scales;
+    g1.a_g = a->g;
+    g1.S = a->rows;
+    g1.offsets = offsets;
+    g1.E = E;
+    g1.w_data = w1->data;
+    g1.w_scales = w1->scales;
+    g1.w_g = w1->g;
+    g1.N = 2 * I;
+    g1.K = d;
+    g1.fmt = fmt;
+    g1.epilogue = DS4G_EPI_SWIGLU_REQUANT;
+    g1.oq_data = h_q->data;
+    g1.oq_scales = h_q->scales;
+    g1.oq_g = h_q->g;
+    g1.max_rows = max_rows_per_expert;
+    g1.ksplit = 1;
+    GemmArgs g2 = {};
+    g2.a_data = h_q->data;
+    g2.a_scales = h_q->scales;
+    g2.a_g = h_q->g;
+    g2.S = a->rows;
+    g2.offsets = offsets;
+    g2.E = E;
+    g2.w_data = w2->data;
+    g2.w_scales = w2->scales;
+    g2.w_g = w2->g;
+    g2.N = d;
+    g2.K = I;
+    g2.fmt = fmt;
+    g2.epilogue = kEpiCombine;
+    g2.out = out;
+    g2.max_rows = max_rows_per_expert;
+    g2.r2s = row_to_slot;
+    g2.route_w = route_w;
+    g2.topk = k;
+    g2.ksplit = 1;
+    return cuda_status(launch_ffn_dtc(g1, g2, counters, S(stream)));
+}
+
+ds4g_status ds4g_segment_ids(const int32_t* offsets, int nseg, int modulo, int64_t rows, int32_t* out,
+                             void* stream)
+{
+    if (nseg < 1 || modulo < 1 || rows < 0) return DS4G_ERR_INVALID_ARG;
+    if (rows > 0 && (!offsets || !out)) return DS4G_ERR_INVALID_ARG;
+    return cuda_status(launch_segment_ids(offsets, nseg, modulo, rows, out, S(stream)));
 }
 
 ds4g_status ds4g_zero_fill(void* p, size_t bytes, void* stream)

@@ -158,6 +158,7 @@ __host__ __device__ constexpr bool fp8_act(int fmt) { return fmt == DS4G_MXFP8 |
 // internal epilogue mode: FC2 with the weighted combine fused (adds into the
 // token outputs instead of storing per-row results)
 constexpr int kEpiCombine = 2;
+constexpr int kEpiFfn = 3;        // decode kernel: FC1 + SwiGLU + requantisation, then FC2 + combine, one launch
 
 __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d)
 {

@@ -47,6 +47,7 @@ constexpr int BM = 128;            // tile rows (tokens)
 constexpr int BKB = 128;           // bytes of K per stage per row (256 FP4)
 constexpr int STAGES = 4;
 constexpr int kEpiWarps = 8;
+constexpr int kProducer2Warp = 4 + kEpiWarps;   // the second TMA producer (two MMA issuers)
 constexpr int A_BYTES = BM * BKB;  // 16 KB
 constexpr int kTmemCols = 512;
 constexpr int kColAcc = 0;
@@ -85,7 +86,7 @@ struct Cfg {
     static constexpr int SF_STAGES = 2 * NISS;
     static constexpr int COL_SFA = NACC * TBN;
     static_assert(COL_SFA + NISS * SF_COLS <= 512, "TMEM columns");
-    static constexpr int THREADS = 32 * (4 + kEpiWarps);
+    static constexpr int THREADS = 32 * (4 + kEpiWarps + (NISS == 2 ? 1 : 0));
     static constexpr int SF_ROW = KPS * WPS * 4;                     // scale bytes per row per scale stage
     static constexpr int SFA_BYTES = BM * SF_ROW;                    // one scale stage of A
     static constexpr int SFB_BYTES = 256 * SF_ROW;                   // one scale stage of W (two 128-row groups)
@@ -107,7 +108,7 @@ struct Cfg {
     static constexpr int STAGE_OFF = DATA_BYTES + SF_BYTES + BAR_BYTES + 2 * PREFIX_BYTES;
     static constexpr size_t SMEM = 1024 + (size_t)STAGE_OFF + STAGE_BYTES;
     static_assert(SMEM <= 232448, "shared memory per CTA");
-    static_assert((2 * NST + 3 * SF_STAGES + 4) * 8 + 16 <= BAR_BYTES, "barrier block");
+    static_assert((2 * NST + 3 * SF_STAGES + 6) * 8 + 16 <= BAR_BYTES, "barrier block");
 };
 
 // ---- PTX wrappers ----------------------------------------------------------
@@ -468,7 +469,8 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
     uint64_t* sf_empty = sf_ready + SF_STAGES;             // [SF_STAGES] MMAs done with the scales
     uint64_t* tmem_full = sf_empty + SF_STAGES;            // [NACC] accumulator complete
     uint64_t* tmem_empty = tmem_full + 2;                  // [NACC] accumulator drained
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tmem_empty + 2);
+    uint64_t* drain = tmem_empty + 2;                      // [NISS] each issuer's tensor-core work finished
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int32_t* total_tiles = reinterpret_cast<int32_t*>(tmem_slot + 2);
     int32_t* prefix = reinterpret_cast<int32_t*>(smem + C::DATA_BYTES + C::SF_BYTES + C::BAR_BYTES);
@@ -478,8 +480,13 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
     const int E = p.E;
     const int64_t K = p.K;
     constexpr int KPS = C::KPS;
-    const int nks = (int)ceil_div(K, C::KE);
-    const int nsfs = (nks + KPS - 1) / KPS;      // scale stages per tile
+    // split K (plain epilogue, few tiles): every tile comes ksplit times,
+    // part q taking K stages [q nks, (q + 1) nks) and adding its partial sums
+    // into the zeroed output (the host splits only into equal parts of whole
+    // scale stages)
+    const int ksplit = (EPI == DS4G_EPI_NONE && p.ksplit > 1) ? p.ksplit : 1;
+    const int nks = (int)ceil_div(K, C::KE) / ksplit;   // K stages per tile (part)
+    const int nsfs = (nks + KPS - 1) / KPS;              // scale stages per tile (part)
     const int I = p.N / 2;
     // SwiGLU: the last tile may be ragged (I % (TBN/2) != 0); its columns past
     // I are computed from other rows and never stored
@@ -504,6 +511,8 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
             mbar_init(smem_u32(&tmem_full[b2]), 1);
             mbar_init(smem_u32(&tmem_empty[b2]), 32 * kEpiWarps);
         }
+        mbar_init(smem_u32(&drain[0]), 1);
+        mbar_init(smem_u32(&drain[1]), 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -547,7 +556,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
         }
         if (lane == 31) {
             prefix[E] = incl;
-            int32_t tot = incl * n_tiles;
+            int32_t tot = incl * n_tiles * ksplit;
             if ((int64_t)soff[E] > p.S) {   // inconsistent offsets: do nothing
                 raise_error(kErrBadOffsets);
                 tot = 0;
@@ -561,61 +570,69 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
     const uint32_t tmem = *tmem_slot;
     const int64_t ntiles = *total_tiles;
 
-    if (warp == 0) {
-        // ================= TMA producer =================
-        // This CTA's tiles in groups of NISS consecutive ones; the stages of a
-        // group are interleaved (K stage by K stage, member by member) so that
-        // each MMA issuer finds its next stage while the other works.
+    // Ring slots belong to tile group members: member m of a group (issuer m,
+    // producer m) uses data slots m, m + NISS, ... and scale slots m, m +
+    // NISS, counting its own uses l = 0, 1, ... (slot NISS (l % depth) + m,
+    // phase (l / depth) & 1).  Each slot then has one producer and one
+    // consumer taking its uses in order, which the parity waits require.
+    constexpr int DPM = STAGES / NISS;       // data slots per member
+    constexpr int SPM = SF_STAGES / NISS;    // scale slots per member
+    static_assert(DPM * NISS == STAGES && SPM * NISS == SF_STAGES && SPM == 2, "ring split");
+
+    if (warp == 0 || (NISS == 2 && warp == kProducer2Warp)) {
+        // ================= TMA producer(s) =================
+        // This CTA's tiles come in groups of NISS consecutive ones.  Producer
+        // pp (warp 0, and warp 12 with two issuers) loads the data and scale
+        // stages of member pp of each group, the ones issuer pp consumes.  A
+        // thread that has issued copies and then waits on a barrier first
+        // waits for its copies to land; with two producers one's copies are
+        // in flight while the other waits for a free slot.
         if (lane == 0) {
-            uint32_t it = 0, sit = 0;
+            const int pp = (warp == 0) ? 0 : 1;
+            uint32_t ld = 0, ls = 0;           // this member's data / scale uses issued
             bool ok = true;
             for (int64_t j0 = 0; ok; j0 += NISS) {
                 const int64_t t0 = tile0 + j0 * tstride;
                 if (t0 >= ntiles) break;
                 const int gsz = (NISS == 2 && t0 + tstride < ntiles) ? 2 : 1;
-                Tile tls[NISS];
-                int64_t y0s[NISS], y1s[NISS];
-#pragma unroll
-                for (int u = 0; u < NISS; ++u) {
-                    if (u < gsz) {
-                        tls[u] = tile_of(t0 + u * tstride, prefix, soff, E, n_tiles, nb);
-                        w_rows<EPI, TBN>(tls[u], p.N, I, y0s[u], y1s[u]);
+                if (pp >= gsz) break;                                   // the CTA's last group has one member
+                const int64_t t = t0 + pp * tstride;
+                const Tile tl = tile_of(t / ksplit, prefix, soff, E, n_tiles, nb);
+                const int kb = (int)(t % ksplit) * nks;                  // first K stage of this part
+                int64_t y0, y1;
+                w_rows<EPI, TBN>(tl, p.N, I, y0, y1);
+                for (int ks = 0; ks < nks; ++ks) {
+                    if ((ks % KPS) == 0) {
+                        const int r = NISS * (int)(ls % SPM) + pp;
+                        if (!mbar_wait(smem_u32(&sf_empty[r]), ((ls / SPM) & 1) ^ 1, abort_flag)) { ok = false; break; }
+                        const uint32_t fb = smem_u32(&sf_full[r]);
+                        mbar_arrive_tx(fb, C::SFA_BYTES + TBN * C::SF_ROW);
+                        const int x = ((kb + ks) / KPS) * C::SF_ROW;
+                        tma_load_2d(smem_u32(sSFA + r * C::SFA_BYTES), &map_sfa, fb, x, (int)tl.m0);
+                        tma_load_2d(smem_u32(sSFB + r * C::SFB_BYTES), &map_sfb, fb, x, (int)y0);
+                        tma_load_2d(smem_u32(sSFB + r * C::SFB_BYTES + C::HALF * C::SF_ROW), &map_sfb, fb, x, (int)y1);
+                        ++ls;
                     }
-                }
-                for (int ks = 0; ks < nks && ok; ++ks) {
-#pragma unroll
-                    for (int u = 0; u < NISS; ++u) {
-                        if (u >= gsz || !ok) continue;
-                        const Tile& tl = tls[u];
-                        if ((ks % KPS) == 0) {
-                            const int r = sit % SF_STAGES;
-                            if (!mbar_wait(smem_u32(&sf_empty[r]), ((sit / SF_STAGES) & 1) ^ 1, abort_flag)) { ok = false; break; }
-                            const uint32_t fb = smem_u32(&sf_full[r]);
-                            mbar_arrive_tx(fb, C::SFA_BYTES + TBN * C::SF_ROW);
-                            const int x = (ks / KPS) * C::SF_ROW;
-                            tma_load_2d(smem_u32(sSFA + r * C::SFA_BYTES), &map_sfa, fb, x, (int)tl.m0);
-                            tma_load_2d(smem_u32(sSFB + r * C::SFB_BYTES), &map_sfb, fb, x, (int)y0s[u]);
-                            tma_load_2d(smem_u32(sSFB + r * C::SFB_BYTES + C::HALF * C::SF_ROW), &map_sfb, fb, x, (int)y1s[u]);
-                            ++sit;
-                        }
-                        const int s = it % STAGES;
-                        if (!mbar_wait(smem_u32(&empty[s]), ((it / STAGES) & 1) ^ 1, abort_flag)) { ok = false; break; }
-                        const uint32_t fb = smem_u32(&full[s]);
-                        mbar_arrive_tx(fb, A_BYTES + C::B_TX);
-                        tma_load_2d(smem_u32(sA + s * A_BYTES), &map_a, fb, ks * BKB, (int)tl.m0);
-                        tma_load_2d(smem_u32(sB + s * B_BYTES), &map_b, fb, ks * BKB, (int)y0s[u]);
-                        tma_load_2d(smem_u32(sB + s * B_BYTES + B_BYTES / 2), &map_b, fb, ks * BKB, (int)y1s[u]);
-                        ++it;
-                    }
+                    const int s = NISS * (int)(ld % DPM) + pp;
+                    if (!mbar_wait(smem_u32(&empty[s]), ((ld / DPM) & 1) ^ 1, abort_flag)) { ok = false; break; }
+                    const uint32_t fb = smem_u32(&full[s]);
+                    mbar_arrive_tx(fb, A_BYTES + C::B_TX);
+                    const int kx = (kb + ks) * BKB;
+                    tma_load_2d(smem_u32(sA + s * A_BYTES), &map_a, fb, kx, (int)tl.m0);
+                    tma_load_2d(smem_u32(sB + s * B_BYTES), &map_b, fb, kx, (int)y0);
+                    tma_load_2d(smem_u32(sB + s * B_BYTES + B_BYTES / 2), &map_b, fb, kx, (int)y1);
+                    ++ld;
                 }
             }
             if (!ok) {
-                // let the copies already issued land before the CTA goes away
+                // let this member's copies in flight land before the CTA goes
+                // away: its latest uses of each slot (earlier ones completed
+                // before their slot was refilled)
                 volatile int never = 0;
-                for (uint32_t j = (it > STAGES ? it - STAGES : 0); j < it; ++j)
-                    mbar_wait(smem_u32(&full[j % STAGES]), (j / STAGES) & 1, &never);
-                for (uint32_t j = (sit > SF_STAGES ? sit - SF_STAGES : 0); j < sit; ++j)
-                    mbar_wait(smem_u32(&sf_full[j % SF_STAGES]), (j / SF_STAGES) & 1, &never);
+                for (uint32_t l = (ld > (uint32_t)DPM ? ld - DPM : 0u); l < ld; ++l)
+                    mbar_wait(smem_u32(&full[NISS * (int)(l % DPM) + pp]), (l / DPM) & 1, &never);
+                for (uint32_t l = (ls > (uint32_t)SPM ? ls - SPM : 0u); l < ls; ++l)
+                    mbar_wait(smem_u32(&sf_full[NISS * (int)(l % SPM) + pp]), (l / SPM) & 1, &never);
             }
         }
         __syncwarp();
@@ -630,88 +647,101 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
             const uint32_t ibase = idesc_base<FMT, TBN>();
             const uint32_t col_sfa = tmem + C::COL_SFA + pi * C::SF_COLS;
             const uint32_t col_sfb = col_sfa + 4 * C::WPS;
-            uint32_t it_base = 0, sit_base = 0;
+            uint32_t ld = 0, ls = 0;           // this member's data / scale uses consumed
             bool ok = true;
             for (int64_t j0 = 0; ok; j0 += NISS) {
                 const int64_t t0 = tile0 + j0 * tstride;
                 if (t0 >= ntiles) break;
                 const int gsz = (NISS == 2 && t0 + tstride < ntiles) ? 2 : 1;
-                if (pi < gsz) {
-                    const int64_t jt = j0 + pi;                        // this CTA's local tile index
-                    const int buf = (NISS == 2) ? pi : (int)(jt % NACC);
-                    const uint32_t use = (NISS == 2) ? (uint32_t)(j0 / 2) : (uint32_t)(jt / NACC);
-                    if (!mbar_wait(smem_u32(&tmem_empty[buf]), (use & 1) ^ 1, abort_flag)) { ok = false; break; }
-                    const uint32_t acc = tmem + kColAcc + buf * TBN;
-                    tc_fence_after();
-                    for (int ks = 0; ks < nks; ++ks) {
-                        const uint32_t it = it_base + (uint32_t)(ks * gsz + pi);
-                        const uint32_t sit = sit_base + (uint32_t)((ks / KPS) * gsz + pi);
-                        const int r = sit % SF_STAGES;
-                        if ((ks % KPS) == 0) {
-                            if (!mbar_wait(smem_u32(&sf_ready[r]), (sit / SF_STAGES) & 1, abort_flag)) { ok = false; break; }
-                        }
-                        const int s = it % STAGES;
-                        if (!mbar_wait(smem_u32(&full[s]), (it / STAGES) & 1, abort_flag)) { ok = false; break; }
-                        tc_fence_after();
-                        // this K stage's scale words -> TMEM
-                        const int w0 = (ks % KPS) * C::WPS;
-                        const uint32_t sfa_s = smem_u32(sSFA + r * C::SFA_BYTES);
-                        const uint32_t sfb_s = smem_u32(sSFB + r * C::SFB_BYTES);
-#pragma unroll
-                        for (int c = 0; c < C::WPS; ++c) {
-                            utccp(col_sfa + 4 * c, desc_sf(sfa_s + (w0 + c) * 512));
-                            utccp(col_sfb + 8 * c, desc_sf(sfb_s + ((w0 + c) * 2 + 0) * 512));
-                            utccp(col_sfb + 8 * c + 4, desc_sf(sfb_s + ((w0 + c) * 2 + 1) * 512));
-                        }
-                        const int64_t krem = K - (int64_t)ks * C::KE;
-                        const int nmma = krem >= C::KE ? 4 : (int)(krem / (C::KE / 4));
-                        const uint32_t a_s = smem_u32(sA + s * A_BYTES);
-                        const uint32_t b_s = smem_u32(sB + s * B_BYTES);
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            if (j < nmma) {
-                                // scale word (4 TMEM columns) and byte of MMA j:
-                                // MX K = 64 takes 2 scales (bytes 0-1 / 2-3 of
-                                // word j / 2), NV K = 64 all 4 of word j, MXFP8
-                                // K = 32 byte j of the stage's one word
-                                const int c = (FMT == DS4G_MXFP4) ? (j >> 1) : (FMT == DS4G_NVFP4 ? j : 0);
-                                const uint32_t sfid = (FMT == DS4G_MXFP4) ? (uint32_t)((j & 1) * 2)
-                                                                         : (FMT == DS4G_NVFP4 ? 0u : (uint32_t)j);
-                                const uint32_t idesc = ibase | (sfid << 4) | (sfid << 29);
-                                mma<FMT>(acc, desc_sw128(a_s + 32 * j), desc_sw128(b_s + 32 * j), idesc,
-                                         (ks > 0 || j > 0) ? 1u : 0u, col_sfa + 4 * c, col_sfb + 8 * c);
-                            }
-                        }
-                        tc_commit(smem_u32(&empty[s]));
-                        if ((ks % KPS) == KPS - 1 || ks == nks - 1) tc_commit(smem_u32(&sf_empty[r]));
+                if (pi >= gsz) break;
+                const int64_t jt = j0 + pi;                        // this CTA's local tile index
+                const int buf = (NISS == 2) ? pi : (int)(jt % NACC);
+                const uint32_t use = (NISS == 2) ? (uint32_t)(j0 / 2) : (uint32_t)(jt / NACC);
+                if (!mbar_wait(smem_u32(&tmem_empty[buf]), (use & 1) ^ 1, abort_flag)) break;
+                const uint32_t acc = tmem + kColAcc + buf * TBN;
+                const int kb = (int)((t0 + pi * tstride) % ksplit) * nks;   // first K stage of this part
+                tc_fence_after();
+                int r = 0;
+                for (int ks = 0; ks < nks; ++ks) {
+                    if ((ks % KPS) == 0) {
+                        r = NISS * (int)(ls % SPM) + pi;
+                        if (!mbar_wait(smem_u32(&sf_ready[r]), (ls / SPM) & 1, abort_flag)) { ok = false; break; }
+                        ++ls;
                     }
-                    if (!ok) break;
-                    tc_commit(smem_u32(&tmem_full[buf]));
+                    const int s = NISS * (int)(ld % DPM) + pi;
+                    if (!mbar_wait(smem_u32(&full[s]), (ld / DPM) & 1, abort_flag)) { ok = false; break; }
+                    ++ld;
+                    tc_fence_after();
+                    // this K stage's scale words -> TMEM
+                    const int w0 = (ks % KPS) * C::WPS;
+                    const uint32_t sfa_s = smem_u32(sSFA + r * C::SFA_BYTES);
+                    const uint32_t sfb_s = smem_u32(sSFB + r * C::SFB_BYTES);
+#pragma unroll
+                    for (int c = 0; c < C::WPS; ++c) {
+                        utccp(col_sfa + 4 * c, desc_sf(sfa_s + (w0 + c) * 512));
+                        utccp(col_sfb + 8 * c, desc_sf(sfb_s + ((w0 + c) * 2 + 0) * 512));
+                        utccp(col_sfb + 8 * c + 4, desc_sf(sfb_s + ((w0 + c) * 2 + 1) * 512));
+                    }
+                    const int64_t krem = K - (int64_t)(kb + ks) * C::KE;
+                    const int nmma = krem >= C::KE ? 4 : (int)(krem / (C::KE / 4));
+                    const uint32_t a_s = smem_u32(sA + s * A_BYTES);
+                    const uint32_t b_s = smem_u32(sB + s * B_BYTES);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        if (j < nmma) {
+                            // scale word (4 TMEM columns) and byte of MMA j:
+                            // MX K = 64 takes 2 scales (bytes 0-1 / 2-3 of
+                            // word j / 2), NV K = 64 all 4 of word j, MXFP8
+                            // K = 32 byte j of the stage's one word
+                            const int c = (FMT == DS4G_MXFP4) ? (j >> 1) : (FMT == DS4G_NVFP4 ? j : 0);
+                            const uint32_t sfid = (FMT == DS4G_MXFP4) ? (uint32_t)((j & 1) * 2)
+                                                                     : (FMT == DS4G_NVFP4 ? 0u : (uint32_t)j);
+                            const uint32_t idesc = ibase | (sfid << 4) | (sfid << 29);
+                            mma<FMT>(acc, desc_sw128(a_s + 32 * j), desc_sw128(b_s + 32 * j), idesc,
+                                     (ks > 0 || j > 0) ? 1u : 0u, col_sfa + 4 * c, col_sfb + 8 * c);
+                        }
+                    }
+                    tc_commit(smem_u32(&empty[s]));
+                    if ((ks % KPS) == KPS - 1 || ks == nks - 1) tc_commit(smem_u32(&sf_empty[r]));
                 }
-                it_base += (uint32_t)(nks * gsz);
-                sit_base += (uint32_t)(nsfs * gsz);
+                if (!ok) break;
+                tc_commit(smem_u32(&tmem_full[buf]));
             }
+            // no tensor-core work of this thread may be in flight when the CTA
+            // releases its tensor memory (an early exit leaves some)
+            tc_commit(smem_u32(&drain[pi]));
+            volatile int never = 0;
+            mbar_wait(smem_u32(&drain[pi]), 0, &never);
         }
         __syncwarp();
     } else if (warp == 2) {
         // ================= scale transposer =================
-        uint32_t sit = 0;
-        for (int64_t t = tile0; t < ntiles; t += tstride) {
-            bool ok = true;
-            for (int pr = 0; pr < nsfs; ++pr, ++sit) {
-                const int r = sit % SF_STAGES;
-                bool w_ok = true;
-                if (lane == 0) w_ok = mbar_wait(smem_u32(&sf_full[r]), (sit / SF_STAGES) & 1, abort_flag);
-                if (!__shfl_sync(0xffffffffu, w_ok ? 1 : 0, 0)) { ok = false; break; }
-                sf_transpose<KPS * C::WPS, 1>(sSFA + r * C::SFA_BYTES, lane);
-                sf_transpose<KPS * C::WPS, 2>(sSFB + r * C::SFB_BYTES, lane);
-                fence_proxy_async();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(smem_u32(&sf_ready[r]));
+        // scale stages in the order the issuers take them: a group's members
+        // interleaved, scale stage by scale stage
+        uint32_t ls[NISS] = {};
+        bool ok = true;
+        for (int64_t j0 = 0; ok; j0 += NISS) {
+            const int64_t t0 = tile0 + j0 * tstride;
+            if (t0 >= ntiles) break;
+            const int gsz = (NISS == 2 && t0 + tstride < ntiles) ? 2 : 1;
+            for (int pr = 0; pr < nsfs && ok; ++pr) {
+#pragma unroll
+                for (int m = 0; m < NISS; ++m) {
+                    if (m >= gsz) break;
+                    const int r = NISS * (int)(ls[m] % SPM) + m;
+                    bool w_ok = true;
+                    if (lane == 0) w_ok = mbar_wait(smem_u32(&sf_full[r]), (ls[m] / SPM) & 1, abort_flag);
+                    if (!__shfl_sync(0xffffffffu, w_ok ? 1 : 0, 0)) { ok = false; break; }
+                    ++ls[m];
+                    sf_transpose<KPS * C::WPS, 1>(sSFA + r * C::SFA_BYTES, lane);
+                    sf_transpose<KPS * C::WPS, 2>(sSFB + r * C::SFB_BYTES, lane);
+                    fence_proxy_async();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(smem_u32(&sf_ready[r]));
+                }
             }
-            if (!ok) break;
         }
-    } else if (warp >= 4) {
+    } else if (warp >= 4 && warp < 4 + kEpiWarps) {
         // ================= epilogue =================
         const int q = warp & 3;                 // TMEM lane quarter this warp may access
         const int half = (warp - 4) >> 2;       // which half of the tile's columns
@@ -723,7 +753,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
             // epilogue) the output rows of this thread's four tile rows are
             // looked up before waiting for the accumulator, so that their
             // global loads overlap the tile's mainloop
-            const Tile tl = tile_of(t, prefix, soff, E, n_tiles, nb);
+            const Tile tl = tile_of(t / ksplit, prefix, soff, E, n_tiles, nb);
             const float gscale = (FMT == DS4G_NVFP4) ? __fmul_rn(p.a_g[0], p.w_g[tl.e]) : 1.0f;
             constexpr bool kDirect = (EPI != DS4G_EPI_SWIGLU_REQUANT) && !C::STAGED;
             float* dk[2][2];
@@ -794,7 +824,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
                                 if (d != 0ull && cc < ncol) {
                                     const float* sr = stg + rl * 33 + cc;
                                     float* g = reinterpret_cast<float*>(d) + col + cc;
-                                    if (EPI == kEpiCombine)
+                                    if (EPI == kEpiCombine || ksplit > 1)     // combine, or one K part of the sum
                                         red_add_v4(g, sr[0], sr[1], sr[2], sr[3]);
                                     else
                                         *reinterpret_cast<float4*>(g) = make_float4(sr[0], sr[1], sr[2], sr[3]);
@@ -829,7 +859,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
                                 const float a1 = __uint_as_float(r[g][2 * k + 1]) * w;
                                 const float b0 = __uint_as_float(r[g][4 + 2 * k]) * w;
                                 const float b1 = __uint_as_float(r[g][4 + 2 * k + 1]) * w;
-                                if (EPI == kEpiCombine) {
+                                if (EPI == kEpiCombine || ksplit > 1) {   // combine, or one K part of the sum
                                     red_add_v2(g0, a0, a1);
                                     red_add_v2(g0 + 8, b0, b1);
                                 } else {
@@ -1062,12 +1092,40 @@ static int combine_band_tiles(const GemmArgs& a, int tbn)
     return (int)(nb < n_tiles ? nb : n_tiles);
 }
 
+// Plain epilogue with few tiles (a dense GEMM of 64 rows: 16 tiles for 148
+// SMs): each tile's K range in ksplit equal parts of whole scale stages, the
+// largest divisor that keeps the tiles within about one per SM, each part
+// adding into the output (zeroed first).  The tile count is bounded from the
+// host's row bound (max_rows_per_expert).  1 = no split.
+static int plain_ksplit_tc(const GemmArgs& a, int tbn, int sms)
+{
+    if (a.epilogue != DS4G_EPI_NONE) return 1;
+    const int ke = fp8_act(a.fmt) ? 128 : 256, kps = fp8_act(a.fmt) ? 4 : 2;
+    const int nks = (int)ceil_div(a.K, ke);
+    if (nks % kps != 0) return 1;
+    const int64_t rows = a.max_rows > 0 ? a.max_rows : a.S;
+    const int64_t est = (a.E < a.S ? a.E : a.S) * ceil_div(rows, tc::BM) * ceil_div(a.N, tbn);
+    if (est * 2 > sms) return 1;
+    int best = 1;
+    for (int q = 2; q <= nks / kps; ++q)
+        if ((nks / kps) % q == 0 && est * q <= sms) best = q;
+    return best;
+}
+
 cudaError_t launch_gemm_tc(const GemmArgs& a_in, cudaStream_t st)
 {
     if (a_in.S == 0) return cudaSuccess;
     if (a_in.E > tc::kMaxE || !gemm_tc_supports(a_in.fmt, a_in.K)) return cudaErrorInvalidValue;
     GemmArgs a = a_in;
-    if (a.epilogue == kEpiCombine) a.band_tiles = combine_band_tiles(a, a.N % 224 == 0 ? 224 : 256);
+    const int tbn = a.N % 224 == 0 ? 224 : 256;
+    if (a.epilogue == kEpiCombine) a.band_tiles = combine_band_tiles(a, tbn);
+    int dev = 0, sms = kNumSMs;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    a.ksplit = plain_ksplit_tc(a, tbn, sms);
+    if (a.ksplit > 1) {
+        cudaError_t e = cudaMemsetAsync(a.out, 0, sizeof(float) * (size_t)a.S * a.N, st);
+        if (e != cudaSuccess) return e;
+    }
     if (a.fmt == DS4G_MXFP8)
         return a.epilogue == DS4G_EPI_NONE ? run_tc_plain<DS4G_MXFP8, DS4G_EPI_NONE>(a, st)
              : a.epilogue == kEpiCombine   ? run_tc_plain<DS4G_MXFP8, kEpiCombine>(a, st)

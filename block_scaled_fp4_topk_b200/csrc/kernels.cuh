@@ -24,6 +24,9 @@ cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, const uint8_
                            int32_t* slot_to_row, uint8_t* ad, uint8_t* as, float* ag, void* ws,
                            cudaStream_t st);
 
+cudaError_t launch_segment_ids(const int32_t* offsets, int nseg, int modulo, int64_t rows, int32_t* out,
+                               cudaStream_t st);
+
 struct GemmArgs {
     const uint8_t* a_data;
     const uint8_t* a_scales;
@@ -49,6 +52,7 @@ struct GemmArgs {
     int topk;
     int chained;             // decode kernel: launched to overlap the previous kernel on the stream
     int band_tiles;          // prefill kernel, combine epilogue: column tiles per band of the tile order (0: all)
+    int ksplit;              // plain epilogue with few tiles: equal K parts added into the zeroed output (0, 1: none)
 };
 
 cudaError_t launch_gemv(const GemmArgs& a, cudaStream_t st);
@@ -56,6 +60,8 @@ bool gemm_tc_supports(int fmt, int64_t K);
 cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st);
 bool gemv_tc_supports(int fmt, int64_t K, int N, int epilogue, int E);
 cudaError_t launch_gemv_tc(const GemmArgs& a, cudaStream_t st);
+bool ffn_dtc_supports(int fmt, int64_t d, int I, int E);
+cudaError_t launch_ffn_dtc(const GemmArgs& fc1, const GemmArgs& fc2, int32_t* ctr, cudaStream_t st);
 
 cudaError_t launch_swiglu_requant(const float* y1, int64_t rows, int I, int fmt, uint8_t* hd, uint8_t* hs,
                                   const float* hg, float* h_debug, cudaStream_t st);

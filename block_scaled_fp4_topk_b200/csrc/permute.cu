@@ -219,6 +219,30 @@ k_perm_small(const int32_t* __restrict__ idx, int S, int E, int k, int64_t rb, i
     }
 }
 
+// segment ids: row r of [0, rows) lies in segment s when offsets[s] - offsets[0]
+// <= r < offsets[s + 1] - offsets[0]; out[r] = s % modulo (binary search per row)
+__global__ void k_segment_ids(const int32_t* __restrict__ offsets, int nseg, int modulo, int64_t rows,
+                              int32_t* __restrict__ out)
+{
+    const int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (r >= rows) return;
+    const int64_t v = r + offsets[0];
+    int lo = 0, hi = nseg - 1;          // largest s with offsets[s] <= v
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (offsets[mid] <= v) lo = mid; else hi = mid - 1;
+    }
+    out[r] = lo % modulo;
+}
+
+cudaError_t launch_segment_ids(const int32_t* offsets, int nseg, int modulo, int64_t rows, int32_t* out,
+                               cudaStream_t st)
+{
+    if (rows == 0) return cudaSuccess;
+    k_segment_ids<<<(unsigned)ceil_div(rows, 256), 256, 0, st>>>(offsets, nseg, modulo, rows, out);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, const uint8_t* xd, const uint8_t* xs,
                            const float* xg, int64_t K, int fmt, int32_t* offsets, int32_t* row_to_slot,
                            int32_t* slot_to_row, uint8_t* ad, uint8_t* as, float* ag, void* ws_,

@@ -63,8 +63,10 @@ _SIGS = {
     "ds4g_swiglu_requant": ([_vp, _i64, _i32, _i32, _P, _vp, _vp], _i32),
     "ds4g_grouped_gemm_fp4_combine": ([_P, _vp, _i32, _i32, _P, _i32, _vp, _vp, _i32, _i32, _vp, _vp], _i32),
     "ds4g_moe_combine": ([_vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp], _i32),
+    "ds4g_segment_ids": ([_vp, _i32, _i32, _i64, _vp, _vp], _i32),
     "ds4g_grouped_gemm_fp4_combine_chained": ([_P, _vp, _i32, _i32, _P, _i32, _vp, _vp, _i32, _i32, _vp, _vp],
                                               _i32),
+    "ds4g_moe_ffn_fp4": ([_P, _vp, _i32, _i32, _P, _P, _i32, _i32, _P, _vp, _vp, _i32, _i32, _vp, _vp, _vp], _i32),
     "ds4g_zero_fill": ([_vp, _sz, _vp], _i32),
     "ds4g_permute_static_max_bytes": ([], _sz),
     "ds4g_moe_permute_static": ([_vp, _i32, _i32, _i32, _P, _vp, _vp, _vp, _P, _vp], _i32),
@@ -279,6 +281,32 @@ def ds4g_grouped_gemm_fp4_combine_chained(a, offsets, E, max_rows_per_expert, w,
     return out
 
 
+def ffn_supported(fmt, d, I, E):
+    """whether ds4g_moe_ffn_fp4 takes these shapes (the decode kernel's tiling
+    of both GEMMs, as include/ds4g.h states it)"""
+    kmul = 512 if fmt == MXFP4 else 256
+    return (fmt in (MXFP4, NVFP4) and 1 <= E <= 512 and d % kmul == 0 and I % kmul == 0 and I % 64 == 0
+            and d % 128 == 0)
+
+
+def ffn_counters(E, device="cuda"):
+    """the zeroed per-expert counters [E + 1] that ds4g_moe_ffn_fp4 needs"""
+    return torch.zeros(E + 1, dtype=torch.int32, device=device)
+
+
+def ds4g_moe_ffn_fp4(a, offsets, E, max_rows_per_expert, w1, w2, d, I, h_q, row_to_slot, route_w, out, counters):
+    """FC1 + SwiGLU/requantisation into h_q, then FC2 with the combine added
+    into out [T][d] (not zeroed), as one launch (decode sizes); counters:
+    int32 [E + 1], zero before the call and after it."""
+    T, k = route_w.shape
+    ac, w1c, w2c, hc = a.c(), w1.c(), w2.c(), h_q.c()
+    _check("ds4g_moe_ffn_fp4",
+           _lib.ds4g_moe_ffn_fp4(ctypes.byref(ac), offsets.data_ptr(), E, max_rows_per_expert, ctypes.byref(w1c),
+                                 ctypes.byref(w2c), d, I, ctypes.byref(hc), row_to_slot.data_ptr(),
+                                 route_w.data_ptr(), T, k, out.data_ptr(), counters.data_ptr(), _stream()))
+    return out
+
+
 def ds4g_zero_fill(t):
     """zero-fills a device tensor on the current stream"""
     _check("ds4g_zero_fill", _lib.ds4g_zero_fill(t.data_ptr(), t.numel() * t.element_size(), _stream()))
@@ -306,3 +334,12 @@ def ds4g_moe_combine(y2, slot_to_row, w, out=None):
     _check("ds4g_moe_combine", _lib.ds4g_moe_combine(y2.data_ptr(), slot_to_row.data_ptr(), w.data_ptr(), T, k, d,
                                                      out.data_ptr(), _stream()))
     return out
+
+
+def ds4g_segment_ids(offsets, nseg, modulo, rows, out=None):
+    """out[r] = (group of row offsets[0] + r) % modulo, int32 [rows]"""
+    if out is None:
+        out = torch.empty(max(rows, 1), dtype=torch.int32, device=offsets.device)
+    _check("ds4g_segment_ids", _lib.ds4g_segment_ids(offsets.data_ptr(), nseg, modulo, rows, out.data_ptr(),
+                                                     _stream()))
+    return out[:rows]

@@ -14,7 +14,7 @@ from .ds4g import EPI_NONE, EPI_SWIGLU_REQUANT, MXFP4, MXFP8, NVFP4, Fp4Tensor
 
 class MoeLayer:
     def __init__(self, w1, w2, E, k, d, I, fmt, g_h=None, fused=True, fused_combine=True, fused_dispatch=True,
-                 chained=True, act_fmt=None, shared=None):
+                 chained=True, act_fmt=None, shared=None, one_launch=False):
         """w1: Fp4Tensor [E*2I][d] (gate rows then up rows per expert),
         w2: Fp4Tensor [E*d][I]; NVFP4 weights carry one tensor scale per
         expert (w.g has E floats); g_h: the static NVFP4 tensor scale of h.
@@ -25,7 +25,10 @@ class MoeLayer:
         take the separate routing / quantisation / permutation calls).
         shared: (ws1 [2I_s][d], ws2 [d][I_s]) MXFP8 weights of a shared expert
         that every token also goes through (FP8 activations only); its output
-        is added to the routed experts' sum with weight 1."""
+        is added to the routed experts' sum with weight 1.
+        one_launch: at decode sizes (at most 16 tokens, shapes the decode
+        kernel tiles) FC1 + SwiGLU/requant and FC2 + combine run as one
+        launch (ds4g_moe_ffn_fp4); other sizes take the two calls."""
         self.w1, self.w2 = w1, w2
         self.E, self.k, self.d, self.I, self.fmt = E, k, d, I, fmt
         self.act_fmt = fmt if act_fmt is None else act_fmt
@@ -40,6 +43,7 @@ class MoeLayer:
                 raise ValueError("the shared expert takes MXFP8 weights and FP8 activations")
             self.I_s = shared[0].rows // 2
         self.chained = chained and fused_combine
+        self.one_launch = one_launch and self.fused and self.chained and self.act_fmt == fmt and fmt in (MXFP4, NVFP4)
         self.g_h = None
         if fmt == NVFP4:
             dev = w1.data.device
@@ -64,6 +68,7 @@ class MoeLayer:
                 pws=ds4g.permute_workspace(T, self.k, self.E, device),
                 dws=ds4g.dispatch_workspace(T, self.k, self.E, self.fmt, False, device),
                 qws=torch.empty(16, dtype=torch.uint8, device=device),
+                ctr=ds4g.ffn_counters(self.E, device),
             )
             if self.fmt == NVFP4:
                 b["hq"].g = self.g_h
@@ -79,14 +84,28 @@ class MoeLayer:
             self._bufs[key] = b
         return b
 
+    def uses_one_launch(self, T):
+        """whether the FFN of a T-token step runs as one launch"""
+        return self.one_launch and T <= 16 and ds4g.ffn_supported(self.fmt, self.d, self.I, self.E)
+
     def forward(self, x, logits, h_debug=None, out=None):
         """x: bf16 [T][d] (device), logits: fp32 [T][E] (device) -> fp32 [T][d]
         (written into `out` when given, else into the layer's own buffer)"""
         T = x.shape[0]
         b = self.buffers(T, x.device)
         self.dispatch(x, logits, b, out)
+        if h_debug is None and self.uses_one_launch(T):
+            return self.ffn(b, T, out)
         self.fc1(b, T, h_debug)
         return self.fc2(b, T, out)
+
+    def ffn(self, b, T, out=None):
+        """FC1 + SwiGLU/requant and FC2 + combine into out (zeroed before the
+        dispatch) as one launch"""
+        out = b["out"] if out is None else out
+        ds4g.ds4g_moe_ffn_fp4(b["a"], b["offsets"], self.E, T, self.w1, self.w2, self.d, self.I, b["hq"], b["r2s"],
+                              b["w"], out, b["ctr"])
+        return out
 
     def dispatch(self, x, logits, b, out=None):
         """routing, activation quantisation and the expert-contiguous
@@ -163,6 +182,14 @@ class MoeLayer:
         self._warm(x, logits)
         T = x.shape[0]
         b = self.buffers(T, x.device)
+        if self.uses_one_launch(T):
+            names = ["dispatch", "ffn"]
+            graphs = [torch.cuda.CUDAGraph() for _ in names]
+            with torch.cuda.graph(graphs[0]):
+                self.dispatch(x, logits, b)
+            with torch.cuda.graph(graphs[1]):
+                out = self.ffn(b, T)
+            return list(zip(names, graphs)), out
         names = ["dispatch", "fc1_swiglu", "fc2_combine"]
         graphs = [torch.cuda.CUDAGraph() for _ in names]
         with torch.cuda.graph(graphs[0]):

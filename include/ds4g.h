@@ -211,6 +211,12 @@ ds4g_status ds4g_moe_dispatch(const float* logits, const void* x, int dtype, int
  *   otherwise: a dp4a weight-streaming kernel (any segment length).
  *   FP8 activations always take the 128-row tensor-core kernel
  *   (kind::mxf8f6f4): K % 512 == 0 and the N rule above, else DS4G_ERR_SHAPE.
+ *   With NONE and few tiles for the SMs (a dense GEMM of a few rows, e.g.
+ *   M = 1 or 64 at N = 4096) both tensor-core kernels split each tile's K
+ *   range into equal parts that add their partial sums into out with fp32
+ *   atomics (out is zeroed first on the stream): the result may then differ
+ *   in its last bits from run to run.  Chosen from the shapes and
+ *   max_rows_per_expert alone.
  * Shapes: K % 64 == 0; NONE needs N % 64 == 0 unless a tensor-core kernel
  *   takes the call; SWIGLU_REQUANT needs I % 32 == 0.  offsets[E] must
  *   equal S. */
@@ -262,6 +268,48 @@ ds4g_status ds4g_grouped_gemm_fp4_combine_chained(const ds4g_fp4* a, const int32
                                                   int max_rows_per_expert, const ds4g_fp4* w, int N,
                                                   const int32_t* row_to_slot, const float* route_w, int T, int k,
                                                   float* out, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * The decode FFN in one launch ("[DeepSeek V4] Triton FP4 ...", "Why Triton
+ * is the only way on SM120": launch overhead at decode sizes; the fused
+ * SwiGLU + quantisation of "Moore Threads ..."): the work of
+ *   ds4g_grouped_gemm_fp4(a, offsets, E, max_rows_per_expert, w1, 2I,
+ *                         DS4G_EPI_SWIGLU_REQUANT, NULL, h_q, NULL) followed by
+ *   ds4g_grouped_gemm_fp4_combine_chained(h_q, offsets, E, max_rows_per_expert,
+ *                                         w2, d, row_to_slot, route_w, T, k, out)
+ * as one persistent kernel: each expert's FC2 tiles start as soon as all of
+ * that expert's FC1 tiles have stored their h rows (a per-expert completion
+ * counter; every wait on one is bounded), so FC2's weight streaming overlaps
+ * the end of FC1 with no launch between them.  a: [T*k] rows of d, fmt MXFP4
+ * or NVFP4; w1: E*2I rows of d and w2: E*d rows of I, same fmt; h_q: [T*k]
+ * rows of I (written; NVFP4: its g is the caller's static tensor scale of h,
+ * read); out: fp32 [T][d], added into (zero it before the call, as for the
+ * chained combine).  counters: int32 [E + 1] device memory owned by the
+ * caller, all zero on entry; the call leaves them zero (its last CTA resets
+ * them), also after a device-side wait gave up.  Calls that share a counter
+ * array must not overlap on the GPU.  Decode shapes only:
+ * max_rows_per_expert <= 16 and the decode kernel's tiling for both GEMMs
+ * (MXFP4: d and I multiples of 512, NVFP4: of 256; I % 64 == 0, d % 128 ==
+ * 0), E <= 512; otherwise DS4G_ERR_SHAPE.  Launched with programmatic stream
+ * serialization like the decode kernel; its CTAs wait on one another, and
+ * the grid is sized to be resident on the device at once (one CTA, or one
+ * CTA pair, per SM pair). */
+ds4g_status ds4g_moe_ffn_fp4(const ds4g_fp4* a, const int32_t* offsets, int E, int max_rows_per_expert,
+                             const ds4g_fp4* w1, const ds4g_fp4* w2, int d, int I, ds4g_fp4* h_q,
+                             const int32_t* row_to_slot, const float* route_w, int T, int k, float* out,
+                             int32_t* counters, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Segment ids, for expert parallelism across GPUs ("Moore Threads ..." MoE
+ * dispatch / combine; "DGX Spark native FP4 ..." sec. 6, several GPUs): a
+ * receiving rank holds rows grouped by source rank and, within a source, by
+ * its own expert; offsets [nseg + 1] (int32, device, non-decreasing) are
+ * those groups' boundaries.  Writes out[r] = s % modulo for every row r of
+ * [0, rows), s the group holding row offsets[0] + r (with modulo = experts
+ * per rank: the row's local expert).  rows must be offsets[nseg] -
+ * offsets[0]; rows beyond the last boundary get the last group. */
+ds4g_status ds4g_segment_ids(const int32_t* offsets, int nseg, int modulo, int64_t rows, int32_t* out,
+                             void* stream);
 
 /* Zero-fills bytes of device memory at p on the stream (cudaMemsetAsync). */
 ds4g_status ds4g_zero_fill(void* p, size_t bytes, void* stream);

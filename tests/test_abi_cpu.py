@@ -121,3 +121,29 @@ def test_empty_combine_is_a_no_op():
     from block_scaled_fp4_topk_b200 import ds4g
     # zero tokens: validated, nothing to launch
     assert ds4g._lib.ds4g_moe_combine(None, None, None, 0, 6, 7168, None, None) == 0
+
+
+def test_ffn_call_rejected_on_the_host():
+    import numpy as np
+    from block_scaled_fp4_topk_b200 import ds4g
+    L = ds4g._lib
+    buf = np.zeros(1 << 16, np.uint8)              # 64-byte aligned host buffer, never read
+    offs = np.zeros(5, np.int32)
+    op = offs.ctypes.data_as(ctypes.c_void_p)
+    out = buf.ctypes.data_as(ctypes.c_void_p)
+    E, d, I, T, k = 4, 512, 512, 4, 2
+    a, h = _fp4(T * k, d, buf=buf), _fp4(T * k, I, buf=buf)
+    w1, w2 = _fp4(E * 2 * I, d, buf=buf), _fp4(E * d, I, buf=buf)
+
+    def call(a=a, max_rows=4, w1=w1, w2=w2, d=d, I=I, h=h, T=T, k=k, ctr=out):
+        return L.ds4g_moe_ffn_fp4(ctypes.byref(a), op, E, max_rows, ctypes.byref(w1), ctypes.byref(w2), d, I,
+                                  ctypes.byref(h), op, out, T, k, out, ctr, None)
+    assert call(a=_fp4(T * k + 1, d, buf=buf)) == 2            # a must have T * k rows
+    assert call(max_rows=17) == 2                              # decode sizes only
+    assert call(a=_fp4(T * k, 96, buf=buf), d=96) == 2         # the decode kernel's K rule
+    assert call(w2=_fp4(E * d, 256, buf=buf)) == 2             # w2's K must be I
+    assert call(h=_fp4(T * k, 256, buf=buf)) == 2              # h_q rows of I
+    assert call(ctr=None) == 1                                 # the counters are required
+    assert call(k=0) == 1
+    a8 = _fp4(T * k, d, fmt=2, buf=buf)
+    assert call(a=a8) == 1                                     # FP4 activations only

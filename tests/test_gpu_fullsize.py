@@ -263,3 +263,47 @@ def test_decode_graph_replays_with_changing_routing(name, replays):
         ref, _, _ = _chain(wl, xq, idx, w, np.arange(wl.T))
         rel = _rel_l2(o.cpu().numpy().astype(np.float64), ref)
         assert rel <= L2_MAX, f"replay {r}: layer relative L2 {rel:.3e}"
+
+
+@pytest.mark.parametrize("name,replays", [("decode_t1", 3), ("decode_t4", 2), ("decode_t8", 2)])
+def test_decode_one_launch_ffn_replays(name, replays):
+    """The decode layer with FC1 -> FC2 + combine as one launch
+    (ds4g_moe_ffn_fp4), captured once and replayed with new activations and
+    routing before every replay: each replay's offsets bit-exact and its
+    output within relative L2 1e-2 of the oracle's chain; after the last one
+    the combine per element from the GPU's own h codes and routing weights,
+    and the per-expert counters back at zero"""
+    wl = workloads.WORKLOADS[name]
+    base = _layer(MX)
+    layer = MoeLayer(base.w1, base.w2, wl.E, wl.k, wl.d, wl.I, MX, g_h=workloads.G_H, one_launch=True)
+    assert layer.uses_one_launch(wl.T)
+    x = bf16_dev(workloads.host_x_bits(wl, 0))
+    lg = torch.from_numpy(workloads.host_logits(wl, 0)).to(dev())
+    graph, out = layer.capture(x, lg)
+    b = layer.buffers(wl.T, dev())
+    inputs, outs, offs = [], [], []
+    for r in range(1, replays + 1):
+        xb, lr = workloads.host_x_bits(wl, 10 + r), workloads.host_logits(wl, 10 + r)
+        inputs.append((xb, lr))
+        x.copy_(bf16_dev(xb))
+        lg.copy_(torch.from_numpy(lr).to(dev()))
+        graph.replay()
+        outs.append(out.clone())
+        offs.append(b["offsets"].clone())
+    torch.cuda.synchronize()
+    ds4g.ds4g_check_device()
+    assert not b["ctr"].any(), "counters not reset"
+    for r, ((xb, lr), o, of) in enumerate(zip(inputs, outs, offs)):
+        idx, w = oracle.route_topk(lr, wl.k)
+        offsets, r2s, s2r = oracle.moe_permute(idx, wl.E)
+        assert np.array_equal(of.cpu().numpy(), offsets), f"replay {r}: offsets"
+        xq = oracle.quantize(synth.bf16_bits_to_f32(xb), wl.fmt)
+        last = r == len(inputs) - 1
+        gpu = (from_dev(b["hq"]), s2r, b["w"].cpu().numpy()) if last else None
+        ref, up, bound = _chain(wl, xq, idx, w, np.arange(wl.T), gpu=gpu)
+        got = o.cpu().numpy().astype(np.float64)
+        rel = _rel_l2(got, ref)
+        assert rel <= L2_MAX, f"replay {r}: layer relative L2 {rel:.3e}"
+        if last:
+            err = np.abs(got - up)
+            assert np.all(err <= bound), f"combine: worst excess {(err - bound).max():.3e}"

@@ -264,14 +264,16 @@ def _ref_gemm(a, offsets, w, gw, N):
 # (K % 512 MX / % 256 NV), the dp4a kernel otherwise
 GEMV_CASES = [([3, 0, 1, 8, 5], 512, 7168), ([1, 1, 1, 1, 1, 1], 256, 2048), ([2, 0, 0, 7], 256, 256),
               ([8], 4096, 256), ([1], 128, 128), ([16, 9, 0, 13], 256, 1024), ([1, 2], 384, 1024),
-              ([1], 4096, 7168)]                      # the dense configuration at M = 1 (one expert)
+              ([1], 4096, 7168),                      # the dense configuration at M = 1 (one expert)
+              ([3], 2048, 4096)]                      # one expert, few tiles: K split over 8 parts
 # tensor-core kernel cases (MX needs K % 512, NV K % 256; others take the
 # GEMV kernel with long segments, which is covered as well)
 TC_CASES = [([300, 0, 1, 129, 77], 512, 512), ([256, 128], 256, 1024), ([9, 200, 0, 0, 1000], 256, 512),
             ([130], 512, 7168), ([17, 140], 256, 768), ([40, 12], 256, 384),
             # N a multiple of 224: 224-column tiles, two accumulators
             ([300, 0, 1, 129, 77], 448, 512), ([130, 20], 224, 2048), ([17, 600], 672, 1024),
-            ([64], 4096, 7168)]                       # the dense configuration at M = 64 (one expert)
+            ([64], 4096, 7168),                       # the dense configuration at M = 64 (one expert)
+            ([40], 2048, 4096)]                       # one expert, few tiles: K split over 8 parts
 
 
 @pytest.mark.parametrize("fmt", [MX, NV])
@@ -451,6 +453,69 @@ def test_fc2_combine_chained(fmt, T, k, E, d, I):
              1e-6 * (oracle.moe_combine(np.abs(y2), s2r, np.abs(w64)) + np.abs(base)) + 1e-7)
     got = out.cpu().numpy()
     assert np.all(np.abs(got - ref) <= bound), f"worst excess {(np.abs(got - ref) - bound).max():.3e}"
+
+
+def _decode_weights(E, touched, n_rows, K, fmt, stream):
+    """an expert weight tensor whose touched experts hold random weights (the
+    others zero: no row reads them)"""
+    blk = oracle.BLOCK[fmt]
+    data = np.zeros((E * n_rows, K // 2), np.uint8)
+    scales = np.zeros((E * n_rows, K // blk), np.uint8)
+    gw = [1.0] * E
+    for e in touched:
+        q = oracle.quantize(synth.normal_f32((n_rows, K), e, stream, 0.02), fmt)
+        data[e * n_rows:(e + 1) * n_rows], scales[e * n_rows:(e + 1) * n_rows] = q.data, q.scales
+        gw[e] = q.g if fmt == NV else 1.0
+    return oracle.Fp4(data, scales, 1.0, fmt), (gw if fmt == NV else None)
+
+
+# the one-launch decode FFN: FC1 split over CTA pairs (few items) or not,
+# and (NV) K stage counts that are odd in both GEMMs
+FFN_CASES = {MX: [(1, 6, 32, 2048, 1024), (3, 6, 64, 1024, 512), (8, 6, 64, 1024, 1024), (4, 2, 8, 512, 512)],
+             NV: [(1, 6, 32, 2048, 1024), (3, 6, 64, 1024, 512), (8, 6, 64, 1024, 1024), (4, 2, 8, 768, 256)]}
+
+
+@pytest.mark.parametrize("fmt,T,k,E,d,I", [(f,) + c for f in (MX, NV) for c in FFN_CASES[f]])
+def test_moe_ffn_one_launch(fmt, T, k, E, d, I):
+    """ds4g_moe_ffn_fp4 twice in a row on the same buffers and counters, with
+    new activations and routing the second time: each call's h codes are a
+    valid rounding of the oracle's h, and out = (what it held) + the oracle's
+    FC2 + combine of those h codes; the counters are zero after each call"""
+    routes = []
+    for call in range(2):
+        lg = synth.logits(T, E, 7 + call, 1.5)
+        idx, rw = oracle.route_topk(lg, k)
+        routes.append((rw, oracle.moe_permute(idx, E)))
+    touched = sorted({e for _, (offsets, _, _) in routes for e in range(E) if offsets[e + 1] > offsets[e]})
+    W1, g1 = _decode_weights(E, touched, 2 * I, d, fmt, 92)
+    W2, g2 = _decode_weights(E, touched, d, I, fmt, 93)
+    w1_d, w2_d = to_dev(W1, g_per_expert=g1), to_dev(W2, g_per_expert=g2)
+    S = T * k
+    hq = ds4g.Fp4Tensor.empty(S, I, fmt, dev())
+    if fmt == NV:
+        hq.g.fill_(G_H)
+    ctr = ds4g.ffn_counters(E, dev())
+    out = torch.empty((T, d), dtype=torch.float32, device=dev())
+    for call, (rw, (offsets, r2s, s2r)) in enumerate(routes):
+        a = oracle.quantize(_x_f32(S, d, 91 + call), fmt)
+        base = synth.normal_f32((T, d), call, 94, 1.0)
+        out.copy_(torch.from_numpy(base))
+        rw32 = rw.astype(np.float32)
+        ds4g.ds4g_moe_ffn_fp4(to_dev(a), torch.from_numpy(offsets).to(dev()), E, T, w1_d, w2_d, d, I, hq,
+                              torch.from_numpy(r2s).to(dev()), torch.from_numpy(rw32).to(dev()), out, ctr)
+        ds4g.ds4g_check_device()
+        assert not ctr.any(), f"call {call}: counters left {ctr.cpu().numpy()}"
+        hq_host = from_dev(hq)
+        y1, ab1 = _ref_gemm(a, offsets, W1, g1, 2 * I)
+        h_ref, dh = _h_bound(y1, ab1, I)
+        check_requant(hq_host, h_ref, dh, fmt, g=G_H)
+        y2, ab2 = _ref_gemm(hq_host, offsets, W2, g2, d)
+        w64 = rw32.astype(np.float64)
+        ref = base.astype(np.float64) + oracle.moe_combine(y2, s2r, w64)
+        bound = (oracle.moe_combine(1e-5 * ab2 + 1e-6, s2r, np.abs(w64)) +
+                 1e-6 * (oracle.moe_combine(np.abs(y2), s2r, np.abs(w64)) + np.abs(base)) + 1e-7)
+        got = out.cpu().numpy()
+        assert np.all(np.abs(got - ref) <= bound), f"call {call}: worst excess {(np.abs(got - ref) - bound).max():.3e}"
 
 
 # ---- combine -----------------------------------------------------------------------
