@@ -295,11 +295,9 @@ def tokens_per_s(T, steps, ms, world):
 
 
 TIMED_SECONDS = 1.0
-# decode sizes run the FFN (FC1 -> FC2 + combine) as one launch
-ONE_LAUNCH = True
 
 
-def calibrate_steps(step, st, world, device, lo=20, hi=4000):
+def calibrate_steps(step, st, world, device, lo=20, hi=20000):
     """number of steps that fill about TIMED_SECONDS, from a few timed steps
     after the warm-up (the slowest rank's estimate, so all ranks agree)"""
     import torch
@@ -329,8 +327,7 @@ def run_ours(args, rank, world, local_rank):
         return run_dense(args, rank, world, dev, wl)
     st = torch.cuda.current_stream()
     w1, w2 = synthetic_weights(wl.E, wl.d, wl.I, wl.fmt, device=dev)
-    layer = MoeLayer(w1, w2, wl.E, wl.k, wl.d, wl.I, wl.fmt, g_h=workloads.G_H, act_fmt=wl.afmt,
-                     one_launch=ONE_LAUNCH)
+    layer = MoeLayer(w1, w2, wl.E, wl.k, wl.d, wl.I, wl.fmt, g_h=workloads.G_H, act_fmt=wl.afmt)
     one = layer.uses_one_launch(wl.T)
     # inputs resident in HBM (bf16 activations, fp32 logits), each rank its own token shard
     x = torch.empty((wl.T, wl.d), dtype=torch.bfloat16, device=dev)
@@ -367,8 +364,7 @@ def run_ours(args, rank, world, local_rank):
     layers, graphs, gouts = [layer], [graph], [gout]
     for r in range(1, R):
         w1r, w2r = synthetic_weights(wl.E, wl.d, wl.I, wl.fmt, seed=r, device=dev)
-        layers.append(MoeLayer(w1r, w2r, wl.E, wl.k, wl.d, wl.I, wl.fmt, g_h=workloads.G_H, act_fmt=wl.afmt,
-                               one_launch=ONE_LAUNCH))
+        layers.append(MoeLayer(w1r, w2r, wl.E, wl.k, wl.d, wl.I, wl.fmt, g_h=workloads.G_H, act_fmt=wl.afmt))
         gr, go = layers[r].capture(x, lg)
         graphs.append(gr)
         gouts.append(go)

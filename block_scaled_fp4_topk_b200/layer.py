@@ -14,7 +14,7 @@ from .ds4g import EPI_NONE, EPI_SWIGLU_REQUANT, MXFP4, MXFP8, NVFP4, Fp4Tensor
 
 class MoeLayer:
     def __init__(self, w1, w2, E, k, d, I, fmt, g_h=None, fused=True, fused_combine=True, fused_dispatch=True,
-                 chained=True, act_fmt=None, shared=None, one_launch=False):
+                 chained=True, act_fmt=None, shared=None, one_launch=True):
         """w1: Fp4Tensor [E*2I][d] (gate rows then up rows per expert),
         w2: Fp4Tensor [E*d][I]; NVFP4 weights carry one tensor scale per
         expert (w.g has E floats); g_h: the static NVFP4 tensor scale of h.
@@ -28,7 +28,8 @@ class MoeLayer:
         is added to the routed experts' sum with weight 1.
         one_launch: at decode sizes (at most 16 tokens, shapes the decode
         kernel tiles) FC1 + SwiGLU/requant and FC2 + combine run as one
-        launch (ds4g_moe_ffn_fp4); other sizes take the two calls."""
+        launch (ds4g_moe_ffn_fp4); other sizes, and one_launch=False, take
+        the two calls (FC2 chained to FC1)."""
         self.w1, self.w2 = w1, w2
         self.E, self.k, self.d, self.I, self.fmt = E, k, d, I, fmt
         self.act_fmt = fmt if act_fmt is None else act_fmt

@@ -19,11 +19,12 @@ seeded inputs:
   - the whole layer on the same token sample against the oracle's own chain
     (routing, quantisation, FC1, SwiGLU, requantisation, FC2, combine):
     relative L2 <= 1e-2.
-And the captured decode layer (split FC1 at T = 1, plain at T = 4) replayed
-back to back with different inputs and routing on every replay, each replay
-against the oracle's chain (offsets bit-exact, output relative L2 <= 1e-2):
-routing-dependent ordering errors between the layer's kernels only show when
-the routing changes between steps."""
+And the captured decode layer (split FC1 at T = 1, plain at T = 4; as two
+calls, and at T = 1 / 4 / 8 with FC1 -> FC2 + combine as one launch)
+replayed back to back with different inputs and routing on every replay,
+each replay against the oracle's chain (offsets bit-exact, output relative
+L2 <= 1e-2): routing-dependent ordering errors between the layer's kernels
+only show when the routing changes between steps."""
 import numpy as np
 import pytest
 import torch
@@ -120,7 +121,9 @@ def _run(name):
     xb = workloads.host_x_bits(wl)
     lg = workloads.host_logits(wl)
     hdbg = torch.empty((wl.S, wl.I), dtype=torch.float32, device=dev())
-    out = layer.forward(bf16_dev(xb), torch.from_numpy(lg).to(dev()), h_debug=hdbg)   # as the bench runs it
+    # the two-call FFN (h_debug asks for FC1's h; the bench's decode steps run
+    # the one-launch FFN, checked in test_decode_one_launch_ffn_replays)
+    out = layer.forward(bf16_dev(xb), torch.from_numpy(lg).to(dev()), h_debug=hdbg)
     ds4g.ds4g_check_device()
     b = dict(layer.buffers(wl.T, dev()))
     # FC2 rows as well (the layer fuses FC2 with the combine): the plain epilogue
@@ -229,13 +232,14 @@ def test_fullsize_layer(name):
 
 @pytest.mark.parametrize("name,replays", [("decode_t1", 4), ("decode_t4", 3)])
 def test_decode_graph_replays_with_changing_routing(name, replays):
-    """The decode layer captured once (MoeLayer.capture, FC2 chained to FC1;
-    FC1 split over CTA pairs at T = 1) and replayed back to back with new
+    """The decode layer captured once as two calls (MoeLayer.capture with
+    one_launch=False: FC2 chained to FC1; FC1 split over CTA pairs at T = 1) and replayed back to back with new
     activations and router logits before every replay, no host sync in
     between; each replay's offsets bit-exact and its output within relative
     L2 1e-2 of the oracle's chain on that replay's inputs"""
     wl = workloads.WORKLOADS[name]
-    layer = _layer(MX)
+    base = _layer(MX)
+    layer = MoeLayer(base.w1, base.w2, wl.E, wl.k, wl.d, wl.I, MX, g_h=workloads.G_H, one_launch=False)
     x = bf16_dev(workloads.host_x_bits(wl, 0))
     lg = torch.from_numpy(workloads.host_logits(wl, 0)).to(dev())
     graph, out = layer.capture(x, lg)
