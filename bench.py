@@ -35,7 +35,11 @@ L2_BYTES = 126 * 1000 * 1000
 # 969.7 MB algorithmic, 1.025x) scaled to the full launch by its algorithmic bytes
 # (3350.2 MB); workloads without a capture of the current kernel report null
 FC1_TRAFFIC = {"prefill16k": (3424476035, "profiles/k_gemm_tc_fc1_prof_prefill16k_nvfp4.md (stand-in, scaled)"),
-               "prefill": (2332878592, "profiles/dram_traffic_k_gemm_tc_prefill_T2048_mxfp4.md (full-size launch)")}
+               "prefill": (2332878592, "profiles/dram_traffic_k_gemm_tc_prefill_T2048_mxfp4.md (full-size launch)"),
+               # the one-launch decode FFN: the decode stand-in's traffic ratio (1.00882) x the algorithmic bytes
+               "decode_t8": (1039043879, "profiles/k_gemv_tc_ffn_prof_decode_t8_mxfp4.md (stand-in ratio, scaled)"),
+               "decode_t4": (566727518, "profiles/k_gemv_tc_ffn_prof_decode_t8_mxfp4.md (stand-in ratio, scaled)"),
+               "decode_t1": (141681879, "profiles/k_gemv_tc_ffn_prof_decode_t8_mxfp4.md (stand-in ratio, scaled)")}
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)

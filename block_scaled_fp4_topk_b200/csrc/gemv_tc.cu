@@ -12,7 +12,7 @@
 // Roles (one persistent CTA per SM, 288 threads):
 //   warps 0, 8  TMA producers, alternate scale stages: weight tile (128 rows
 //           x 256 K) and the expert's activation rows (16 rows x 256 K), 10
-//           stages; row-major scale boxes of both (512 K per scale stage, 5
+//           stages; row-major scale boxes of both (512 K per scale stage, 6
 //           scale stages for MXFP4, 4 for NVFP4)
 //   warps 1, 3  MMA issuers, alternate scale stages: scales -> TMEM
 //           (tcgen05.cp), 4 MMAs per data stage, double-buffered 16-column

@@ -18,8 +18,10 @@ adaptation of DeepSeek-V4": MoE dispatch / combine across devices;
      splits reversed), which combine them with their routing weights.
 
 The data plane is NCCL; the row counts travel to the host once per step
-(the splits of the exchanges).  MXFP4 weights and activations (the format the
-pages' routed experts are released in).
+(the splits of the exchanges).  MXFP4 or NVFP4 weights and activations.  With
+NVFP4 every rank quantises its activations with one shared tensor scale, the
+largest of the ranks' own (an all-reduce of one float before the dispatch),
+so that an expert's rows from all ranks share their scale, as its GEMMs need.
 
 The host-side pieces (the plan of the exchanges and the exchange itself) are
 plain functions so that multi-rank tests can run them on CPU tensors.
@@ -29,7 +31,7 @@ import torch
 import torch.distributed as dist
 
 from . import ds4g
-from .ds4g import EPI_NONE, EPI_SWIGLU_REQUANT, MXFP4, Fp4Tensor
+from .ds4g import EPI_NONE, EPI_SWIGLU_REQUANT, MXFP4, NVFP4, Fp4Tensor
 
 
 def experts_per_rank(E, G):
@@ -61,6 +63,13 @@ def recv_layout(recv_expert_counts, G):
     return per_source, bounds
 
 
+def shared_tensor_scale(g_local, group=None):
+    """the NVFP4 activation tensor scale every rank quantises with: the
+    largest of the ranks' own (fp32 [1], in place)"""
+    dist.all_reduce(g_local, op=dist.ReduceOp.MAX, group=group)
+    return g_local
+
+
 def exchange(send, send_splits, recv_splits, group=None):
     """all_to_all of the rows of `send` (first dimension split by
     send_splits, one part per rank) into a new tensor of sum(recv_splits)
@@ -73,26 +82,36 @@ def exchange(send, send_splits, recv_splits, group=None):
 
 class EpMoeLayer:
     """One MoE layer with its experts split over the ranks of `group`
-    (NCCL).  w1_local [El*2I][d], w2_local [El*d][I]: MXFP4 weights of this
-    rank's experts, El = E / world_size."""
+    (NCCL).  w1_local [El*2I][d], w2_local [El*d][I]: MXFP4 or NVFP4 weights
+    of this rank's experts, El = E / world_size (NVFP4: w.g holds the El
+    experts' tensor scales); g_h: the static NVFP4 tensor scale of h."""
 
-    def __init__(self, w1_local, w2_local, E, k, d, I, group=None):
+    def __init__(self, w1_local, w2_local, E, k, d, I, group=None, g_h=1.0):
         self.group = group
         self.G = dist.get_world_size(group)
         self.rank = dist.get_rank(group)
         self.El = experts_per_rank(E, self.G)
         self.w1, self.w2 = w1_local, w2_local
         self.E, self.k, self.d, self.I = E, k, d, I
-        if w1_local.fmt != MXFP4 or w2_local.fmt != MXFP4:
-            raise ValueError("expert parallelism takes MXFP4 weights")
+        self.fmt = w1_local.fmt
+        if self.fmt not in (MXFP4, NVFP4) or w2_local.fmt != self.fmt:
+            raise ValueError("expert parallelism takes MXFP4 or NVFP4 weights, both GEMMs the same")
+        self.g_h = None
+        if self.fmt == NVFP4:
+            self.g_h = torch.tensor([g_h], dtype=torch.float32, device=w1_local.data.device)
 
     def forward(self, x, logits):
         """x bf16 [T][d], logits fp32 [T][E] (this rank's tokens, device) ->
         fp32 [T][d]"""
         dev = x.device
         T = x.shape[0]
-        G, El = self.G, self.El
-        idx, w, xq, offsets, r2s, s2r, a = ds4g.ds4g_moe_dispatch(logits, x, self.k, MXFP4)
+        G, El, fmt = self.G, self.El, self.fmt
+        g = None
+        if fmt == NVFP4:
+            # one activation tensor scale for all ranks (this rank's own from
+            # a quantisation pass, then the largest over the ranks)
+            g = shared_tensor_scale(ds4g.ds4g_quantize_mx(x, NVFP4).g.clone(), self.group)
+        idx, w, xq, offsets, r2s, s2r, a = ds4g.ds4g_moe_dispatch(logits, x, self.k, fmt, g_in=g)
         S = T * self.k
         offs_h = offsets.cpu().numpy()
         sc = send_counts(offs_h, G)
@@ -103,12 +122,14 @@ class EpMoeLayer:
         # the quantised rows (codes and scales) to their experts' ranks
         rd = exchange(a.data[:S], sc, rc, self.group)
         rs = exchange(a.scales[:S], sc, rc, self.group)
-        recv = Fp4Tensor(rd, rs, None, MXFP4)
+        recv = Fp4Tensor(rd, rs, g, fmt)
         # each received row's local expert, then the expert-contiguous order
         bnd = torch.from_numpy(bounds.astype(np.int32)).to(dev)
         ids = ds4g.ds4g_segment_ids(bnd, G * El, El, R)
         offs_l, r2s_l, s2r_l, a_l = ds4g.ds4g_moe_permute(ids.view(R, 1), El, recv)
-        hq = Fp4Tensor.empty(R, self.I, MXFP4, dev)
+        hq = Fp4Tensor.empty(R, self.I, fmt, dev)
+        if fmt == NVFP4:
+            hq.g = self.g_h
         ds4g.ds4g_grouped_gemm_fp4(a_l, offs_l, El, R, self.w1, 2 * self.I, EPI_SWIGLU_REQUANT, out_q=hq)
         y2 = ds4g.ds4g_grouped_gemm_fp4(hq, offs_l, El, R, self.w2, self.d, EPI_NONE)
         # FC2 rows back in received order, then to their source ranks

@@ -74,6 +74,9 @@ WORKLOADS = {
     # 4096 tokens, i.e. the same 384 rows per expert on average
     "prof_prefill16k": Workload("prof_prefill16k", T=4096, E=64, k=6, d=7168, I=2048, fmt=NV,
                                 bias_sigma=BIAS_SIGMA),
+    # profiling stand-in for "decode_t8": 64 experts (1.5 GB of weights per
+    # layer) and the same 48 routed slots
+    "prof_decode_t8": Workload("prof_decode_t8", T=8, E=64, k=6, d=7168, I=2048, fmt=MX, bias_sigma=0.0),
 }
 
 

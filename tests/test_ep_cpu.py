@@ -1,14 +1,17 @@
 """Expert parallelism's host side on CPU: two gloo ranks, each with its own
 tokens and half of the experts, run the plan and the exchanges of
-block_scaled_fp4_topk_b200.ep (row counts, quantised rows, FC2 rows back)
-with the oracle doing each step's arithmetic in place of the library's
-kernels.  Every rank's output must equal the single-rank oracle layer on its
-own tokens bit for bit: the exchange only moves rows, and every row meets the
-same arithmetic.  Also: the plan's arithmetic on hand-written counts."""
+block_scaled_fp4_topk_b200.ep (row counts, quantised rows, FC2 rows back;
+for NVFP4 also the shared activation tensor scale) with the oracle doing each
+step's arithmetic in place of the library's kernels.  Every rank's output
+must equal the single-rank oracle layer on its own tokens (quantised with the
+same tensor scale) bit for bit: the exchange only moves rows, and every row
+meets the same arithmetic.  Also: the plan's arithmetic on hand-written
+counts."""
 import os
 import socket
 
 import numpy as np
+import pytest
 import torch.multiprocessing as mp
 
 E, K_TOP, D, I, T = 8, 2, 256, 128, 24
@@ -22,11 +25,18 @@ def _free_port():
     return p
 
 
-def _weights(e):
+def _weights(e, fmt):
     import oracle
     from synth import workloads
-    wl = workloads.Workload("ep_cpu", T=T, E=E, k=K_TOP, d=D, I=I, fmt=oracle.MX, bias_sigma=1.5)
-    return (oracle.quantize(workloads.host_w1(wl, e), oracle.MX), oracle.quantize(workloads.host_w2(wl, e), oracle.MX))
+    wl = workloads.Workload("ep_cpu", T=T, E=E, k=K_TOP, d=D, I=I, fmt=fmt, bias_sigma=1.5)
+    return oracle.quantize(workloads.host_w1(wl, e), fmt), oracle.quantize(workloads.host_w2(wl, e), fmt)
+
+
+def _h_q(y1, fmt):
+    """h = SwiGLU(y1) requantised (NVFP4: with the static tensor scale of h)"""
+    import oracle
+    from synth import workloads
+    return oracle.quantize(oracle.swiglu(y1.astype(np.float32)), fmt, g=workloads.G_H if fmt == oracle.NV else None)
 
 
 def _tokens(rank):
@@ -36,40 +46,40 @@ def _tokens(rank):
     return synth.bf16_bits_to_f32(workloads.host_x_bits(wl, rank)), workloads.host_logits(wl, rank)
 
 
-def _expert_rows(a, rows, e, which):
+def _expert_rows(a, rows, e, which, fmt):
     import oracle
-    W1, W2 = _weights(e)
+    W1, W2 = _weights(e, fmt)
     if which == 1:
         return oracle.expert_gemm_rows(a, rows, W1, (0, 2 * I))[0]
     return oracle.expert_gemm_rows(a, rows, W2, (0, D))[0]
 
 
-def _local_layer(x, lg):
-    """the single-rank oracle layer on these tokens, all experts"""
+def _local_layer(x, lg, fmt, g):
+    """the single-rank oracle layer on these tokens, all experts (NVFP4: the
+    activations quantised with tensor scale g)"""
     import oracle
     idx, w = oracle.route_topk(lg, K_TOP)
-    xq = oracle.quantize(x, oracle.MX)
+    xq = oracle.quantize(x, fmt, g=g)
     offsets, r2s, s2r = oracle.moe_permute(idx, E)
     a = oracle.gather_rows(xq, r2s, K_TOP)
     y2 = np.zeros((a.data.shape[0], D))
     for e in range(E):
         rows = np.arange(offsets[e], offsets[e + 1])
         if len(rows):
-            y1 = _expert_rows(a, rows, e, 1)
-            hq = oracle.quantize(oracle.swiglu(y1.astype(np.float32)), oracle.MX)
-            y2[rows] = _expert_rows(hq, np.arange(len(rows)), e, 2)
+            y1 = _expert_rows(a, rows, e, 1, fmt)
+            y2[rows] = _expert_rows(_h_q(y1, fmt), np.arange(len(rows)), e, 2, fmt)
     return oracle.moe_combine(y2, s2r, w)
 
 
-def _rank(rank, world, port, q):
+def _rank(rank, world, port, q, fmt):
     try:
-        _rank_body(rank, world, port, q)
+        _rank_body(rank, world, port, q, fmt)
     except BaseException as exc:          # report at once instead of leaving the parent waiting
         q.put((rank, False, float("nan"), repr(exc), None))
         raise
 
 
-def _rank_body(rank, world, port, q):
+def _rank_body(rank, world, port, q, fmt):
     import torch
     import torch.distributed as dist
     import oracle
@@ -78,9 +88,14 @@ def _rank_body(rank, world, port, q):
     dist.init_process_group("gloo", rank=rank, world_size=world)
     G, El = world, ep.experts_per_rank(E, world)
     x, lg = _tokens(rank)
+    # NVFP4: one activation tensor scale for all ranks, the largest of theirs
+    g = None
+    if fmt == oracle.NV:
+        g_local = torch.tensor([oracle.quantize(x, oracle.NV).g], dtype=torch.float32)
+        g = float(ep.shared_tensor_scale(g_local).item())
     # dispatch on this rank's tokens, all E experts
     idx, w = oracle.route_topk(lg, K_TOP)
-    xq = oracle.quantize(x, oracle.MX)
+    xq = oracle.quantize(x, fmt, g=g)
     offsets, r2s, s2r = oracle.moe_permute(idx, E)
     a = oracle.gather_rows(xq, r2s, K_TOP)
     # the plan and the exchanges of the library's expert-parallel layer
@@ -94,29 +109,29 @@ def _rank_body(rank, world, port, q):
     # order, FC1, SwiGLU, requantisation, FC2, rows back in received order
     ids = np.repeat(np.arange(G * El) % El, np.diff(bounds)).astype(np.int32)
     offs_l, r2s_l, s2r_l = oracle.moe_permute(ids.reshape(R, 1), El)
-    a_l = oracle.gather_rows(oracle.Fp4(rd, rs, 1.0, oracle.MX), r2s_l, 1)
+    a_l = oracle.gather_rows(oracle.Fp4(rd, rs, 1.0 if g is None else g, fmt), r2s_l, 1)
     y2_l = np.zeros((R, D))
     for le in range(El):
         rows = np.arange(offs_l[le], offs_l[le + 1])
         if len(rows):
             e = rank * El + le
-            y1 = _expert_rows(a_l, rows, e, 1)
-            hq = oracle.quantize(oracle.swiglu(y1.astype(np.float32)), oracle.MX)
-            y2_l[rows] = _expert_rows(hq, np.arange(len(rows)), e, 2)
+            y1 = _expert_rows(a_l, rows, e, 1, fmt)
+            y2_l[rows] = _expert_rows(_h_q(y1, fmt), np.arange(len(rows)), e, 2, fmt)
     y2_recv = y2_l[s2r_l]
     y2_back = ep.exchange(torch.from_numpy(y2_recv), rc, sc).numpy()
     out = oracle.moe_combine(y2_back, s2r, w)
-    ref = _local_layer(x, lg)
+    ref = _local_layer(x, lg, fmt, g)
     q.put((rank, bool(np.array_equal(out, ref)), float(np.abs(out - ref).max()), sc, rc))
     dist.barrier()
     dist.destroy_process_group()
 
 
-def test_two_rank_expert_parallel_exchange_matches_local_layer():
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_two_rank_expert_parallel_exchange_matches_local_layer(fmt):
     world, port = 2, _free_port()
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
-    procs = [ctx.Process(target=_rank, args=(r, world, port, q)) for r in range(world)]
+    procs = [ctx.Process(target=_rank, args=(r, world, port, q, fmt)) for r in range(world)]
     for p in procs:
         p.start()
     res = sorted((q.get(timeout=300) for _ in range(world)), key=lambda r: r[0])
