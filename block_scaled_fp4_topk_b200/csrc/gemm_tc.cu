@@ -628,11 +628,14 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
                 // let this member's copies in flight land before the CTA goes
                 // away: its latest uses of each slot (earlier ones completed
                 // before their slot was refilled)
-                volatile int never = 0;
-                for (uint32_t l = (ld > (uint32_t)DPM ? ld - DPM : 0u); l < ld; ++l)
+                for (uint32_t l = (ld > (uint32_t)DPM ? ld - DPM : 0u); l < ld; ++l) {
+                    volatile int never = 0;
                     mbar_wait(smem_u32(&full[NISS * (int)(l % DPM) + pp]), (l / DPM) & 1, &never);
-                for (uint32_t l = (ls > (uint32_t)SPM ? ls - SPM : 0u); l < ls; ++l)
+                }
+                for (uint32_t l = (ls > (uint32_t)SPM ? ls - SPM : 0u); l < ls; ++l) {
+                    volatile int never = 0;
                     mbar_wait(smem_u32(&sf_full[NISS * (int)(l % SPM) + pp]), (l / SPM) & 1, &never);
+                }
             }
         }
         __syncwarp();

@@ -502,14 +502,17 @@ k_gemv_tc(const __grid_constant__ Maps m0, const __grid_constant__ Maps m1, cons
             if (!waited) release_deferred();
             if (!ok) {
                 // let this thread's copies in flight land before the CTA goes
-                // away (stop at the first wait that gives up)
-                volatile int never = 0;
-                bool go = true;
-                for (uint32_t j = (it_next > STAGES + 2 ? it_next - STAGES - 2 : 0); j < it_next && go; ++j) {
-                    if ((int)((j >> 1) & 1) == pi) go = mbar_wait(smem_u32(&full[j % STAGES]), (j / STAGES) & 1, &never);
+                // away: its stages among the last ring's worth.  Each wait has
+                // its own bound; one that runs out means the slot has moved
+                // on, i.e. that stage landed and was consumed long ago.
+                for (uint32_t j = (it_next > STAGES ? it_next - STAGES : 0); j < it_next; ++j) {
+                    volatile int never = 0;
+                    if ((int)((j >> 1) & 1) == pi) mbar_wait(smem_u32(&full[j % STAGES]), (j / STAGES) & 1, &never);
                 }
-                for (uint32_t j = (sit_next > SF_STAGES + 1 ? sit_next - SF_STAGES - 1 : 0); j < sit_next && go; ++j)
-                    if ((int)(j & 1) == pi) go = mbar_wait(smem_u32(&sf_full[j % SF_STAGES]), (j / SF_STAGES) & 1, &never);
+                for (uint32_t j = (sit_next > SF_STAGES ? sit_next - SF_STAGES : 0); j < sit_next; ++j) {
+                    volatile int never = 0;
+                    if ((int)(j & 1) == pi) mbar_wait(smem_u32(&sf_full[j % SF_STAGES]), (j / SF_STAGES) & 1, &never);
+                }
             }
         }
         __syncwarp();

@@ -518,6 +518,51 @@ def test_moe_ffn_one_launch(fmt, T, k, E, d, I):
         assert np.all(np.abs(got - ref) <= bound), f"call {call}: worst excess {(np.abs(got - ref) - bound).max():.3e}"
 
 
+def test_moe_ffn_wait_gives_up_cleanly():
+    """A device-side bounded wait that runs out, made on purpose without any
+    fault: the per-expert counters start far below zero, so no FC2 item's
+    wait for its expert's FC1 items can succeed.  Every CTA gives up after
+    its bound, the call reports DS4G_ERR_DEVICE through ds4g_check_device,
+    the last CTA leaves the counters at zero, and the next call on the same
+    context and buffers is correct."""
+    fmt, T, k, E, d, I = MX, 4, 2, 8, 512, 512
+    lg = synth.logits(T, E, 3, 1.5)
+    idx, rw = oracle.route_topk(lg, k)
+    offsets, r2s, s2r = oracle.moe_permute(idx, E)
+    touched = [e for e in range(E) if offsets[e + 1] > offsets[e]]
+    W1, g1 = _decode_weights(E, touched, 2 * I, d, fmt, 95)
+    W2, g2 = _decode_weights(E, touched, d, I, fmt, 96)
+    S = T * k
+    a = oracle.quantize(_x_f32(S, d, 97), fmt)
+    args = (to_dev(a), torch.from_numpy(offsets).to(dev()), E, T, to_dev(W1, g_per_expert=g1),
+            to_dev(W2, g_per_expert=g2), d, I)
+    hq = ds4g.Fp4Tensor.empty(S, I, fmt, dev())
+    r2s_d, rw_d = torch.from_numpy(r2s).to(dev()), torch.from_numpy(rw.astype(np.float32)).to(dev())
+    out = torch.zeros((T, d), dtype=torch.float32, device=dev())
+    ctr = ds4g.ffn_counters(E, dev())
+    ctr[:E] = -(1 << 20)                               # a completion count no FC1 item can bring to its target
+    ds4g.ds4g_moe_ffn_fp4(*args, hq, r2s_d, rw_d, out, ctr)
+    torch.cuda.synchronize()
+    with pytest.raises(ds4g.Ds4gError) as ei:
+        ds4g.ds4g_check_device()
+    assert ei.value.status == 5                        # DS4G_ERR_DEVICE
+    assert not ctr.any(), "the counters are left at zero after a wait gave up"
+    ds4g.ds4g_check_device()                           # the error word was read and cleared
+    out.zero_()
+    ds4g.ds4g_moe_ffn_fp4(*args, hq, r2s_d, rw_d, out, ctr)
+    ds4g.ds4g_check_device()
+    y1, ab1 = _ref_gemm(a, offsets, W1, g1, 2 * I)
+    h_ref, dh = _h_bound(y1, ab1, I)
+    hq_host = from_dev(hq)
+    check_requant(hq_host, h_ref, dh, fmt)
+    y2, ab2 = _ref_gemm(hq_host, offsets, W2, g2, d)
+    w64 = rw.astype(np.float32).astype(np.float64)
+    ref = oracle.moe_combine(y2, s2r, w64)
+    bound = (oracle.moe_combine(1e-5 * ab2 + 1e-6, s2r, np.abs(w64)) +
+             1e-6 * oracle.moe_combine(np.abs(y2), s2r, np.abs(w64)) + 1e-7)
+    assert np.all(np.abs(out.cpu().numpy() - ref) <= bound)
+
+
 # ---- combine -----------------------------------------------------------------------
 
 def test_combine():
