@@ -292,8 +292,7 @@ ds4g_status ds4g_grouped_gemm_fp4_combine_chained(const ds4g_fp4* a, const int32
  * (MXFP4: d and I multiples of 512, NVFP4: of 256; I % 64 == 0, d % 128 ==
  * 0), E <= 512; otherwise DS4G_ERR_SHAPE.  Launched with programmatic stream
  * serialization like the decode kernel; its CTAs wait on one another, and
- * the grid is sized to be resident on the device at once (one CTA, or one
- * CTA pair, per SM pair). */
+ * the grid is sized to be resident on the device at once (one CTA per SM). */
 ds4g_status ds4g_moe_ffn_fp4(const ds4g_fp4* a, const int32_t* offsets, int E, int max_rows_per_expert,
                              const ds4g_fp4* w1, const ds4g_fp4* w2, int d, int I, ds4g_fp4* h_q,
                              const int32_t* row_to_slot, const float* route_w, int T, int k, float* out,

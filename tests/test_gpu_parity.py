@@ -469,8 +469,8 @@ def _decode_weights(E, touched, n_rows, K, fmt, stream):
     return oracle.Fp4(data, scales, 1.0, fmt), (gw if fmt == NV else None)
 
 
-# the one-launch decode FFN: FC1 split over CTA pairs (few items) or not,
-# and (NV) K stage counts that are odd in both GEMMs
+# the one-launch decode FFN (one CTA per SM): few items (fewer FC1 items
+# than SMs) and many, and (NV) K stage counts that are odd in both GEMMs
 FFN_CASES = {MX: [(1, 6, 32, 2048, 1024), (3, 6, 64, 1024, 512), (8, 6, 64, 1024, 1024), (4, 2, 8, 512, 512)],
              NV: [(1, 6, 32, 2048, 1024), (3, 6, 64, 1024, 512), (8, 6, 64, 1024, 1024), (4, 2, 8, 768, 256)]}
 
