@@ -13,7 +13,8 @@
 // 0") run the same kernel with kind::mxf8f6f4, against MXFP4 weights (loaded
 // unpacked, one byte per element) or MXFP8 weights (a shared expert's).
 //
-// Design (one persistent CTA per SM, 384 threads, warp-specialised):
+// Design (one persistent CTA per SM, 384 threads, 448 with two MMA issuers,
+// warp-specialised):
 //   warp 0   TMA producer: tiles of A (128 rows x 128 bytes of K) and W
 //            (up to 256 rows x 128 bytes) into 128B-swizzled shared memory
 //            (4 stages), and the row-major scale bytes of two (FP4) or four
@@ -24,6 +25,7 @@
 //            accumulator
 //   warp 2   scale transposer: rewrites each scale stage in place from row
 //            order into the 32-line x 16-byte chunks tcgen05.cp expects
+//            (with two issuers warp 13 does the second issuer's stages)
 //   warp 3   TMEM allocator (and, with two accumulators, the second issuer)
 //   warps 4-11  epilogue: two warps per TMEM lane quarter, each reading half
 //            of the tile's columns with tcgen05.ld (thread = tile row), then
@@ -48,6 +50,7 @@ constexpr int BKB = 128;           // bytes of K per stage per row (256 FP4)
 constexpr int STAGES = 4;
 constexpr int kEpiWarps = 8;
 constexpr int kProducer2Warp = 4 + kEpiWarps;   // the second TMA producer (two MMA issuers)
+constexpr int kTransposer2Warp = 5 + kEpiWarps; // the second scale transposer (two MMA issuers)
 constexpr int A_BYTES = BM * BKB;  // 16 KB
 constexpr int kTmemCols = 512;
 constexpr int kColAcc = 0;
@@ -86,7 +89,7 @@ struct Cfg {
     static constexpr int SF_STAGES = 2 * NISS;
     static constexpr int COL_SFA = NACC * TBN;
     static_assert(COL_SFA + NISS * SF_COLS <= 512, "TMEM columns");
-    static constexpr int THREADS = 32 * (4 + kEpiWarps + (NISS == 2 ? 1 : 0));
+    static constexpr int THREADS = 32 * (4 + kEpiWarps + (NISS == 2 ? 2 : 0));
     static constexpr int SF_ROW = KPS * WPS * 4;                     // scale bytes per row per scale stage
     static constexpr int SFA_BYTES = BM * SF_ROW;                    // one scale stage of A
     static constexpr int SFB_BYTES = 256 * SF_ROW;                   // one scale stage of W (two 128-row groups)
@@ -717,31 +720,31 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUt
             mbar_wait(smem_u32(&drain[pi]), 0, &never);
         }
         __syncwarp();
-    } else if (warp == 2) {
-        // ================= scale transposer =================
-        // scale stages in the order the issuers take them: a group's members
-        // interleaved, scale stage by scale stage
-        uint32_t ls[NISS] = {};
+    } else if (warp == 2 || (NISS == 2 && warp == kTransposer2Warp)) {
+        // ================= scale transposer(s) =================
+        // one per tile group member (warp 2, and warp 13 with two issuers),
+        // taking that member's scale stages in order, so that neither
+        // issuer's scales wait behind the other's (with one warp for both,
+        // the issuers waited 14-23% of their time for transposed scales)
+        const int m = (warp == 2) ? 0 : 1;
+        uint32_t ls = 0;
         bool ok = true;
         for (int64_t j0 = 0; ok; j0 += NISS) {
             const int64_t t0 = tile0 + j0 * tstride;
             if (t0 >= ntiles) break;
             const int gsz = (NISS == 2 && t0 + tstride < ntiles) ? 2 : 1;
+            if (m >= gsz) break;                                    // the CTA's last group has one member
             for (int pr = 0; pr < nsfs && ok; ++pr) {
-#pragma unroll
-                for (int m = 0; m < NISS; ++m) {
-                    if (m >= gsz) break;
-                    const int r = NISS * (int)(ls[m] % SPM) + m;
-                    bool w_ok = true;
-                    if (lane == 0) w_ok = mbar_wait(smem_u32(&sf_full[r]), (ls[m] / SPM) & 1, abort_flag);
-                    if (!__shfl_sync(0xffffffffu, w_ok ? 1 : 0, 0)) { ok = false; break; }
-                    ++ls[m];
-                    sf_transpose<KPS * C::WPS, 1>(sSFA + r * C::SFA_BYTES, lane);
-                    sf_transpose<KPS * C::WPS, 2>(sSFB + r * C::SFB_BYTES, lane);
-                    fence_proxy_async();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(smem_u32(&sf_ready[r]));
-                }
+                const int r = NISS * (int)(ls % SPM) + m;
+                bool w_ok = true;
+                if (lane == 0) w_ok = mbar_wait(smem_u32(&sf_full[r]), (ls / SPM) & 1, abort_flag);
+                if (!__shfl_sync(0xffffffffu, w_ok ? 1 : 0, 0)) { ok = false; break; }
+                ++ls;
+                sf_transpose<KPS * C::WPS, 1>(sSFA + r * C::SFA_BYTES, lane);
+                sf_transpose<KPS * C::WPS, 2>(sSFB + r * C::SFB_BYTES, lane);
+                fence_proxy_async();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&sf_ready[r]));
             }
         }
     } else if (warp >= 4 && warp < 4 + kEpiWarps) {
