@@ -31,12 +31,12 @@ import numpy as np
 
 L2_BYTES = 126 * 1000 * 1000
 # DRAM bytes (read + write) of one launch of the dominant kernel, from an ncu
-# capture of the kernel as it is now; workloads without one report null.  The
-# prefill GEMM gained its second scale transposer after its last captures
-# (prefill16k stand-in 1.022x, prefill T = 2048 full launch 1.033x of the
-# algorithmic bytes; its loads and stores did not change), so those report null.
-FC1_TRAFFIC = {"prefill16k": (None, "none of the current kernel; profiles/k_gemm_tc_fc1_prof_prefill16k_nvfp4.md "
-                                    "(1.022x, the kernel before its second scale transposer)"),
+# capture of the kernel as it is now; workloads without one report null.
+# prefill16k: the 64-expert stand-in's FC1 launch (990.7 MB against 969.7 MB
+# algorithmic, 1.022x) scaled to the full launch by its algorithmic bytes
+# (3350.2 MB).  prefill: its full-size capture (1.033x) predates the prefill
+# GEMM's second scale transposer, so it reports null.
+FC1_TRAFFIC = {"prefill16k": (3422842407, "profiles/k_gemm_tc_fc1_prof_prefill16k_nvfp4.md (stand-in, scaled)"),
                "prefill": (None, "none of the current kernel; profiles/dram_traffic_k_gemm_tc_prefill_T2048_mxfp4.md "
                                  "(1.033x, the kernel before its second scale transposer)"),
                # the one-launch decode FFN: the decode stand-in's traffic ratio (1.00882) x the algorithmic bytes
