@@ -80,3 +80,25 @@ def test_default_workload_is_the_largest_layer():
     from synth import workloads
     wl = workloads.WORKLOADS[a.workload]
     assert (wl.T, wl.fmt) == (16384, 1)
+
+
+def test_prefill16k_traffic_is_the_scaled_stand_in_capture():
+    """roofline.traffic of the default run = the stand-in FC1 launch's DRAM
+    bytes (ncu: 963,205,376 read + 27,490,560 written, the capture in
+    profiles/k_gemm_tc_fc1_prof_prefill16k_nvfp4.md) scaled by the two launches'
+    algorithmic bytes, each from its own routing (here the oracle's, which the
+    GPU's routing matches bit for bit)"""
+    import oracle
+    import synth
+    from synth import workloads
+    alg = {}
+    for name in ("prof_prefill16k", "prefill16k"):
+        wl = workloads.WORKLOADS[name]
+        idx, _ = oracle.route_topk(synth.logits(wl.T, wl.E, 0, wl.bias_sigma), wl.k)
+        offsets = np.concatenate([[0], np.cumsum(np.bincount(idx.ravel(), minlength=wl.E))]).astype(np.int32)
+        alg[name] = bench.algorithmic(wl, offsets)
+    assert alg["prof_prefill16k"]["touched"] == 51 and alg["prefill16k"]["touched"] == 172
+    assert alg["prof_prefill16k"]["fc1_bytes"] == 969_670_656 and alg["prefill16k"]["fc1_bytes"] == 3_350_200_320
+    measured = 963_205_376 + 27_490_560
+    scaled = round(measured * alg["prefill16k"]["fc1_bytes"] / alg["prof_prefill16k"]["fc1_bytes"])
+    assert bench.FC1_TRAFFIC["prefill16k"][0] == scaled
