@@ -83,11 +83,11 @@ def test_default_workload_is_the_largest_layer():
 
 
 def test_prefill16k_traffic_is_the_scaled_stand_in_capture():
-    """roofline.traffic of the default run = the stand-in FC1 launch's DRAM
-    bytes (ncu: 963,205,376 read + 27,490,560 written, the capture in
-    profiles/k_gemm_tc_fc1_prof_prefill16k_nvfp4.md) scaled by the two launches'
-    algorithmic bytes, each from its own routing (here the oracle's, which the
-    GPU's routing matches bit for bit)"""
+    """roofline.traffic of the default run = the DRAM bytes ncu counted for one
+    FC1 launch of the current kernel on the 64-expert stand-in (963,205,376
+    read + 27,490,560 written) scaled by the two launches' algorithmic bytes,
+    each from its own routing (here the oracle's, which the GPU's routing
+    matches bit for bit)"""
     import oracle
     import synth
     from synth import workloads
